@@ -1,0 +1,156 @@
+"""ctypes binding of the C oracle (test infrastructure only).
+
+Float inputs may be fp32 arrays or bf16 bit patterns (``np.uint16``); both
+are widened to fp64 exactly before the C code sees them ("read inputs at
+their stored precision").
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int64), ("I", ctypes.c_int64),
+                ("E", ctypes.c_int64), ("k", ctypes.c_int64), ("bits", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("act", ctypes.c_int32),
+                ("fusion", ctypes.c_int32), ("normalize", ctypes.c_int32),
+                ("has_fc3", ctypes.c_int32), ("alpha", ctypes.c_double),
+                ("beta", ctypes.c_double), ("limit", ctypes.c_double)]
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        lib.oracle_forward.restype = ctypes.c_int
+        lib.oracle_gated_act.restype = ctypes.c_double
+        lib.oracle_gated_act.argtypes = [ctypes.c_int32] + [ctypes.c_double] * 5
+        lib.oracle_plain_act.restype = ctypes.c_double
+        lib.oracle_plain_act.argtypes = [ctypes.c_int32, ctypes.c_double]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def to_f64(a: Optional[np.ndarray]) -> Optional[np.ndarray]:
+    """Widen stored values to fp64: uint16 arrays are bf16 bit patterns."""
+    if a is None:
+        return None
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray((a.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a, typ):
+    return None if a is None else a.ctypes.data_as(typ)
+
+
+def unpack(packed: np.ndarray, N: int, K: int, bits: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    assert packed.size == N * K * bits // 8
+    q = np.empty((N, K), dtype=np.int32)
+    _load().oracle_unpack(_p(packed, _u8p), ctypes.c_int64(N), ctypes.c_int64(K),
+                          ctypes.c_int32(bits), _p(q, _i32p))
+    return q
+
+
+def dequant(packed: np.ndarray, scales: np.ndarray, N: int, K: int, bits: int,
+            block_size: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    s = to_f64(scales)
+    assert s.size == (N * (K // block_size) if block_size > 0 else N)
+    w = np.empty((N, K), dtype=np.float64)
+    _load().oracle_dequant(_p(packed, _u8p), _p(s, _f64p), ctypes.c_int64(N), ctypes.c_int64(K),
+                           ctypes.c_int32(bits), ctypes.c_int64(block_size), _p(w, _f64p))
+    return w
+
+
+def route(logits: np.ndarray, k: int, normalize: bool):
+    lg = to_f64(logits)
+    T, E = lg.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    _load().oracle_route(_p(lg, _f64p), ctypes.c_int64(T), ctypes.c_int64(E), ctypes.c_int64(k),
+                         ctypes.c_int32(int(normalize)), _p(idx, _i32p), _p(w, _f64p))
+    return idx, w
+
+
+def permute(idx: np.ndarray, E: int):
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    offsets = np.empty(E + 1, dtype=np.int32)
+    perm = np.empty(T * k, dtype=np.int32)
+    inv = np.empty((T, k), dtype=np.int32)
+    _load().oracle_permute(_p(idx, _i32p), ctypes.c_int64(T), ctypes.c_int64(E), ctypes.c_int64(k),
+                           _p(offsets, _i32p), _p(perm, _i32p), _p(inv, _i32p))
+    return offsets, perm, inv
+
+
+def gated_act(act: int, g: float, u: float, alpha: float, beta: float, limit: float) -> float:
+    return float(_load().oracle_gated_act(act, g, u, alpha, beta, limit))
+
+
+def plain_act(act: int, a: float) -> float:
+    return float(_load().oracle_plain_act(act, a))
+
+
+def forward(inp, tokens: Optional[Sequence[int]] = None, want_h: bool = False) -> dict:
+    """Run the whole forward on ``inp`` (an object with the fields of a
+    generated input set: ``cfg``, ``x``, ``logits``, ``fc1_w`` ... ``shared``).
+
+    ``tokens`` restricts the run to a subset of token rows (tokens are
+    independent, so the result equals those rows of the full output).
+    Returns ``y`` [T', H] fp64 (unrounded), ``topk_idx``, ``topk_w`` and,
+    with ``want_h``, ``h`` [T'*k, I].
+    """
+    c = inp.cfg
+    x = to_f64(inp.x)
+    lg = to_f64(inp.logits)
+    sh = to_f64(inp.shared)
+    if tokens is not None:
+        tokens = np.asarray(tokens, dtype=np.int64)
+        x, lg = np.ascontiguousarray(x[tokens]), np.ascontiguousarray(lg[tokens])
+        sh = None if sh is None else np.ascontiguousarray(sh[tokens])
+    T = x.shape[0]
+    cfg = _Cfg(T=T, H=c.H, I=c.I, E=c.E, k=c.k, bits=c.bits, block_size=c.block_size,
+               act=c.act, fusion=c.fusion, normalize=int(c.normalize), has_fc3=int(c.has_fc3),
+               alpha=float(c.alpha), beta=float(c.beta),
+               limit=float(c.limit) if c.limit is not None else math.inf)
+    y = np.empty((T, c.H), dtype=np.float64)
+    idx = np.empty((T, c.k), dtype=np.int32)
+    w = np.empty((T, c.k), dtype=np.float64)
+    h = np.empty((T * c.k, c.I), dtype=np.float64) if want_h else None
+    u8 = lambda a: None if a is None else np.ascontiguousarray(a, dtype=np.uint8)  # noqa: E731
+    f1w, f2w, f3w = u8(inp.fc1_w), u8(inp.fc2_w), u8(inp.fc3_w)
+    f1s, f2s, f3s = to_f64(inp.fc1_s), to_f64(inp.fc2_s), to_f64(inp.fc3_s)
+    f1b, f2b, f3b = to_f64(inp.fc1_b), to_f64(inp.fc2_b), to_f64(inp.fc3_b)
+    rc = _load().oracle_forward(
+        ctypes.byref(cfg), _p(x, _f64p), _p(lg, _f64p),
+        _p(f1w, _u8p), _p(f1s, _f64p), _p(f1b, _f64p),
+        _p(f2w, _u8p), _p(f2s, _f64p), _p(f2b, _f64p),
+        _p(f3w, _u8p), _p(f3s, _f64p), _p(f3b, _f64p),
+        _p(sh, _f64p), _p(y, _f64p), _p(idx, _i32p), _p(w, _f64p), _p(h, _f64p))
+    if rc != 0:
+        raise MemoryError("oracle_forward: allocation failed")
+    out = dict(y=y, topk_idx=idx, topk_w=w)
+    if want_h:
+        out["h"] = h
+    return out

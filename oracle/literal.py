@@ -1,0 +1,137 @@
+"""A second, deliberately literal statement of the whole forward (tiny shapes).
+
+TEST INFRASTRUCTURE ONLY. It exists to cross-check ``qmoe_oracle.c`` by brute
+force: routing enumerates every k-subset of experts, weights are rebuilt
+element by element from their bytes, and every expert is run token by token
+with Python floats (fp64). Use it for T, H, I, E of a few dozen at most.
+
+Definitions followed are the same passages as the C oracle: the "QMoE"
+operator page (layouts, pack_size, block_size, swiglu_fusion, activation
+attributes, k, normalize_routing_weights), the "MoE" page summary (top-k,
+gated FFN, weighted combine), the "QLinearWoQ" summary (x @ dequant(W).T + b)
+and "ClikaRT::nn::QMoEWoQ" forward() (shared_output folds into the combine).
+"""
+from __future__ import annotations
+
+import itertools
+import math
+
+import numpy as np
+
+from .binding import to_f64
+
+
+def _code(byte_row, k, bits):
+    if bits == 8:
+        return int(byte_row[k])
+    b = int(byte_row[k // 2])
+    return b & 15 if k % 2 == 0 else b >> 4
+
+
+def dense_weight(packed, scales, N, K, bits, bs):
+    """[N][K] list of Python floats."""
+    z = 2 ** (bits - 1)
+    W = []
+    for n in range(N):
+        row = []
+        for k in range(K):
+            s = scales[n][k // bs] if bs > 0 else scales[n]
+            row.append((_code(packed[n], k, bits) - z) * float(s))
+        W.append(row)
+    return W
+
+
+def select_experts(logits_row, k):
+    """Brute force: the k-subset with the largest logit sum; among equal sums
+    the lexicographically smallest sorted id tuple. Returned in list order
+    (logit descending, id ascending)."""
+    E = len(logits_row)
+    best, best_sum = None, -math.inf
+    for sub in itertools.combinations(range(E), k):
+        s = sum(logits_row[e] for e in sub)
+        if s > best_sum:
+            best, best_sum = sub, s
+    return sorted(best, key=lambda e: (-logits_row[e], e))
+
+
+def route_weights(logits_row, sel, normalize):
+    m = max(logits_row)
+    ex = [math.exp(v - m) for v in logits_row]
+    p = [v / sum(ex) for v in ex]
+    w = [p[e] for e in sel]
+    if normalize:
+        tot = sum(w)
+        w = [v / tot for v in w]
+    return w
+
+
+def activation(act, g, u, alpha, beta, limit, gated):
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))  # noqa: E731
+    if not gated:
+        a = g
+        return {0: max(a, 0.0), 1: 0.5 * a * (1 + math.erf(a / math.sqrt(2))),
+                2: a * sig(a), 4: a}[act]
+    if act == 3:
+        al = 1.0 if alpha == 0 else alpha
+        if math.isfinite(limit) and limit > 0:
+            g = min(g, limit)
+            u = max(-limit, min(limit, u))
+        return (u + beta) * g * sig(al * g)
+    base = {0: max(g, 0.0), 1: 0.5 * g * (1 + math.erf(g / math.sqrt(2))),
+            2: g * sig(g), 4: g}[act]
+    return base * u
+
+
+def forward(inp):
+    c = inp.cfg
+    x = to_f64(inp.x)
+    lg = to_f64(inp.logits)
+    sh = to_f64(inp.shared)
+    fused = c.fusion in (1, 2)
+    gated = fused or c.has_fc3
+    N1 = (2 if fused else 1) * c.I
+
+    def scl(a):
+        return to_f64(a).tolist()
+
+    def bias(a, e):
+        return [0.0] * 10**6 if a is None else to_f64(a)[e].tolist()
+
+    W1 = [dense_weight(inp.fc1_w[e], scl(inp.fc1_s)[e], N1, c.H, c.bits, c.block_size)
+          for e in range(c.E)]
+    W2 = [dense_weight(inp.fc2_w[e], scl(inp.fc2_s)[e], c.H, c.I, c.bits, c.block_size)
+          for e in range(c.E)]
+    W3 = ([dense_weight(inp.fc3_w[e], scl(inp.fc3_s)[e], c.I, c.H, c.bits, c.block_size)
+           for e in range(c.E)] if c.has_fc3 else None)
+
+    y = np.zeros((c.T, c.H))
+    sels, wts = [], []
+    for t in range(c.T):
+        row = lg[t].tolist()
+        sel = select_experts(row, c.k)
+        w = route_weights(row, sel, c.normalize)
+        sels.append(sel)
+        wts.append(w)
+        xt = x[t].tolist()
+        for j, e in enumerate(sel):
+            b1, b2, b3 = bias(inp.fc1_b, e), bias(inp.fc2_b, e), bias(inp.fc3_b, e)
+            a = [sum(xt[kk] * W1[e][n][kk] for kk in range(c.H)) + b1[n] for n in range(N1)]
+            h = []
+            for i in range(c.I):
+                if not gated:
+                    h.append(activation(c.act, a[i], None, c.alpha, c.beta, c.limit, False))
+                    continue
+                if c.fusion == 1:
+                    g, u = a[2 * i], a[2 * i + 1]
+                elif c.fusion == 2:
+                    g, u = a[i], a[c.I + i]
+                else:
+                    g = a[i]
+                    u = sum(xt[kk] * W3[e][i][kk] for kk in range(c.H)) + b3[i]
+                h.append(activation(c.act, g, u, c.alpha, c.beta, c.limit, True))
+            for m in range(c.H):
+                o = sum(h[i] * W2[e][m][i] for i in range(c.I)) + b2[m]
+                y[t, m] += w[j] * o
+        if sh is not None:
+            y[t] += sh[t]
+    return dict(y=y, topk_idx=np.array(sels, dtype=np.int32), topk_w=np.array(wts))

@@ -1,0 +1,305 @@
+/*
+ * qmoe_oracle.c -- CPU oracle for the weight-only-quantized MoE forward.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file's library. The CUDA path
+ * shares no code, header, table or helper with it.
+ *
+ * It states the plain definition of the operator in fp64:
+ *   - "QMoE" operator page (graiphic.io), input list and attributes: tensor
+ *     layouts, pack_size = 8 / expert_weight_bits along K, per-column or
+ *     per-K-block scales, swiglu_fusion layouts, activation attributes,
+ *     k and normalize_routing_weights;
+ *   - "MoE" page (clika_runtime.nn), class summary: a router picks the top-k
+ *     experts per token, each runs its gated FFN, and the outputs are combined
+ *     under the router weights;
+ *   - "QLinearWoQ" page, class summary: each linear is
+ *     y = x @ dequant(W).T + b;
+ *   - "ClikaRT::nn::QMoEWoQ" page, forward(): [T, H] in, [T, H] out, and the
+ *     optional shared_output folds into the routed combine.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   - codes are unsigned; the zero point is implicit and equals 2^(bits-1);
+ *   - with 4 bits, even k sits in the low nibble of byte k/2;
+ *   - selection is by raw logit, ties go to the lower expert id, the list is
+ *     ordered by (logit descending, id ascending);
+ *   - weights are the softmax over all E experts restricted to the selection,
+ *     renormalised over the k when asked;
+ *   - swiglu: g' = min(g, L), u' = clamp(u, -L, L),
+ *     h = (u' + beta) * g' * sigmoid(alpha * g'); alpha == 0 means 1; a limit
+ *     that is <= 0 or not finite means no clamp;
+ *   - the expert output includes its fc2 bias and is then weighted;
+ *   - fusion 1: gate = even rows, up = odd rows; fusion 2: gate = first I
+ *     rows, up = last I rows; fusion 0 with fc3: gate = fc1, up = fc3.
+ *
+ * Every sum is a serial fp64 loop in index order, so the result does not
+ * depend on the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { O_RELU = 0, O_GELU = 1, O_SILU = 2, O_SWIGLU = 3, O_IDENTITY = 4 };
+
+typedef struct oracle_cfg {
+    int64_t T, H, I, E, k;
+    int32_t bits;        /* 4 or 8 */
+    int32_t block_size;  /* 0 = one scale per output row */
+    int32_t act;         /* O_* above */
+    int32_t fusion;      /* 0, 1, 2 */
+    int32_t normalize;
+    int32_t has_fc3;
+    double alpha, beta, limit;
+} oracle_cfg;
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Code of element (n, k) of a packed [N, K/pack] stack (QMoE page, weights). */
+static int32_t code_at(const uint8_t* packed, int64_t K, int bits, int64_t n, int64_t k) {
+    if (bits == 8) return packed[n * K + k];
+    const uint8_t byte = packed[n * (K / 2) + k / 2];
+    return (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+}
+
+void oracle_unpack(const uint8_t* packed, int64_t N, int64_t K, int32_t bits, int32_t* q) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) q[n * K + k] = code_at(packed, K, bits, n, k);
+}
+
+/* One dequantised row: w[k] = (q[n,k] - 2^(bits-1)) * s, s from the block of k
+ * (QMoE page, fcX_scales and block_size). */
+static void dequant_row(const uint8_t* packed, const double* scales, int64_t K, int bits,
+                        int64_t bs, int64_t n, double* w) {
+    const int32_t z = 1 << (bits - 1);
+    for (int64_t k = 0; k < K; ++k) {
+        const double s = bs > 0 ? scales[n * (K / bs) + k / bs] : scales[n];
+        w[k] = (double)(code_at(packed, K, bits, n, k) - z) * s;
+    }
+}
+
+void oracle_dequant(const uint8_t* packed, const double* scales, int64_t N, int64_t K,
+                    int32_t bits, int64_t bs, double* w) {
+    for (int64_t n = 0; n < N; ++n) dequant_row(packed, scales, K, bits, bs, n, w + n * K);
+}
+
+/* Routing ("MoE" page summary; QMoE page attributes k and
+ * normalize_routing_weights). */
+void oracle_route(const double* logits, int64_t T, int64_t E, int64_t k, int32_t normalize,
+                  int32_t* idx, double* w) {
+    char* taken = (char*)malloc((size_t)E);
+    double* p = (double*)malloc(sizeof(double) * (size_t)E);
+    for (int64_t t = 0; t < T; ++t) {
+        const double* l = logits + t * E;
+        memset(taken, 0, (size_t)E);
+        for (int64_t j = 0; j < k; ++j) {
+            int64_t best = -1;
+            for (int64_t e = 0; e < E; ++e)
+                if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+            taken[best] = 1;
+            idx[t * k + j] = (int32_t)best;
+        }
+        double mx = l[0];
+        for (int64_t e = 1; e < E; ++e)
+            if (l[e] > mx) mx = l[e];
+        double z = 0.0;
+        for (int64_t e = 0; e < E; ++e) z += exp(l[e] - mx);
+        for (int64_t e = 0; e < E; ++e) p[e] = exp(l[e] - mx) / z;
+        double sel = 0.0;
+        for (int64_t j = 0; j < k; ++j) sel += p[idx[t * k + j]];
+        for (int64_t j = 0; j < k; ++j)
+            w[t * k + j] = normalize ? p[idx[t * k + j]] / sel : p[idx[t * k + j]];
+    }
+    free(taken);
+    free(p);
+}
+
+/* Token -> expert permutation: segments in expert order, tokens ascending
+ * inside a segment. offsets[E+1], perm_tok[T*k], inv[T*k]. */
+void oracle_permute(const int32_t* idx, int64_t T, int64_t E, int64_t k, int32_t* offsets,
+                    int32_t* perm_tok, int32_t* inv) {
+    int64_t pos = 0;
+    for (int64_t e = 0; e < E; ++e) {
+        offsets[e] = (int32_t)pos;
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t j = 0; j < k; ++j)
+                if (idx[t * k + j] == e) {
+                    perm_tok[pos] = (int32_t)t;
+                    inv[t * k + j] = (int32_t)pos;
+                    ++pos;
+                }
+    }
+    offsets[E] = (int32_t)pos;
+}
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+static double plain_act(int act, double a) {
+    switch (act) {
+        case O_RELU: return a > 0.0 ? a : 0.0;
+        case O_GELU: return 0.5 * a * (1.0 + erf(a / sqrt(2.0)));
+        case O_SILU: return a * sigmoid(a);
+        default: return a; /* identity */
+    }
+}
+
+/* Gated activation h = act(gate, up) (QMoE page: activation_type,
+ * activation_alpha, activation_beta, swiglu_limit). */
+double oracle_gated_act(int32_t act, double g, double u, double alpha, double beta, double limit) {
+    if (act == O_SWIGLU) {
+        const double a = (alpha == 0.0 || !isfinite(alpha)) ? 1.0 : alpha;
+        if (isfinite(limit) && limit > 0.0) {
+            g = g < limit ? g : limit;
+            u = u < -limit ? -limit : (u > limit ? limit : u);
+        }
+        return (u + beta) * g * sigmoid(a * g);
+    }
+    return plain_act(act, g) * u;
+}
+
+double oracle_plain_act(int32_t act, double a) { return plain_act(act, a); }
+
+/*
+ * The whole forward. Float inputs arrive as fp64 arrays holding the stored
+ * values exactly. Outputs: y[T,H] (fp64, unrounded), topk_idx[T,k],
+ * topk_w[T,k], and optionally h[T*k, I] (row t*k+j is the hidden activation of
+ * token t under its j-th expert).
+ */
+int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
+                   const uint8_t* fc1_w, const double* fc1_s, const double* fc1_b,
+                   const uint8_t* fc2_w, const double* fc2_s, const double* fc2_b,
+                   const uint8_t* fc3_w, const double* fc3_s, const double* fc3_b,
+                   const double* shared, double* y, int32_t* topk_idx, double* topk_w,
+                   double* h_out) {
+    const int64_t T = c->T, H = c->H, I = c->I, E = c->E, k = c->k, R = T * k;
+    const int fused = (c->fusion == 1 || c->fusion == 2);
+    const int gated = fused || c->has_fc3;
+    const int64_t N1 = (fused ? 2 : 1) * I;
+    const int64_t bs = c->block_size;
+    const int bits = c->bits;
+    const int64_t pk1 = H * bits / 8, pk2 = I * bits / 8;
+    const int64_t sc1 = bs > 0 ? H / bs : 1, sc2 = bs > 0 ? I / bs : 1;
+
+    oracle_route(logits, T, E, k, c->normalize, topk_idx, topk_w);
+
+    double* a1 = (double*)calloc((size_t)(R * N1), sizeof(double)); /* fc1 pre-activation */
+    double* a3 = c->has_fc3 ? (double*)calloc((size_t)(R * I), sizeof(double)) : NULL;
+    double* h = (double*)calloc((size_t)(R * I), sizeof(double));
+    double* o = (double*)calloc((size_t)(R * H), sizeof(double));
+    int64_t* rows = (int64_t*)malloc(sizeof(int64_t) * (size_t)(R > 0 ? R : 1));
+    if (!a1 || !h || !o || !rows || (c->has_fc3 && !a3)) return -1;
+
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t m = 0; /* routed (t, j) pairs of expert e, as r = t*k + j */
+        for (int64_t r = 0; r < R; ++r)
+            if (topk_idx[r] == e) rows[m++] = r;
+        if (m == 0) continue;
+
+        /* FC1 (and FC3): a[r, n] = sum_k x[t, k] * W[n, k] + b[n] */
+        const uint8_t* w1 = fc1_w + e * N1 * pk1;
+        const double* s1 = fc1_s + e * N1 * sc1;
+#pragma omp parallel
+        {
+            double* wrow = (double*)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(static)
+            for (int64_t n = 0; n < N1; ++n) {
+                dequant_row(w1, s1, H, bits, bs, n, wrow);
+                for (int64_t i = 0; i < m; ++i) {
+                    const int64_t r = rows[i], t = r / k;
+                    double acc = 0.0;
+                    for (int64_t kk = 0; kk < H; ++kk) acc += x[t * H + kk] * wrow[kk];
+                    if (fc1_b) acc += fc1_b[e * N1 + n];
+                    a1[r * N1 + n] = acc;
+                }
+            }
+            if (c->has_fc3) {
+                const uint8_t* w3 = fc3_w + e * I * pk1;
+                const double* s3 = fc3_s + e * I * sc1;
+#pragma omp for schedule(static)
+                for (int64_t n = 0; n < I; ++n) {
+                    dequant_row(w3, s3, H, bits, bs, n, wrow);
+                    for (int64_t i = 0; i < m; ++i) {
+                        const int64_t r = rows[i], t = r / k;
+                        double acc = 0.0;
+                        for (int64_t kk = 0; kk < H; ++kk) acc += x[t * H + kk] * wrow[kk];
+                        if (fc3_b) acc += fc3_b[e * I + n];
+                        a3[r * I + n] = acc;
+                    }
+                }
+            }
+            free(wrow);
+        }
+
+        /* activation: split gate / up by the fusion layout */
+        for (int64_t i = 0; i < m; ++i) {
+            const int64_t r = rows[i];
+            for (int64_t n = 0; n < I; ++n) {
+                double v;
+                if (!gated) {
+                    v = plain_act(c->act, a1[r * N1 + n]);
+                } else {
+                    double g, u;
+                    if (c->fusion == 1) {
+                        g = a1[r * N1 + 2 * n];
+                        u = a1[r * N1 + 2 * n + 1];
+                    } else if (c->fusion == 2) {
+                        g = a1[r * N1 + n];
+                        u = a1[r * N1 + I + n];
+                    } else {
+                        g = a1[r * N1 + n];
+                        u = a3[r * I + n];
+                    }
+                    v = oracle_gated_act(c->act, g, u, c->alpha, c->beta, c->limit);
+                }
+                h[r * I + n] = v;
+            }
+        }
+
+        /* FC2: o[r, m] = sum_i h[r, i] * W2[m, i] + b2[m] */
+        const uint8_t* w2 = fc2_w + e * H * pk2;
+        const double* s2 = fc2_s + e * H * sc2;
+#pragma omp parallel
+        {
+            double* wrow = (double*)malloc(sizeof(double) * (size_t)I);
+#pragma omp for schedule(static)
+            for (int64_t n = 0; n < H; ++n) {
+                dequant_row(w2, s2, I, bits, bs, n, wrow);
+                for (int64_t i = 0; i < m; ++i) {
+                    const int64_t r = rows[i];
+                    double acc = 0.0;
+                    for (int64_t kk = 0; kk < I; ++kk) acc += h[r * I + kk] * wrow[kk];
+                    if (fc2_b) acc += fc2_b[e * H + n];
+                    o[r * H + n] = acc;
+                }
+            }
+            free(wrow);
+        }
+    }
+
+    /* combine: y[t] = sum_j w[t, j] * o[t*k + j] + shared[t], j in list order */
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t n = 0; n < H; ++n) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < k; ++j) acc += topk_w[t * k + j] * o[(t * k + j) * H + n];
+            if (shared) acc += shared[t * H + n];
+            y[t * H + n] = acc;
+        }
+
+    if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)(R * I));
+    free(a1);
+    free(a3);
+    free(h);
+    free(o);
+    free(rows);
+    return 0;
+}
