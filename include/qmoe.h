@@ -1,0 +1,238 @@
+/*
+ * qmoe.h -- C ABI of the B200 (sm_100a) weight-only-quantized MoE forward.
+ *
+ * The operator is the QMoE node defined on the "QMoE" operator page
+ * (graiphic.io: inputs input, router_probs, fc1/fc2/fc3 expert weights,
+ * scales and biases; attributes activation_alpha, activation_beta,
+ * activation_type, block_size, expert_weight_bits, k,
+ * normalize_routing_weights, swiglu_fusion, swiglu_limit, use_sparse_mixer),
+ * with the module lifecycle of "ClikaRT::nn::QMoEWoQ" (make(), set_weights(),
+ * forward(), ~QMoEWoQ()). Expert weights stay packed as 4- or 8-bit integers
+ * and are decoded block by block inside the GEMM dot ("ClikaRT::nn::QMoEWoQ",
+ * class description); no dense copy of any weight is ever made.
+ *
+ * Conventions for every call below
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise, and are
+ *     borrowed for the duration of the call (or of the stream work it
+ *     enqueues, for qmoe_forward).
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.
+ *   - No call throws; each returns a qmoe_status. The handle keeps the text of
+ *     its last error (qmoe_last_error).
+ *   - Packed weight layout is the QMoE page's: a [E, N, K/pack] uint8 stack,
+ *     pack = 8/expert_weight_bits along K. Codes are unsigned with an implicit
+ *     zero point 2^(bits-1); with 4 bits the even k of a pair sits in the low
+ *     nibble. (The page gives no zero-point input; this is the reading taken.)
+ */
+#ifndef QMOE_H
+#define QMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QMOE_API __attribute__((visibility("default")))
+#else
+#define QMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qmoe_status {
+    QMOE_OK = 0,
+    /* Shape, dtype or geometry mismatch; a bias without its declared slot;
+     * block_size not a power of two >= 16 or not dividing H and I; bits not
+     * 4 or 8; k outside [1, E]; a NULL required pointer; a workspace too small
+     * or not 256-byte aligned ("ClikaRT::nn::QMoEWoQ", set_weights() and
+     * forward(): Error on geometry or shape mismatch). */
+    QMOE_INVALID_ARGUMENT = 1,
+    /* forward() before set_weights() bound the required slots (the "still-fake
+     * slot" error of "ClikaRT::nn::QMoEWoQ", forward() and initialize_impl()). */
+    QMOE_NOT_BOUND = 2,
+    /* Valid per the pages but not built here: use_sparse_mixer, E > 256,
+     * H or I not a multiple of 64. */
+    QMOE_UNSUPPORTED = 3,
+    QMOE_CUDA_ERROR = 4,
+    /* A bounded device-side wait gave up (see qmoe_read_device_status). */
+    QMOE_TIMEOUT = 5,
+    QMOE_OUT_OF_MEMORY = 6
+} qmoe_status;
+
+/* activation_type, in the order the QMoE page lists them. */
+enum {
+    QMOE_ACT_RELU = 0,
+    QMOE_ACT_GELU = 1, /* erf form */
+    QMOE_ACT_SILU = 2,
+    QMOE_ACT_SWIGLU = 3,
+    QMOE_ACT_IDENTITY = 4
+};
+
+enum { QMOE_DTYPE_F32 = 0, QMOE_DTYPE_BF16 = 1 };
+
+/*
+ * Operator attributes ("QMoE" page attribute list; "ClikaRT::nn::QMoEWoQ",
+ * make(): the four counts and the bias flags).
+ *
+ * Gating: the FFN is gated (h = act(gate) * up, or swiglu) when
+ * swiglu_fusion is 1 (rows 2i = gate, 2i+1 = up) or 2 (rows [0, I) = gate,
+ * [I, 2I) = up), or when has_fc3 is set with swiglu_fusion 0 (fc1 = gate,
+ * fc3 = up). Otherwise h = act(fc1 x + b1) and swiglu is invalid.
+ *
+ * swiglu: g' = min(g, L), u' = clamp(u, -L, L),
+ *         h = (u' + beta) * g' * sigmoid(alpha * g').
+ * activation_alpha == 0 reads as 1 (the page's default 0 would not be
+ * SwiGLU); swiglu_limit <= 0 or non-finite means no clamp (the page states the
+ * limit is infinite when not provided).
+ */
+typedef struct qmoe_config {
+    int64_t num_experts;          /* E, 1..256 */
+    int64_t hidden_size;          /* H, multiple of 64 */
+    int64_t inter_size;           /* I, multiple of 64 */
+    int64_t k;                    /* experts per token, 1..E */
+    int32_t expert_weight_bits;   /* 4 or 8 */
+    int32_t block_size;           /* 0 = one scale per output row; else power of two >= 16 */
+    int32_t activation_type;      /* QMOE_ACT_* */
+    int32_t swiglu_fusion;        /* 0, 1, 2 */
+    float activation_alpha;
+    float activation_beta;
+    float swiglu_limit;
+    int32_t normalize_routing_weights; /* renormalise the k weights to sum to 1 */
+    int32_t act_dtype;            /* dtype of x, router_logits, shared_output, biases and y */
+    int32_t scale_dtype;          /* dtype of fc1/fc2/fc3 scales */
+    int32_t has_fc1_bias;
+    int32_t has_fc2_bias;
+    int32_t has_fc3;
+    int32_t has_fc3_bias;
+    int32_t use_sparse_mixer;     /* must be 0 */
+    int32_t reserved;             /* must be 0 */
+} qmoe_config;
+
+typedef struct qmoe_handle qmoe_handle;
+
+/*
+ * qmoe_create -- "ClikaRT::nn::QMoEWoQ", make(): validate the attributes and
+ * declare storage-free weight slots. Allocates host memory only; touches no
+ * GPU. On success *out owns a handle that qmoe_destroy releases.
+ */
+QMOE_API qmoe_status qmoe_create(const qmoe_config* cfg, qmoe_handle** out);
+
+/*
+ * qmoe_set_weights -- "ClikaRT::nn::QMoEWoQ", set_weights() followed by the
+ * one-time pack of initialize_impl().
+ *
+ *   fc1_w  [E, N1, H*bits/8] uint8, N1 = 2I if swiglu_fusion is 1 or 2, else I
+ *   fc1_s  [E, N1, H/block_size] or [E, N1] (block_size 0), scale_dtype
+ *   fc1_b  [E, N1] act_dtype; required iff has_fc1_bias, else must be NULL
+ *   fc2_w  [E, H, I*bits/8] uint8
+ *   fc2_s  [E, H, I/block_size] or [E, H]
+ *   fc2_b  [E, H]; required iff has_fc2_bias
+ *   fc3_w  [E, I, H*bits/8], fc3_s like fc1_s with I rows; required iff has_fc3
+ *   fc3_b  [E, I]; required iff has_fc3_bias
+ *
+ * All pointers are device pointers. The call re-lays the packed bytes into the
+ * kernels' tile order in handle-owned device memory of the same size (the
+ * weights stay quantized; this copy is the one resident copy), waits for that
+ * work on `stream`, and returns; the caller may then free its buffers. A
+ * second call drops the previous pack and packs again.
+ */
+QMOE_API qmoe_status qmoe_set_weights(qmoe_handle* h,
+                             const void* fc1_w, const void* fc1_s, const void* fc1_b,
+                             const void* fc2_w, const void* fc2_s, const void* fc2_b,
+                             const void* fc3_w, const void* fc3_s, const void* fc3_b,
+                             void* stream);
+
+/*
+ * qmoe_workspace_size -- bytes of device scratch that qmoe_forward needs for
+ * T tokens (routing lists, permutation, hidden activations, partial sums).
+ * Returns 0 for a NULL handle or T < 0.
+ */
+QMOE_API size_t qmoe_workspace_size(const qmoe_handle* h, int64_t T);
+
+/*
+ * qmoe_forward -- "ClikaRT::nn::QMoEWoQ", forward(): one MoE step.
+ *
+ *   x              [T, H] act_dtype
+ *   router_logits  [T, E] act_dtype (logits; softmax is applied inside)
+ *   shared_output  [T, H] act_dtype or NULL (folded into the combine)
+ *   y              [T, H] act_dtype (written)
+ *   workspace      >= qmoe_workspace_size(h, T) bytes, 256-byte aligned,
+ *                  owned by the caller; contents on entry are ignored
+ *
+ * Enqueues all work on `stream` and returns without waiting; it never
+ * synchronises the host. The handle is only read, so concurrent calls on
+ * different streams with different workspaces are safe. T == 0 is a no-op.
+ * A 3-D [B, S, H] input is passed as T = B*S.
+ */
+QMOE_API qmoe_status qmoe_forward(const qmoe_handle* h, int64_t T, const void* x, const void* router_logits,
+                         const void* shared_output, void* y, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * qmoe_forward_profiled -- qmoe_forward that also records CUDA events on
+ * `stream` around its kernels: events[i] just before launch i and
+ * events[n_events - 1] after the last launch. `events` holds cudaEvent_t
+ * handles created by the caller with timing enabled; n_events must equal
+ * qmoe_launches_for(h, T) + 1. The kernels and their order are the same as
+ * qmoe_forward's, so elapsed times between consecutive events are the
+ * per-kernel device times of a normal forward.
+ */
+QMOE_API qmoe_status qmoe_forward_profiled(const qmoe_handle* h, int64_t T, const void* x,
+                                           const void* router_logits, const void* shared_output,
+                                           void* y, void* workspace, size_t workspace_bytes,
+                                           void* stream, void* const* events, int32_t n_events);
+
+/*
+ * qmoe_debug_routing -- copy the routing and permutation of the last forward
+ * that used `workspace` into caller DEVICE buffers (test support; enqueued on
+ * `stream`). Any output pointer may be NULL to skip it.
+ *   topk_idx [T, k] int32   selected experts, (logit desc, id asc) order
+ *   topk_w   [T, k] float   router weights
+ *   offsets  [E + 1] int32  segment starts; offsets[E] = T*k
+ *   perm_tok [T*k] int32    token of each permuted row
+ *   inv      [T, k] int32   permuted row of (token, slot)
+ */
+QMOE_API qmoe_status qmoe_debug_routing(const qmoe_handle* h, int64_t T, const void* workspace,
+                               int32_t* topk_idx, float* topk_w, int32_t* offsets,
+                               int32_t* perm_tok, int32_t* inv, void* stream);
+
+/*
+ * qmoe_debug_hidden -- copy the hidden activations h [T*k, I] (permuted row
+ * order, act_dtype) of the last forward that used `workspace` into a caller
+ * DEVICE buffer (test support; enqueued on `stream`).
+ */
+QMOE_API qmoe_status qmoe_debug_hidden(const qmoe_handle* h, int64_t T, const void* workspace,
+                              void* hidden, void* stream);
+
+/*
+ * qmoe_read_device_status -- wait for `stream`, then read the device-side
+ * status word of `workspace` (QMOE_OK or QMOE_TIMEOUT when a bounded device
+ * wait gave up in the last forward that used it).
+ */
+QMOE_API qmoe_status qmoe_read_device_status(const qmoe_handle* h, const void* workspace, void* stream);
+
+/* qmoe_destroy -- "ClikaRT::nn::QMoEWoQ", ~QMoEWoQ(): release the packed
+ * weights and the handle. NULL is a no-op. */
+QMOE_API void qmoe_destroy(qmoe_handle* h);
+
+/* Static text for a status code. */
+QMOE_API const char* qmoe_status_string(qmoe_status s);
+
+/* Text of the handle's last error ("" if none); valid until the next call on
+ * the handle. */
+QMOE_API const char* qmoe_last_error(const qmoe_handle* h);
+
+/* The forward path qmoe_forward takes for T tokens: 0 = fp32 SIMT path,
+ * 1 = weight-streaming decode path (mma.sync), 2 = tcgen05 grouped GEMM.
+ * -1 for a NULL handle. */
+QMOE_API int32_t qmoe_path_for(const qmoe_handle* h, int64_t T);
+
+/* Number of kernel launches qmoe_forward enqueues for T tokens. */
+QMOE_API int32_t qmoe_launches_for(const qmoe_handle* h, int64_t T);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMOE_H */

@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every symbol that include/qmoe.h declares, and rejects bad configurations
+and calls before touching the device."""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from weight_only_quantized_warp_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def q():
+    libbuild.build()
+    from weight_only_quantized_warp_b200 import qmoe
+    return qmoe
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "qmoe.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"QMOE_API\s+[\w\s\*]+?\b(qmoe_\w+)\s*\(", text)))
+
+
+def test_header_declares_every_binding_name(q):
+    assert _declared() == sorted(q.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(q):
+    lib = ctypes.CDLL(q.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_config_struct_layout(q):
+    assert ctypes.sizeof(q.qmoe_config) == 96
+    assert q.qmoe_config.expert_weight_bits.offset == 32
+    assert q.qmoe_config.activation_alpha.offset == 48
+    assert q.qmoe_config.reserved.offset == 92
+
+
+def _cfg(q, **kw):
+    base = dict(num_experts=8, hidden_size=256, inter_size=512, k=2, expert_weight_bits=4,
+                block_size=64, activation_type=q.ACT_SWIGLU, swiglu_fusion=2,
+                activation_alpha=0.0, activation_beta=0.0, swiglu_limit=math.inf,
+                normalize_routing_weights=1, act_dtype=q.DTYPE_BF16, scale_dtype=q.DTYPE_BF16)
+    base.update(kw)
+    return q.qmoe_config(**base)
+
+
+BAD = [
+    (dict(k=0), 1), (dict(k=9), 1), (dict(expert_weight_bits=3), 1), (dict(expert_weight_bits=0), 1),
+    (dict(block_size=8), 1), (dict(block_size=48), 1), (dict(block_size=512), 1),
+    (dict(activation_type=7), 1), (dict(swiglu_fusion=3), 1),
+    (dict(swiglu_fusion=0, activation_type=3), 1),              # swiglu without a gate/up pair
+    (dict(swiglu_fusion=1, has_fc3=1), 1),                      # fc3 only when unfused
+    (dict(has_fc3_bias=1), 1),                                  # bias without its slot
+    (dict(act_dtype=5), 1), (dict(scale_dtype=2), 1), (dict(reserved=1), 1),
+    (dict(num_experts=0), 1), (dict(hidden_size=0), 1),
+    (dict(use_sparse_mixer=1), 3),                              # valid per the page, not built
+    (dict(num_experts=512, k=2), 3),
+    (dict(hidden_size=96, block_size=32), 3),                   # not a multiple of 64
+]
+
+
+@pytest.mark.parametrize("kw,status", BAD, ids=[str(i) for i in range(len(BAD))])
+def test_create_rejects(q, kw, status):
+    h = ctypes.c_void_p()
+    assert q.lib.qmoe_create(ctypes.byref(_cfg(q, **kw)), ctypes.byref(h)) == status
+    assert not h.value
+
+
+def test_create_accepts_and_plans_without_gpu(q):
+    h = q.qmoe_create(_cfg(q))
+    try:
+        assert q.qmoe_workspace_size(h, 0) > 0
+        ws8 = q.qmoe_workspace_size(h, 8)
+        assert ws8 > q.qmoe_workspace_size(h, 1) and ws8 % 256 == 0
+        assert q.qmoe_workspace_size(h, -1) == 0
+        assert q.qmoe_path_for(h, 8) == q.PATH_DECODE
+        assert q.qmoe_launches_for(h, 8) == 5
+        assert q.qmoe_launches_for(h, 0) == 0
+    finally:
+        q.qmoe_destroy(h)
+    hf = q.qmoe_create(_cfg(q, act_dtype=q.DTYPE_F32, scale_dtype=q.DTYPE_F32))
+    assert q.qmoe_path_for(hf, 8) == q.PATH_SIMT
+    q.qmoe_destroy(hf)
+    q.qmoe_destroy(None)  # no-op
+
+
+def test_forward_before_set_weights_is_not_bound(q):
+    h = q.qmoe_create(_cfg(q))
+    try:
+        st = q.lib.qmoe_forward(h, 4, 16, 16, None, 16, 256, 1 << 20, None)
+        assert st == q.QMOE_NOT_BOUND
+        assert b"set_weights" in q.lib.qmoe_last_error(h)
+    finally:
+        q.qmoe_destroy(h)
+
+
+def test_set_weights_argument_errors_precede_device_work(q):
+    h = q.qmoe_create(_cfg(q, has_fc1_bias=1))
+    try:
+        a = 256  # any non-null address; validation fails before it is used
+        # missing required slot
+        assert q.lib.qmoe_set_weights(h, None, a, a, a, a, None, None, None, None, None) == 1
+        # declared fc1 bias missing
+        assert q.lib.qmoe_set_weights(h, a, a, None, a, a, None, None, None, None, None) == 1
+        # fc2 bias given without its declared slot
+        assert q.lib.qmoe_set_weights(h, a, a, a, a, a, a, None, None, None, None) == 1
+        # fc3 given without has_fc3
+        assert q.lib.qmoe_set_weights(h, a, a, a, a, a, None, a, a, None, None) == 1
+        assert b"bias" in q.lib.qmoe_last_error(h) or b"fc3" in q.lib.qmoe_last_error(h)
+    finally:
+        q.qmoe_destroy(h)
+
+
+def test_status_strings(q):
+    for s, name in [(0, b"QMOE_OK"), (1, b"QMOE_INVALID_ARGUMENT"), (2, b"QMOE_NOT_BOUND"),
+                    (3, b"QMOE_UNSUPPORTED"), (4, b"QMOE_CUDA_ERROR"), (5, b"QMOE_TIMEOUT"),
+                    (6, b"QMOE_OUT_OF_MEMORY")]:
+        assert q.lib.qmoe_status_string(s) == name

@@ -1,0 +1,163 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Routing indices, the permutation (offsets, permuted token list, inverse) are
+compared bit for bit; router weights within a few fp32 ulp; the hidden
+activations h and the output y within max-relative error 1e-2 (bf16
+activations, fp32 accumulation) or 1e-4 (fp32 activations).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+
+from weight_only_quantized_warp_b200 import inputs as gen
+
+from gpu_helpers import check_full, check_routing, check_sampled, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _cfg(**kw):
+    base = dict(T=24, H=320, I=192, E=8, k=2, bits=4, block_size=64, act=gen.ACT_SWIGLU, fusion=2,
+                normalize=True, act_dtype=gen.DT_BF16, scale_dtype=gen.DT_BF16)
+    base.update(kw)
+    return gen.MoEConfig(**base)
+
+
+def test_tiny_config_fp32(cuda_device):
+    cfg, seed, kw = gen.tiny()
+    inp = gen.make_inputs(cfg, seed, **kw)
+    g = run_gpu(inp)
+    assert g.path == 0
+    check_full(inp, g)
+
+
+# Small shapes that span several row tiles, k-groups and CTAs, with ragged
+# tails (row tiles not a multiple of 8 warps; segments not a multiple of 8).
+CASES = {
+    "int4_bs64_fusion2": dict(),
+    "int4_bs128_fusion1": dict(H=384, I=640, block_size=128, fusion=1),
+    "int4_bs32_swiglu_clamp_bias": dict(block_size=32, fusion=1, alpha=1.702, beta=1.0, limit=7.0,
+                                        has_fc1_bias=True, has_fc2_bias=True),
+    "int4_bs16": dict(block_size=16),
+    "int4_percol": dict(block_size=0),
+    "int8_bs128": dict(H=384, I=640, bits=8, block_size=128),
+    "int8_bs32": dict(bits=8, block_size=32),
+    "int8_bs16": dict(bits=8, block_size=16),
+    "int8_percol_fc3_silu_shared": dict(bits=8, block_size=0, fusion=0, has_fc3=True, act=gen.ACT_SILU,
+                                        normalize=False, has_shared=True),
+    "fc3_with_biases": dict(fusion=0, has_fc3=True, act=gen.ACT_SWIGLU, has_fc1_bias=True,
+                            has_fc3_bias=True, has_fc2_bias=True),
+    "plain_relu": dict(fusion=0, act=gen.ACT_RELU, has_fc1_bias=True),
+    "plain_gelu": dict(fusion=0, act=gen.ACT_GELU),
+    "plain_identity": dict(fusion=0, act=gen.ACT_IDENTITY),
+    "gated_gelu": dict(fusion=1, act=gen.ACT_GELU),
+    "f32_scales_bf16_acts_bs64": dict(scale_dtype=gen.DT_F32),
+    "f32_scales_bf16_acts_bs16": dict(scale_dtype=gen.DT_F32, block_size=16),
+    "f32_scales_int8_bs16": dict(scale_dtype=gen.DT_F32, bits=8, block_size=16),
+    "many_tokens_several_passes": dict(T=200, E=4, k=2),
+    "e64_k6": dict(T=40, E=64, k=6, bits=8, block_size=0, fusion=0, has_fc3=True,
+                   act=gen.ACT_SILU, normalize=False),
+    "k_equals_E": dict(T=9, E=4, k=4),
+    "t1": dict(T=1),
+    "fp32_acts_int8": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, bits=8, block_size=32,
+                           has_fc1_bias=True, has_fc2_bias=True, has_shared=True),
+    "fp32_acts_percol_fc3": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_BF16, block_size=0,
+                                 fusion=0, has_fc3=True, act=gen.ACT_SILU),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_parity_small(cuda_device, name):
+    cfg = _cfg(**CASES[name])
+    inp = gen.make_inputs(cfg, seed=100 + list(CASES).index(name), bias_std=0.1)
+    g = run_gpu(inp)
+    check_full(inp, g)
+
+
+def test_all_tokens_to_one_expert_and_empty_experts(cuda_device):
+    cfg = _cfg(T=37, k=1)
+    inp = gen.make_inputs(cfg, seed=5)
+    lg = np.zeros((cfg.T, cfg.E), dtype=np.float32)
+    lg[:, 5] = 3.0
+    inp.logits = gen.f32_to_bf16_bits(lg)
+    g = run_gpu(inp)
+    assert g.offsets.tolist() == [0] * 6 + [37] * 3
+    check_full(inp, g)
+
+
+def test_logit_ties_break_to_lowest_id(cuda_device):
+    cfg = _cfg(T=64, E=16, k=3)
+    inp = gen.make_inputs(cfg, seed=6)
+    rng = np.random.default_rng(6)
+    lg = rng.integers(-2, 3, size=(cfg.T, cfg.E)).astype(np.float32) * 0.25  # many exact ties
+    inp.logits = gen.f32_to_bf16_bits(lg)
+    g = run_gpu(inp)
+    check_full(inp, g)
+
+
+def test_zero_tokens_is_a_noop(cuda_device):
+    import torch
+    from weight_only_quantized_warp_b200 import qmoe
+    cfg = _cfg(T=4)
+    inp = gen.make_inputs(cfg, seed=7)
+    m = qmoe.QMoE(cfg)
+    m.set_weights_from(inp)
+    y = torch.full((0, cfg.H), 1.0, dtype=torch.bfloat16, device="cuda")
+    x = torch.empty((0, cfg.H), dtype=torch.bfloat16, device="cuda")
+    lg = torch.empty((0, cfg.E), dtype=torch.bfloat16, device="cuda")
+    m.forward(x, lg, out=y)
+    torch.cuda.synchronize()
+
+
+def test_repeated_forward_is_bitwise_deterministic(cuda_device):
+    cfg = _cfg(T=50, bits=4, block_size=128, H=384, I=640)
+    inp = gen.make_inputs(cfg, seed=8)
+    a = run_gpu(inp)
+    b = run_gpu(inp, repeat=3)
+    np.testing.assert_array_equal(a.y, b.y)
+    np.testing.assert_array_equal(a.hidden, b.hidden)
+
+
+def test_rebind_replaces_the_pack(cuda_device):
+    import torch
+    from weight_only_quantized_warp_b200 import qmoe
+    cfg = _cfg(T=8)
+    a = gen.make_inputs(cfg, seed=9)
+    b = gen.make_inputs(cfg, seed=10)
+    b.x, b.logits = a.x, a.logits
+    m = qmoe.QMoE(cfg)
+    m.set_weights_from(a)
+    m.set_weights_from(b)
+    y = m.forward(qmoe.to_device(b.x, "cuda"), qmoe.to_device(b.logits, "cuda"))
+    torch.cuda.synchronize()
+    import oracle
+    from gpu_helpers import max_rel, to_numpy
+    assert max_rel(to_numpy(y), oracle.forward(b)["y"]) <= 1e-2
+
+
+# ------------------------------------------------------------ full-size configs
+
+def _sample(T, n=8, seed=0):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(T, size=min(n, T), replace=False))
+
+
+@pytest.mark.parametrize("name", ["mixtral_decode", "gpt_oss", "deepseek"])
+def test_full_size_configs(cuda_device, name):
+    cfg, seed, kw = gen.workload(name)
+    inp = gen.make_inputs(cfg, seed, **kw)
+    g = run_gpu(inp)
+    tokens = np.arange(cfg.T) if cfg.T <= 8 else _sample(cfg.T)
+    check_sampled(inp, g, tokens)
+
+
+@pytest.mark.parametrize("bits,T", [(4, 1), (4, 16), (8, 1), (8, 128)])
+def test_sweep_configs(cuda_device, bits, T):
+    cfg, seed, kw = gen.sweep(bits, T)
+    inp = gen.make_inputs(cfg, seed, **kw)
+    g = run_gpu(inp)
+    check_sampled(inp, g, _sample(T, 4, seed))

@@ -1,0 +1,476 @@
+// qmoe_api.cu -- the C ABI declared in include/qmoe.h: attribute validation,
+// the one-time pack, the per-call plan and workspace layout, and the launch
+// sequence of the forward. The lifecycle follows "ClikaRT::nn::QMoEWoQ":
+// make() declares storage-free slots, set_weights() binds and (here) packs
+// once, forward() serves from the pack, ~QMoEWoQ() releases it.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "qmoe_internal.cuh"
+
+namespace qmoe {
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Resident warps per SM assumed when sizing the FC2 split-K.
+static constexpr int64_t kSms = 148;
+
+Plan make_plan(const qmoe_handle& h, int64_t T) {
+    const qmoe_config& c = h.cfg;
+    Plan p;
+    p.T = T;
+    p.R = T * c.k;
+    const bool bf16 = c.act_dtype == QMOE_DTYPE_BF16;
+    p.path = bf16 ? kPathDecode : kPathSimt;
+    const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size;
+    if (p.path == kPathDecode) {
+        const int64_t per_expert = ceil_div(std::max<int64_t>(p.R, 1), E);
+        p.nt = per_expert <= 8 ? 1 : (per_expert <= 16 ? 2 : 4);
+        // enough FC2 warps (one per 16-row tile per touched expert per split)
+        // to give every SM several resident warps
+        const int64_t touched = std::min<int64_t>(E, std::max<int64_t>(p.R, 1));
+        const int64_t warps = touched * (H / kTileRows);
+        const int64_t want = kSms * 48;
+        const int64_t ngr = I / kgroup_of(c.expert_weight_bits);
+        int64_t s = ceil_div(want, warps);
+        s = std::min<int64_t>(s, 8);
+        s = std::min<int64_t>(s, ngr);
+        p.fc2_splits = int(std::max<int64_t>(s, 1));
+    }
+    p.launches = 5;
+    const size_t R = size_t(p.R);
+    const size_t act = bf16 ? 2 : 4;
+    size_t off = 0;
+    p.off_status = off;  off = align256(off + 16);  // fixed place, independent of T
+    p.off_idx = off;     off = align256(off + R * 4);
+    p.off_w = off;       off = align256(off + R * 4);
+    p.off_inv = off;     off = align256(off + R * 4);
+    p.off_perm = off;    off = align256(off + R * 4);
+    p.off_offsets = off; off = align256(off + size_t(E + 1) * 4);
+    p.off_h = off;       off = align256(off + R * size_t(I) * act);
+    p.off_o = off;       off = align256(off + size_t(p.fc2_splits) * R * size_t(H) * 4);
+    p.total = off;
+    return p;
+}
+
+}  // namespace qmoe
+
+using namespace qmoe;
+
+namespace {
+
+qmoe_status fail(const qmoe_handle* h, qmoe_status s, const char* fmt, ...) {
+    if (h) {
+        char buf[512];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(buf, sizeof buf, fmt, ap);
+        va_end(ap);
+        h->last_error = buf;
+    }
+    return s;
+}
+
+qmoe_status cuda_fail(const qmoe_handle* h, cudaError_t e, const char* where) {
+    return fail(h, QMOE_CUDA_ERROR, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+qmoe_status validate(const qmoe_config& c, std::string& why) {
+    char buf[256];
+    auto bad = [&](qmoe_status s, const char* msg) {
+        why = msg;
+        return s;
+    };
+    if (c.num_experts < 1 || c.hidden_size < 1 || c.inter_size < 1)
+        return bad(QMOE_INVALID_ARGUMENT, "num_experts, hidden_size and inter_size must be >= 1");
+    if (c.k < 1 || c.k > c.num_experts) return bad(QMOE_INVALID_ARGUMENT, "k must lie in [1, num_experts]");
+    if (c.expert_weight_bits != 4 && c.expert_weight_bits != 8)
+        return bad(QMOE_INVALID_ARGUMENT, "expert_weight_bits must be 4 or 8");
+    if (c.block_size != 0) {
+        if (!pow2(c.block_size) || c.block_size < 16)
+            return bad(QMOE_INVALID_ARGUMENT, "block_size must be 0 or a power of two >= 16");
+        if (c.hidden_size % c.block_size || c.inter_size % c.block_size)
+            return bad(QMOE_INVALID_ARGUMENT, "hidden_size and inter_size must divide by block_size");
+    }
+    if (c.activation_type < QMOE_ACT_RELU || c.activation_type > QMOE_ACT_IDENTITY)
+        return bad(QMOE_INVALID_ARGUMENT, "activation_type out of range");
+    if (c.swiglu_fusion < 0 || c.swiglu_fusion > 2)
+        return bad(QMOE_INVALID_ARGUMENT, "swiglu_fusion must be 0, 1 or 2");
+    if (c.has_fc3 && c.swiglu_fusion != 0)
+        return bad(QMOE_INVALID_ARGUMENT, "fc3 is only defined with swiglu_fusion 0");
+    if (c.has_fc3_bias && !c.has_fc3) return bad(QMOE_INVALID_ARGUMENT, "fc3 bias without an fc3 slot");
+    const bool gated = c.swiglu_fusion != 0 || c.has_fc3;
+    if (!gated && c.activation_type == QMOE_ACT_SWIGLU)
+        return bad(QMOE_INVALID_ARGUMENT, "swiglu needs a gate and an up projection (fusion 1/2 or fc3)");
+    if ((c.act_dtype != QMOE_DTYPE_F32 && c.act_dtype != QMOE_DTYPE_BF16) ||
+        (c.scale_dtype != QMOE_DTYPE_F32 && c.scale_dtype != QMOE_DTYPE_BF16))
+        return bad(QMOE_INVALID_ARGUMENT, "act_dtype and scale_dtype must be F32 or BF16");
+    if (c.reserved != 0) return bad(QMOE_INVALID_ARGUMENT, "reserved must be 0");
+    if (c.use_sparse_mixer) return bad(QMOE_UNSUPPORTED, "use_sparse_mixer is not built");
+    if (c.num_experts > 256) return bad(QMOE_UNSUPPORTED, "num_experts > 256 is not built");
+    if (c.hidden_size % 64 || c.inter_size % 64) {
+        snprintf(buf, sizeof buf, "hidden_size (%lld) and inter_size (%lld) must be multiples of 64",
+                 (long long)c.hidden_size, (long long)c.inter_size);
+        return bad(QMOE_UNSUPPORTED, buf);
+    }
+    if (c.num_experts * c.k > (int64_t(1) << 20))
+        return bad(QMOE_UNSUPPORTED, "num_experts * k too large");
+    return QMOE_OK;
+}
+
+void free_pack(uint8_t*& w1, void*& s1, float*& b1, uint8_t*& w2, void*& s2, float*& b2) {
+    cudaFree(w1);
+    cudaFree(s1);
+    cudaFree(b1);
+    cudaFree(w2);
+    cudaFree(s2);
+    cudaFree(b2);
+    w1 = nullptr;
+    s1 = nullptr;
+    b1 = nullptr;
+    w2 = nullptr;
+    s2 = nullptr;
+    b2 = nullptr;
+}
+
+float resolved_alpha(float a) { return (a == 0.0f || !std::isfinite(a)) ? 1.0f : a; }
+float resolved_limit(float l) { return (std::isfinite(l) && l > 0.0f) ? l : INFINITY; }
+
+}  // namespace
+
+extern "C" {
+
+const char* qmoe_status_string(qmoe_status s) {
+    switch (s) {
+        case QMOE_OK: return "QMOE_OK";
+        case QMOE_INVALID_ARGUMENT: return "QMOE_INVALID_ARGUMENT";
+        case QMOE_NOT_BOUND: return "QMOE_NOT_BOUND";
+        case QMOE_UNSUPPORTED: return "QMOE_UNSUPPORTED";
+        case QMOE_CUDA_ERROR: return "QMOE_CUDA_ERROR";
+        case QMOE_TIMEOUT: return "QMOE_TIMEOUT";
+        case QMOE_OUT_OF_MEMORY: return "QMOE_OUT_OF_MEMORY";
+    }
+    return "QMOE_UNKNOWN_STATUS";
+}
+
+const char* qmoe_last_error(const qmoe_handle* h) { return h ? h->last_error.c_str() : ""; }
+
+qmoe_status qmoe_create(const qmoe_config* cfg, qmoe_handle** out) {
+    if (!cfg || !out) return QMOE_INVALID_ARGUMENT;
+    *out = nullptr;
+    std::string why;
+    const qmoe_status s = validate(*cfg, why);
+    if (s != QMOE_OK) return s;
+    qmoe_handle* h = new (std::nothrow) qmoe_handle();
+    if (!h) return QMOE_OUT_OF_MEMORY;
+    h->cfg = *cfg;
+    h->gated = cfg->swiglu_fusion != 0 || cfg->has_fc3;
+    h->n1 = (h->gated ? 2 : 1) * cfg->inter_size;
+    *out = h;
+    return QMOE_OK;
+}
+
+void qmoe_destroy(qmoe_handle* h) {
+    if (!h) return;
+    free_pack(h->w1, h->s1, h->b1, h->w2, h->s2, h->b2);
+    delete h;
+}
+
+qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_s,
+                             const void* fc1_b, const void* fc2_w, const void* fc2_s,
+                             const void* fc2_b, const void* fc3_w, const void* fc3_s,
+                             const void* fc3_b, void* stream) {
+    if (!h) return QMOE_INVALID_ARGUMENT;
+    std::lock_guard<std::mutex> lock(h->mu);
+    const qmoe_config& c = h->cfg;
+    if (!fc1_w || !fc1_s || !fc2_w || !fc2_s)
+        return fail(h, QMOE_INVALID_ARGUMENT, "fc1/fc2 weights and scales are required");
+    if (bool(fc1_b) != bool(c.has_fc1_bias))
+        return fail(h, QMOE_INVALID_ARGUMENT, "fc1 bias must be given iff has_fc1_bias");
+    if (bool(fc2_b) != bool(c.has_fc2_bias))
+        return fail(h, QMOE_INVALID_ARGUMENT, "fc2 bias must be given iff has_fc2_bias");
+    if ((bool(fc3_w) || bool(fc3_s)) != bool(c.has_fc3) || (c.has_fc3 && (!fc3_w || !fc3_s)))
+        return fail(h, QMOE_INVALID_ARGUMENT, "fc3 weights and scales must be given iff has_fc3");
+    if (bool(fc3_b) != bool(c.has_fc3_bias))
+        return fail(h, QMOE_INVALID_ARGUMENT, "fc3 bias must be given iff has_fc3_bias");
+
+    cudaStream_t st = (cudaStream_t)stream;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return cuda_fail(h, err, "cudaGetDevice");
+    err = prepare_route_permute();
+    if (err != cudaSuccess) return cuda_fail(h, err, "prepare kernels");
+
+    const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size, N1 = h->n1;
+    const int bits = c.expert_weight_bits, bs = c.block_size;
+    const size_t ssz = c.scale_dtype == QMOE_DTYPE_BF16 ? 2 : 4;
+    const int64_t nsb1 = bs ? H / bs : 1, nsb2 = bs ? I / bs : 1;
+    const bool any_b1 = c.has_fc1_bias || c.has_fc3_bias;
+
+    uint8_t *w1 = nullptr, *w2 = nullptr;
+    void *s1 = nullptr, *s2 = nullptr;
+    float *b1 = nullptr, *b2 = nullptr;
+    auto alloc = [&](void** p, size_t n) { return cudaMalloc(p, n < 16 ? 16 : n); };
+    if ((err = alloc((void**)&w1, size_t(E * N1 * H * bits / 8))) != cudaSuccess ||
+        (err = alloc(&s1, size_t(E * N1 * nsb1) * ssz)) != cudaSuccess ||
+        (any_b1 && (err = alloc((void**)&b1, size_t(E * N1) * 4)) != cudaSuccess) ||
+        (err = alloc((void**)&w2, size_t(E * H * I * bits / 8))) != cudaSuccess ||
+        (err = alloc(&s2, size_t(E * H * nsb2) * ssz)) != cudaSuccess ||
+        (c.has_fc2_bias && (err = alloc((void**)&b2, size_t(E * H) * 4)) != cudaSuccess)) {
+        free_pack(w1, s1, b1, w2, s2, b2);
+        cudaGetLastError();
+        return fail(h, QMOE_OUT_OF_MEMORY, "cudaMalloc for the pack: %s", cudaGetErrorString(err));
+    }
+
+    PackArgs p1{};
+    p1.src = (const uint8_t*)fc1_w;
+    p1.s_src = fc1_s;
+    p1.b_src = fc1_b;
+    p1.src_up = (const uint8_t*)fc3_w;
+    p1.s_src_up = fc3_s;
+    p1.b_src_up = fc3_b;
+    p1.dst = w1;
+    p1.s_dst = s1;
+    p1.b_dst = b1;
+    p1.E = E;
+    p1.N = N1;
+    p1.K = H;
+    p1.I = I;
+    p1.bits = bits;
+    p1.block_size = bs;
+    p1.mode = c.has_fc3 ? 3 : c.swiglu_fusion;  // 0 identity, 1 interleaved, 2 concatenated
+    p1.scale_bf16 = c.scale_dtype == QMOE_DTYPE_BF16;
+    p1.act_bf16 = c.act_dtype == QMOE_DTYPE_BF16;
+    PackArgs p2 = p1;
+    p2.src = (const uint8_t*)fc2_w;
+    p2.s_src = fc2_s;
+    p2.b_src = fc2_b;
+    p2.src_up = nullptr;
+    p2.s_src_up = nullptr;
+    p2.b_src_up = nullptr;
+    p2.dst = w2;
+    p2.s_dst = s2;
+    p2.b_dst = b2;
+    p2.N = H;
+    p2.K = I;
+    p2.mode = 0;
+    if ((err = launch_pack(p1, st)) != cudaSuccess || (err = launch_pack(p2, st)) != cudaSuccess ||
+        (err = cudaStreamSynchronize(st)) != cudaSuccess) {
+        free_pack(w1, s1, b1, w2, s2, b2);
+        return cuda_fail(h, err, "pack");
+    }
+    free_pack(h->w1, h->s1, h->b1, h->w2, h->s2, h->b2);
+    h->w1 = w1;
+    h->s1 = s1;
+    h->b1 = b1;
+    h->w2 = w2;
+    h->s2 = s2;
+    h->b2 = b2;
+    h->device = dev;
+    h->bound = true;
+    h->last_error.clear();
+    return QMOE_OK;
+}
+
+size_t qmoe_workspace_size(const qmoe_handle* h, int64_t T) {
+    if (!h || T < 0) return 0;
+    return make_plan(*h, T).total;
+}
+
+int32_t qmoe_path_for(const qmoe_handle* h, int64_t T) {
+    if (!h || T < 0) return -1;
+    return make_plan(*h, T).path;
+}
+
+int32_t qmoe_launches_for(const qmoe_handle* h, int64_t T) {
+    if (!h || T < 0) return -1;
+    return T == 0 ? 0 : make_plan(*h, T).launches;
+}
+
+}  // extern "C"
+
+static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
+                                const void* router_logits, const void* shared_output, void* y,
+                                void* workspace, size_t workspace_bytes, void* stream,
+                                void* const* events, int32_t n_events) {
+    if (!h) return QMOE_INVALID_ARGUMENT;
+    if (!h->bound) return fail(h, QMOE_NOT_BOUND, "forward before set_weights bound the weights");
+    if (T < 0) return fail(h, QMOE_INVALID_ARGUMENT, "T must be >= 0");
+    if (T == 0) return QMOE_OK;
+    if (!x || !router_logits || !y || !workspace)
+        return fail(h, QMOE_INVALID_ARGUMENT, "x, router_logits, y and workspace are required");
+    if (T * h->cfg.k >= (int64_t(1) << 31))
+        return fail(h, QMOE_UNSUPPORTED, "T * k must stay below 2^31");
+    if (reinterpret_cast<uintptr_t>(workspace) & 255)
+        return fail(h, QMOE_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
+    const Plan p = make_plan(*h, T);
+    if (workspace_bytes < p.total)
+        return fail(h, QMOE_INVALID_ARGUMENT, "workspace too small: %zu < %zu", workspace_bytes,
+                    p.total);
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device)
+        return fail(h, QMOE_INVALID_ARGUMENT, "current device %d is not the device the weights live on (%d)",
+                    dev, h->device);
+    const qmoe_config& c = h->cfg;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (events && n_events != p.launches + 1)
+        return fail(h, QMOE_INVALID_ARGUMENT, "n_events must be %d", p.launches + 1);
+    int ev_i = 0;
+    auto mark = [&]() -> cudaError_t {
+        if (!events) return cudaSuccess;
+        return cudaEventRecord((cudaEvent_t)events[ev_i++], st);
+    };
+    char* ws = (char*)workspace;
+    int32_t* idx = (int32_t*)(ws + p.off_idx);
+    float* tw = (float*)(ws + p.off_w);
+    int32_t* inv = (int32_t*)(ws + p.off_inv);
+    int32_t* perm = (int32_t*)(ws + p.off_perm);
+    int32_t* offsets = (int32_t*)(ws + p.off_offsets);
+    void* hid = ws + p.off_h;
+    float* o = (float*)(ws + p.off_o);
+    const int E = int(c.num_experts), k = int(c.k);
+    const int bf16 = c.act_dtype == QMOE_DTYPE_BF16;
+    cudaError_t err;
+    if ((err = cudaMemsetAsync(ws + p.off_status, 0, 16, st)) != cudaSuccess)
+        return cuda_fail(h, err, "status reset");
+    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+    if ((err = launch_route(router_logits, bf16, T, E, k, c.normalize_routing_weights, idx, tw, st)) !=
+        cudaSuccess)
+        return cuda_fail(h, err, "route");
+    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+    if ((err = launch_permute(idx, T, E, k, offsets, perm, inv, st)) != cudaSuccess)
+        return cuda_fail(h, err, "permute");
+
+    FfnArgs f1{};
+    f1.W = h->w1;
+    f1.S = h->s1;
+    f1.bias = h->b1;
+    f1.act = x;
+    f1.rowmap = perm;
+    f1.offsets = offsets;
+    f1.out = hid;
+    f1.N = h->n1;
+    f1.K = c.hidden_size;
+    f1.R = p.R;
+    f1.E = E;
+    f1.bits = c.expert_weight_bits;
+    f1.block_size = c.block_size;
+    f1.gated = h->gated;
+    f1.is_fc1 = 1;
+    f1.act_type = c.activation_type;
+    f1.alpha = resolved_alpha(c.activation_alpha);
+    f1.beta = c.activation_beta;
+    f1.limit = resolved_limit(c.swiglu_limit);
+    f1.splits = 1;
+    f1.scale_bf16 = c.scale_dtype == QMOE_DTYPE_BF16;
+    f1.act_bf16 = bf16;
+    f1.nt = p.nt;
+    FfnArgs f2 = f1;
+    f2.W = h->w2;
+    f2.S = h->s2;
+    f2.bias = nullptr;
+    f2.act = hid;
+    f2.rowmap = nullptr;
+    f2.out = o;
+    f2.N = c.hidden_size;
+    f2.K = c.inter_size;
+    f2.gated = 0;
+    f2.is_fc1 = 0;
+    f2.splits = p.fc2_splits;
+    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+    err = p.path == kPathSimt ? launch_ffn_simt(f1, st) : launch_ffn_decode(f1, st);
+    if (err != cudaSuccess) return cuda_fail(h, err, "fc1");
+    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+    err = p.path == kPathSimt ? launch_ffn_simt(f2, st) : launch_ffn_decode(f2, st);
+    if (err != cudaSuccess) return cuda_fail(h, err, "fc2");
+    CombineArgs ca{};
+    ca.o = o;
+    ca.topk_idx = idx;
+    ca.topk_w = tw;
+    ca.inv = inv;
+    ca.b2 = h->b2;
+    ca.shared = shared_output;
+    ca.y = y;
+    ca.T = T;
+    ca.H = c.hidden_size;
+    ca.R = p.R;
+    ca.k = k;
+    ca.splits = p.fc2_splits;
+    ca.act_bf16 = bf16;
+    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+    if ((err = launch_combine(ca, st)) != cudaSuccess) return cuda_fail(h, err, "combine");
+    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+    return QMOE_OK;
+}
+
+extern "C" {
+
+qmoe_status qmoe_forward(const qmoe_handle* h, int64_t T, const void* x, const void* router_logits,
+                         const void* shared_output, void* y, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    return forward_impl(h, T, x, router_logits, shared_output, y, workspace, workspace_bytes,
+                        stream, nullptr, 0);
+}
+
+qmoe_status qmoe_forward_profiled(const qmoe_handle* h, int64_t T, const void* x,
+                                  const void* router_logits, const void* shared_output, void* y,
+                                  void* workspace, size_t workspace_bytes, void* stream,
+                                  void* const* events, int32_t n_events) {
+    if (!events) return fail(h, QMOE_INVALID_ARGUMENT, "events is required");
+    return forward_impl(h, T, x, router_logits, shared_output, y, workspace, workspace_bytes,
+                        stream, events, n_events);
+}
+
+qmoe_status qmoe_debug_routing(const qmoe_handle* h, int64_t T, const void* workspace,
+                               int32_t* topk_idx, float* topk_w, int32_t* offsets,
+                               int32_t* perm_tok, int32_t* inv, void* stream) {
+    if (!h || !workspace || T < 0) return QMOE_INVALID_ARGUMENT;
+    const Plan p = make_plan(*h, T);
+    const char* ws = (const char*)workspace;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t R = size_t(p.R);
+    cudaError_t err = cudaSuccess;
+    auto cp = [&](void* dst, size_t off, size_t n) {
+        if (dst && n && err == cudaSuccess)
+            err = cudaMemcpyAsync(dst, ws + off, n, cudaMemcpyDeviceToDevice, st);
+    };
+    cp(topk_idx, p.off_idx, R * 4);
+    cp(topk_w, p.off_w, R * 4);
+    cp(offsets, p.off_offsets, size_t(h->cfg.num_experts + 1) * 4);
+    cp(perm_tok, p.off_perm, R * 4);
+    cp(inv, p.off_inv, R * 4);
+    return err == cudaSuccess ? QMOE_OK : cuda_fail(h, err, "debug_routing");
+}
+
+qmoe_status qmoe_debug_hidden(const qmoe_handle* h, int64_t T, const void* workspace, void* hidden,
+                              void* stream) {
+    if (!h || !workspace || !hidden || T < 0) return QMOE_INVALID_ARGUMENT;
+    const Plan p = make_plan(*h, T);
+    const size_t act = h->cfg.act_dtype == QMOE_DTYPE_BF16 ? 2 : 4;
+    const size_t n = size_t(p.R) * size_t(h->cfg.inter_size) * act;
+    if (!n) return QMOE_OK;
+    cudaError_t err = cudaMemcpyAsync(hidden, (const char*)workspace + p.off_h, n,
+                                      cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+    return err == cudaSuccess ? QMOE_OK : cuda_fail(h, err, "debug_hidden");
+}
+
+qmoe_status qmoe_read_device_status(const qmoe_handle* h, const void* workspace, void* stream) {
+    if (!h || !workspace) return QMOE_INVALID_ARGUMENT;
+    const Plan p = make_plan(*h, 0);
+    int32_t v = 0;
+    cudaError_t err = cudaMemcpyAsync(&v, (const char*)workspace + p.off_status, 4,
+                                      cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (err == cudaSuccess) err = cudaStreamSynchronize((cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_fail(h, err, "read_device_status");
+    return v == 0 ? QMOE_OK : QMOE_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,144 @@
+// qmoe_internal.cuh -- declarations shared by the CUDA translation units of
+// the QMoE library: the handle, the per-call plan, the packed weight layout
+// and the kernel launchers. Nothing here is part of the public C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/qmoe.h"
+
+namespace qmoe {
+
+// ---------------------------------------------------------------------------
+// Packed weight layout ("fragment order").
+//
+// A weight W[N, K] of one expert (N output rows, K reduction) is stored as
+// [N/16 row tiles][K/KG k-groups][32 lanes][16 bytes], KG = 64 for 4-bit and
+// 32 for 8-bit codes, so one (row tile, k-group) unit is 512 contiguous bytes
+// and one row tile is contiguous along K. Lane L owns rows r0 = L/4 and
+// r0 + 8 of the tile and the k sub-range [KG/4 * (L%4), KG/4 * (L%4 + 1)) of
+// the group: exactly the operand fragments of an m16n8k16 bf16 MMA whose k
+// axis is permuted consistently for weights and activations (see
+// decode_fragments in ffn_decode.cu). Bytes are the page's codes, re-laid,
+// never decoded: the pack has the same size as the input.
+//
+// FC1 of a gated FFN is re-laid so that row tile t holds gate rows
+// i = 8t..8t+7 in its first 8 rows and the matching up rows in its last 8,
+// whatever the input layout (fused interleaved, fused concatenated, or fc1 +
+// fc3). Scales follow as [N/16][K/bs or 1][16] with the 16 entries in lane
+// order (r0, r0 + 8) pairs; biases as fp32 in packed row order.
+// ---------------------------------------------------------------------------
+constexpr int kTileRows = 16;
+constexpr int kUnitBytes = 512;
+__host__ __device__ constexpr int kgroup_of(int bits) { return bits == 4 ? 64 : 32; }
+
+// Hot-path selection.
+enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2 };
+
+struct Plan {
+    int path = kPathDecode;
+    int64_t T = 0, R = 0;
+    int nt = 1;          // 8-token MMA n-tiles handled per pass (decode path)
+    int fc2_splits = 1;  // split-K factor of FC2 (partials reduced by the combine)
+    int launches = 0;
+    size_t off_idx = 0, off_w = 0, off_inv = 0, off_perm = 0, off_offsets = 0, off_status = 0,
+           off_h = 0, off_o = 0, total = 0;
+};
+
+}  // namespace qmoe
+
+struct qmoe_handle {
+    qmoe_config cfg{};
+    bool gated = false;
+    int64_t n1 = 0;       // packed FC1 rows: 2I gated, I otherwise
+    bool bound = false;
+    uint8_t* w1 = nullptr;
+    void* s1 = nullptr;
+    float* b1 = nullptr;  // packed-row-order fp32, nullptr when no fc1/fc3 bias
+    uint8_t* w2 = nullptr;
+    void* s2 = nullptr;
+    float* b2 = nullptr;  // [E, H] fp32, nullptr when no fc2 bias
+    int device = -1;
+    mutable std::mutex mu;
+    mutable std::string last_error;
+};
+
+namespace qmoe {
+
+Plan make_plan(const qmoe_handle& h, int64_t T);
+
+// ----------------------------------------------------------------- launchers
+// Each returns the cudaError_t of its launch.
+
+// Re-lay one packed stack (and its scales / biases) into fragment order.
+// Row mapping: mode 0 = identity; 1 = fused interleaved gate/up; 2 = fused
+// concatenated gate/up; 3 = gate from `src`, up from `src_up` (fc1 + fc3).
+struct PackArgs {
+    const uint8_t* src;
+    const uint8_t* src_up;   // mode 3 only
+    const void* s_src;
+    const void* s_src_up;    // mode 3 only
+    const void* b_src;       // nullable
+    const void* b_src_up;    // nullable (mode 3)
+    uint8_t* dst;
+    void* s_dst;
+    float* b_dst;            // nullable
+    int64_t E, N, K;         // N = packed rows of one expert
+    int64_t I;               // gated modes: inter size
+    int bits, block_size, mode;
+    int scale_bf16, act_bf16;
+};
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t st);
+
+// Top-k softmax routing: warp per token.
+cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
+                         int32_t* topk_idx, float* topk_w, cudaStream_t st);
+
+// Histogram, scan and stable scatter into per-expert segments (one CTA).
+// prepare_route_permute() raises the permute kernel's shared-memory limit on
+// the current device; call it once per device before the first launch.
+cudaError_t prepare_route_permute();
+cudaError_t launch_permute(const int32_t* topk_idx, int64_t T, int E, int k, int32_t* offsets,
+                           int32_t* perm_tok, int32_t* inv, cudaStream_t st);
+
+// Expert FFN layer over the segments (decode / SIMT paths).
+struct FfnArgs {
+    const uint8_t* W;        // packed weights, fragment order
+    const void* S;           // packed scales
+    const float* bias;       // packed-row-order fp32 (FC1), or nullptr
+    const void* act;         // activations: x [T, K] (FC1) or h [R, K] (FC2)
+    const int32_t* rowmap;   // perm_tok for FC1 (row of x), nullptr for FC2
+    const int32_t* offsets;  // [E + 1]
+    void* out;               // FC1: h [R, I]; FC2: partials [splits, R, N] fp32
+    int64_t N, K, R;
+    int E, bits, block_size;
+    int gated, is_fc1, act_type;
+    float alpha, beta, limit;
+    int splits;
+    int scale_bf16, act_bf16;
+    int nt;
+};
+cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
+cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
+
+// Router-weighted combine with fc2 bias and shared output; sums the FC2
+// split partials in fixed order.
+struct CombineArgs {
+    const float* o;          // [splits, R, H]
+    const int32_t* topk_idx;
+    const float* topk_w;
+    const int32_t* inv;
+    const float* b2;         // [E, H] or nullptr
+    const void* shared;      // [T, H] or nullptr
+    void* y;                 // [T, H]
+    int64_t T, H, R;
+    int k, splits, act_bf16;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+
+}  // namespace qmoe

@@ -1,0 +1,202 @@
+// route_permute.cu -- top-k softmax routing and the token -> expert
+// permutation.
+//
+// Routing follows the "MoE" page (clika_runtime.nn) class summary -- a router
+// picks the top-k experts per token and the outputs combine under the router
+// weights -- with the QMoE page's k and normalize_routing_weights attributes.
+// Readings: selection is by raw logit (exact in any precision, so the
+// selection is bit-identical to any other exact implementation), ties go to
+// the lower expert id, and the list is ordered by (logit descending, id
+// ascending). The weights are the softmax over all E logits restricted to the
+// selection, renormalised over the k when asked.
+//
+// The permutation groups the T*k (token, slot) pairs into per-expert
+// segments, experts ascending and tokens ascending inside a segment: the
+// order in which the "per-expert kernels" ("ClikaRT::nn::QMoEWoQ", class
+// description) consume their rows.
+#include "qmoe_internal.cuh"
+
+namespace qmoe {
+namespace {
+
+constexpr int kMaxPerLane = 8;  // E <= 256
+
+__device__ __forceinline__ bool better(float v, int e, float bv, int be) {
+    return v > bv || (v == bv && e < be);
+}
+
+// One warp per token.
+__global__ void route_kernel(const void* logits, int act_bf16, int64_t T, int E, int k,
+                             int normalize, int32_t* __restrict__ topk_idx,
+                             float* __restrict__ topk_w) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    float v[kMaxPerLane];
+    const int per = (E + 31) >> 5;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = 0.0f;
+        if (i < per && e < E) {
+            v[i] = act_bf16 ? __bfloat162float(((const __nv_bfloat16*)logits)[t * E + e])
+                            : ((const float*)logits)[t * E + e];
+        }
+    }
+    // max over all E
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i)
+        if (i < per && lane + 32 * i < E) mx = fmaxf(mx, v[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    // softmax denominator over all E (fixed reduction tree)
+    float z = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i)
+        if (i < per && lane + 32 * i < E) z += expf(v[i] - mx);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+
+    uint32_t taken = 0;
+    float p_keep[kMaxPerLane];  // p_j kept by lane j%32 in slot j/32
+    float sel = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kMaxPerLane; ++i) {
+            const int e = lane + 32 * i;
+            if (i < per && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, be)) {
+                bv = v[i];
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (better(ov, oe, bv, be)) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        const float p = expf(bv - mx);
+        sel += p;
+        if ((j & 31) == lane) p_keep[j >> 5] = p;
+        if (lane == 0) topk_idx[t * k + j] = be;
+    }
+    const float den = normalize ? sel : z;
+#pragma unroll
+    for (int s = 0; s < kMaxPerLane; ++s) {
+        const int j = lane + 32 * s;
+        if (j < k) topk_w[t * k + j] = p_keep[s] / den;
+    }
+}
+
+// One CTA of 1024 threads. Token chunks of 1024: for each chunk, warp-level
+// bit masks per expert give each (token, expert) pair its rank among the
+// chunk's earlier tokens; a running per-expert base carries across chunks.
+constexpr int kPermThreads = 1024;
+constexpr int kWarps = kPermThreads / 32;
+
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t T, int E, int k, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv) {
+    extern __shared__ uint32_t sm[];
+    uint32_t* mask = sm;                   // [kWarps][E]
+    uint32_t* wpre = mask + kWarps * E;    // [kWarps][E] exclusive prefix over warps
+    int32_t* cnt = (int32_t*)(wpre + kWarps * E);  // [E]
+    int32_t* off = cnt + E;                // [E + 1]
+    int32_t* base = off + E + 1;           // [E]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t R = T * k;
+
+    for (int e = tid; e < E; e += kPermThreads) {
+        cnt[e] = 0;
+        base[e] = 0;
+    }
+    __syncthreads();
+    for (int64_t r = tid; r < R; r += kPermThreads) atomicAdd(&cnt[topk_idx[r]], 1);
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan over E with one warp
+        int carry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            int v = e < E ? cnt[e] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (e < E) off[e] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) off[E] = carry;
+    }
+    __syncthreads();
+    for (int e = tid; e <= E; e += kPermThreads) offsets[e] = off[e];
+
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t t0 = 0; t0 < T; t0 += kPermThreads) {
+        for (int i = tid; i < kWarps * E; i += kPermThreads) mask[i] = 0;
+        __syncthreads();
+        const int64_t t = t0 + tid;
+        if (t < T)
+            for (int j = 0; j < k; ++j) atomicOr(&mask[warp * E + topk_idx[t * k + j]], 1u << lane);
+        __syncthreads();
+        for (int e = tid; e < E; e += kPermThreads) {
+            uint32_t run = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                wpre[w * E + e] = run;
+                run += __popc(mask[w * E + e]);
+            }
+        }
+        __syncthreads();
+        if (t < T) {
+            for (int j = 0; j < k; ++j) {
+                const int e = topk_idx[t * k + j];
+                const int64_t pos = (int64_t)off[e] + base[e] + wpre[warp * E + e] +
+                                    __popc(mask[warp * E + e] & lt);
+                perm_tok[pos] = int32_t(t);
+                inv[t * k + j] = int32_t(pos);
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += kPermThreads)
+            base[e] += wpre[(kWarps - 1) * E + e] + __popc(mask[(kWarps - 1) * E + e]);
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
+                         int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t blocks = (T * 32 + threads - 1) / threads;
+    route_kernel<<<unsigned(blocks), threads, 0, st>>>(logits, act_bf16, T, E, k, normalize,
+                                                       topk_idx, topk_w);
+    return cudaGetLastError();
+}
+
+size_t permute_smem_bytes(int E) {
+    return sizeof(uint32_t) * (2 * kWarps * E) + sizeof(int32_t) * (3 * E + 1);
+}
+
+cudaError_t prepare_route_permute() {
+    return cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(permute_smem_bytes(256)));
+}
+
+cudaError_t launch_permute(const int32_t* topk_idx, int64_t T, int E, int k, int32_t* offsets,
+                           int32_t* perm_tok, int32_t* inv, cudaStream_t st) {
+    permute_kernel<<<1, kPermThreads, permute_smem_bytes(E), st>>>(topk_idx, T, E, k, offsets,
+                                                                  perm_tok, inv);
+    return cudaGetLastError();
+}
+
+}  // namespace qmoe
