@@ -6,11 +6,12 @@
 // description). FC1 applies the gated activation of the QMoE page
 // (activation_type, activation_alpha/beta, swiglu_limit) in its epilogue.
 //
-// Work split: one warp per 16-row weight tile, looping over the tile's
-// k-groups (optionally a K-split of them) and over the expert's routed rows in
-// passes of 8*NT tokens. The weight tile streams from HBM through a ring of
-// D in-flight 16-byte loads per lane; activations (a few hundred KB at decode
-// sizes) are read through L1.
+// Work split: one CTA per (128-row weight block, expert, K-split), one warp
+// per 16-row tile of the block, looping over the tile's k-groups and over the
+// expert's routed rows in passes of 8*NT tokens. The weight tile streams from
+// HBM through a ring of D in-flight 16-byte loads per lane (scales ride along
+// in a parallel ring); the pass's activation rows are staged once per CTA in
+// shared memory with cp.async.
 //
 // Fragments. For an m16n8k16 MMA, lane L holds A rows r0 = L/4 and r0 + 8 at
 // k positions 2c, 2c+1, 2c+8, 2c+9 (c = L%4) and B column r0 at the same k
@@ -34,6 +35,8 @@
 // sees exact integer weights. Smaller blocks (16 and 32 for int4, 16 for
 // int8) cover only part of a group's k-steps, so the scale is folded into the
 // decoded bf16 weight instead (one rounding).
+#include <algorithm>
+
 #include "qmoe_internal.cuh"
 
 namespace qmoe {
@@ -196,164 +199,350 @@ __device__ __forceinline__ void split_range(int64_t ngr, int splits, int split, 
     hi = min(ngr, (split + 1) * per * gpb);
 }
 
-// SMODE: 0 per-column scale after the K loop; 1 block scale after each
-// block's MMAs; 2 block scale folded into the decoded weights.
-template <int BITS, int SMODE, bool SF32, int NT>
-__global__ void __launch_bounds__(kWarps * 32) ffn_decode_kernel(const FfnArgs a) {
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const uint32_t d = uint32_t(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Raw scale pair (rows r0, r0 + 8) of one row tile and block: two bf16 in one
+// word, or two fp32.
+template <bool F32>
+struct ScaleRaw;
+template <>
+struct ScaleRaw<false> {
+    uint32_t v;
+    __device__ __forceinline__ static ScaleRaw load(const void* S, int idx) {
+        return {*reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)S + idx)};
+    }
+    __device__ __forceinline__ void get(float& sa, float& sb) const {
+        sa = __uint_as_float(v << 16);
+        sb = __uint_as_float(v & 0xFFFF0000u);
+    }
+};
+template <>
+struct ScaleRaw<true> {
+    float2 v;
+    __device__ __forceinline__ static ScaleRaw load(const void* S, int idx) {
+        return {*reinterpret_cast<const float2*>((const float*)S + idx)};
+    }
+    __device__ __forceinline__ void get(float& sa, float& sb) const {
+        sa = v.x;
+        sb = v.y;
+    }
+};
+
+// Bytes of one staged activation row for a k range of kr elements: bf16
+// values plus 16 bytes of padding, which spreads the 8 rows a warp reads at
+// one time over all 32 shared-memory banks.
+__host__ __device__ constexpr int64_t staged_row_bytes(int64_t kr) { return kr * 2 + 16; }
+
+// Zero-point folding (int4, scale after the MMA). With A = 128 + q (the code
+// OR-ed into bf16 128.0, no subtraction), sum_k (q - 8) x_k equals
+// sum_k A_k x_k - 136 * sum_k x_k. The activation sums per scale chunk and
+// token are computed once per CTA pass from the staged rows, so the weight
+// decode is 7 bit operations per 8 codes. The products A_k x_k are exact in
+// fp32; the subtraction cancels a term about 17x the result, which costs a few
+// fp32 ulp of that larger term.
+constexpr float kFoldOffset = 136.0f;  // 128 (bf16 magic) + 8 (zero point)
+constexpr int kRing = 8;               // weight loads in flight per lane
+
+// SMODE: 0 per-column scale after the K loop; 1 block scale applied to the MMA
+// partial every P k-groups (P = min(groups per block, kRing), so a block may
+// be applied in several chunks with the same scale); 2 block scale folded
+// into the decoded weights (P = 1).
+//
+// One CTA = 8 warps = the 8 row tiles of one 128-row block of one expert, for
+// one K-split. The CTA stages the activation rows of its current 8*NT tokens
+// (its K range only) in shared memory with cp.async, while every warp already
+// has its first kRing weight loads in flight. The k-group loop has a steady
+// part (loads always in range, no guards), one guarded drain round and a
+// tail; all shared-memory, weight and scale addresses advance by constants.
+template <int BITS, int SMODE, bool SF32, int NT, int P>
+__global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArgs a) {
     constexpr int KG = kgroup_of(BITS);
-    constexpr int D = 8;  // weight loads in flight per lane
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int D = kRing;
+    static_assert(D % P == 0, "scale chunk must divide the ring");
+    constexpr bool FOLD = (BITS == 4 && SMODE != 2);
+    constexpr int GS = kTilesPerBlock * kUnitBytes;  // group stride, 4 KB
+    constexpr int ROWS = 8 * NT;
+    constexpr int KSTEPS = BITS == 4 ? 4 : 2;
+    constexpr int LG_KG = BITS == 4 ? 6 : 5;
+    extern __shared__ __align__(16) uint8_t xs[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r0 = lane >> 2, c = lane & 3;
     const int e = blockIdx.y, split = blockIdx.z;
+    const int64_t rb = blockIdx.x;
     const int64_t nrt = a.N / kTileRows;
-    const int64_t rt = (int64_t)blockIdx.x * kWarps + warp;
-    if (rt >= nrt) return;
+    const int64_t nrb = padded_rows(a.N) / kBlockRows;
+    const int64_t rt = rb * kTilesPerBlock + warp;
+    const bool active = rt < nrt;
     const int64_t seg0 = a.offsets[e];
     const int M = a.offsets[e + 1] - int(seg0);
-    if (M <= 0) return;
+    if (M <= 0) return;  // uniform over the CTA
     const int64_t ngr = a.K / KG;
     const int64_t nsb = a.block_size > 0 ? a.K / a.block_size : 1;
-    const int64_t gpb = (SMODE == 1) ? a.block_size / KG : 1;
+    const int lg_bs = a.block_size > 0 ? __ffs(a.block_size) - 1 : 0;
+    const int lg_gpb = SMODE == 1 ? lg_bs - LG_KG : 0;
     int64_t g_lo, g_hi;
-    split_range(ngr, a.splits, split, gpb, g_lo, g_hi);
+    split_range(ngr, a.splits, split, SMODE == 1 ? (int64_t(1) << lg_gpb) : 1, g_lo, g_hi);
+    const int ng = int(g_hi - g_lo);
+    const int kr = ng * KG;
+    const int rs = int(staged_row_bytes(kr));
+    const int chunks = kr / 8;  // 16-byte chunks per staged row
+    // activation sums for the zero-point fold: [chunk of P groups][row]
+    // (SMODE 1) or [row] (SMODE 0)
+    float* cs = reinterpret_cast<float*>(xs + ROWS * rs);
+    const int nch = FOLD ? (SMODE == 1 ? ng / P : 1) : 0;
 
-    const uint8_t* wtile = a.W + ((int64_t)e * nrt + rt) * ngr * kUnitBytes + lane * 16;
-    const int64_t sbase = ((int64_t)e * nrt + rt) * nsb * 16 + 2 * r0;  // scale of row r0; +1 = r0+8
+    const uint8_t* wp =
+        a.W + (((int64_t)e * nrb + rb) * ngr * kTilesPerBlock + warp) * kUnitBytes + lane * 16 +
+        g_lo * GS;
+    // scale pairs of this tile and lane (rows r0, r0 + 8): base pointer, then
+    // a 32-bit index per chunk
+    const int64_t sb0 = (((int64_t)e * nrb + rb) * nsb * kTilesPerBlock + warp) * 16 + 2 * r0;
+    const void* sbase = SF32 ? (const void*)((const float*)a.S + sb0)
+                             : (const void*)((const __nv_bfloat16*)a.S + sb0);
+    const int kc = SMODE == 2 ? (KG / 4) * c : 0;
+    auto sidx = [&](int ga) -> int {
+        return SMODE == 1 ? (ga >> lg_gpb) * 128 : ((ga * KG + kc) >> lg_bs) * 128;
+    };
     const __nv_bfloat16* act = (const __nv_bfloat16*)a.act;
 
     float s0 = 1.0f, s1 = 1.0f;  // per-column scales
-    if (SMODE == 0) {
-        s0 = load_scale(a.S, sbase, SF32);
-        s1 = load_scale(a.S, sbase + 1, SF32);
-    }
+    if (SMODE == 0 && active) ScaleRaw<SF32>::load(sbase, 0).get(s0, s1);
 
-    for (int p0 = 0; p0 < M; p0 += 8 * NT) {
-        const __nv_bfloat16* xrow[NT];
+    for (int p0 = 0; p0 < M; p0 += ROWS) {
+        uint4 wr[D];
+        ScaleRaw<SF32> sr[D / P];
+        if (active) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int tok = min(p0 + 8 * n + r0, M - 1);
-            const int64_t row = a.rowmap ? a.rowmap[seg0 + tok] : seg0 + tok;
-            xrow[n] = act + row * a.K + (KG / 4) * c;
+            for (int i = 0; i < D; ++i) {
+                if (i < ng) {
+                    wr[i] = ld_stream(wp + i * GS);
+                    if (SMODE != 0 && i % P == 0) sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + i));
+                }
+            }
         }
+        // stage the activation rows of tokens p0 .. p0 + ROWS - 1 (clamped)
+        for (int i = tid; i < ROWS * chunks; i += blockDim.x) {
+            const int row = i / chunks;
+            const int ch = i - row * chunks;
+            const int tok = min(p0 + row, M - 1);
+            const int64_t srow = a.rowmap ? a.rowmap[seg0 + tok] : seg0 + tok;
+            cp_async16(xs + row * rs + ch * 16, act + srow * a.K + g_lo * KG + ch * 8);
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        if (FOLD) {
+            if (SMODE == 1) {
+                // one thread per (chunk, row): fp32 sum in k order
+                constexpr int CK = P * KG;  // k per chunk
+                for (int i = tid; i < nch * ROWS; i += blockDim.x) {
+                    const int b = i / ROWS, row = i - b * ROWS;
+                    const uint4* src = reinterpret_cast<const uint4*>(xs + row * rs + b * CK * 2);
+                    float sum = 0.0f;
+#pragma unroll 4
+                    for (int q = 0; q < CK / 8; ++q) {
+                        const uint4 v = src[q];
+                        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            sum += __uint_as_float(u[h] << 16);
+                            sum += __uint_as_float(u[h] & 0xFFFF0000u);
+                        }
+                    }
+                    cs[i] = sum;
+                }
+            } else {
+                // one warp per row: strided partial sums, then a fixed shuffle tree
+                for (int row = warp; row < ROWS; row += kWarps) {
+                    const uint4* src = reinterpret_cast<const uint4*>(xs + row * rs);
+                    float sum = 0.0f;
+                    for (int q = lane; q < chunks; q += 32) {
+                        const uint4 v = src[q];
+                        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            sum += __uint_as_float(u[h] << 16);
+                            sum += __uint_as_float(u[h] & 0xFFFF0000u);
+                        }
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                    if (lane == 0) cs[row] = sum;
+                }
+            }
+            __syncthreads();
+        }
+
         float acc[NT][4], blk[NT][4];
 #pragma unroll
         for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[n][q] = blk[n][q] = 0.0f;
 
-        uint4 wr[D];
+        // one k-group: decode the lane's 16 bytes, 4 (int4) or 2 (int8) MMA
+        // k-steps per token tile. xg is this lane's activation run of the group.
+        auto group = [&](const uint4 w, const uint8_t* xg, const ScaleRaw<SF32> sc) {
+            uint4 xa[NT][2];
 #pragma unroll
-        for (int i = 0; i < D; ++i)
-            if (g_lo + i < g_hi) wr[i] = ld_stream(wtile + (g_lo + i) * kUnitBytes);
-
-        for (int64_t g = g_lo; g < g_hi; g += D) {
+            for (int n = 0; n < NT; ++n) {
+                xa[n][0] = *reinterpret_cast<const uint4*>(xg + n * 8 * rs);
+                if (BITS == 4) xa[n][1] = *reinterpret_cast<const uint4*>(xg + n * 8 * rs + 16);
+            }
+            float sa = 1.0f, sb = 1.0f;
+            if (SMODE == 2) sc.get(sa, sb);
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int i = 0; i < D; ++i) {
-                const int64_t gi = g + i;
-                if (gi < g_hi) {
-                    const uint4 w = wr[i];
-                    if (gi + D < g_hi) wr[i] = ld_stream(wtile + (gi + D) * kUnitBytes);
-                    // activations of this group: 16 (int4) or 8 (int8) bf16 per token tile
-                    uint4 xa[NT][2];
+            for (int j = 0; j < KSTEPS; ++j) {
+                uint32_t A[4];
+                if (BITS == 4) {
+                    if (FOLD) {
+                        constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;
+                        A[0] = (wv[j] & kMask) | kMagic;
+                        A[1] = ((wv[j] >> 4) & kMask) | kMagic;
+                        A[2] = ((wv[j] >> 8) & kMask) | kMagic;
+                        A[3] = ((wv[j] >> 12) & kMask) | kMagic;
+                    } else if (SF32) {
 #pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        xa[n][0] = ld_act(xrow[n] + gi * KG);
-                        if (BITS == 4) xa[n][1] = ld_act(xrow[n] + gi * KG + 8);
-                    }
-                    // scales of this lane's block
-                    float sa = 1.0f, sb = 1.0f;
-                    if (SMODE == 1) {
-                        const int64_t b = gi * KG / a.block_size;
-                        sa = load_scale(a.S, sbase + b * 16, SF32);
-                        sb = load_scale(a.S, sbase + b * 16 + 1, SF32);
-                    } else if (SMODE == 2) {
-                        const int64_t b = (gi * KG + (KG / 4) * c) / a.block_size;
-                        sa = load_scale(a.S, sbase + b * 16, SF32);
-                        sb = load_scale(a.S, sbase + b * 16 + 1, SF32);
-                    }
-                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-                    constexpr int KSTEPS = BITS == 4 ? 4 : 2;
-#pragma unroll
-                    for (int j = 0; j < KSTEPS; ++j) {
-                        uint32_t A[4];
-                        if (BITS == 4) {
-                            if (SMODE == 2 && SF32) {
-                                const uint32_t x = wv[j];
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const float sc = (q & 1) ? sb : sa;
-                                    A[q] = pack_bf2(nibble_centered(x, q) * sc,
-                                                    nibble_centered(x, q + 4) * sc);
-                                }
-                            } else {
-                                decode_int4(wv[j], A);
-                                if (SMODE == 2) {
-                                    const __nv_bfloat162 pa = __float2bfloat162_rn(sa);
-                                    const __nv_bfloat162 pb = __float2bfloat162_rn(sb);
-                                    const uint32_t ua = *reinterpret_cast<const uint32_t*>(&pa);
-                                    const uint32_t ub = *reinterpret_cast<const uint32_t*>(&pb);
-                                    A[0] = bf2_mul(A[0], ua);
-                                    A[1] = bf2_mul(A[1], ub);
-                                    A[2] = bf2_mul(A[2], ua);
-                                    A[3] = bf2_mul(A[3], ub);
-                                }
-                            }
-                        } else {
-                            const uint32_t lo = wv[2 * j], hi = wv[2 * j + 1];
-                            float f[8];
-#pragma unroll
-                            for (int m = 0; m < 4; ++m) {
-                                f[m] = byte_centered(lo, m);
-                                f[4 + m] = byte_centered(hi, m);
-                            }
-                            if (SMODE == 2) {
-                                if (SF32) {
-#pragma unroll
-                                    for (int m = 0; m < 8; ++m) f[m] *= ((m >> 1) & 1) ? sb : sa;
-                                } else {
-                                    const float ra = __bfloat162float(__float2bfloat16_rn(sa));
-                                    const float rb = __bfloat162float(__float2bfloat16_rn(sb));
-#pragma unroll
-                                    for (int m = 0; m < 8; ++m) f[m] *= ((m >> 1) & 1) ? rb : ra;
-                                }
-                            }
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) A[q] = pack_bf2(f[2 * q], f[2 * q + 1]);
+                        for (int q = 0; q < 4; ++q) {
+                            const float s = (q & 1) ? sb : sa;
+                            A[q] = pack_bf2(nibble_centered(wv[j], q) * s,
+                                            nibble_centered(wv[j], q + 4) * s);
                         }
-#pragma unroll
-                        for (int n = 0; n < NT; ++n) {
-                            const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xa[n][0]);
-                            // kstep j uses activation words 2j, 2j+1 of the lane's run
-                            if (SMODE == 1)
-                                mma_bf16(blk[n], A, xw[2 * j], xw[2 * j + 1]);
-                            else
-                                mma_bf16(acc[n], A, xw[2 * j], xw[2 * j + 1]);
-                        }
+                    } else {
+                        decode_int4(wv[j], A);
+                        const __nv_bfloat162 pa = __float2bfloat162_rn(sa);
+                        const __nv_bfloat162 pb = __float2bfloat162_rn(sb);
+                        const uint32_t ua = *reinterpret_cast<const uint32_t*>(&pa);
+                        const uint32_t ub = *reinterpret_cast<const uint32_t*>(&pb);
+                        A[0] = bf2_mul(A[0], ua);
+                        A[1] = bf2_mul(A[1], ub);
+                        A[2] = bf2_mul(A[2], ua);
+                        A[3] = bf2_mul(A[3], ub);
                     }
-                    if (SMODE == 1 && (((gi + 1) % gpb) == 0 || gi + 1 == g_hi)) {
+                } else {
+                    const uint32_t lo = wv[2 * j], hi = wv[2 * j + 1];
+                    float f[8];
 #pragma unroll
-                        for (int n = 0; n < NT; ++n) {
-                            acc[n][0] = fmaf(sa, blk[n][0], acc[n][0]);
-                            acc[n][1] = fmaf(sa, blk[n][1], acc[n][1]);
-                            acc[n][2] = fmaf(sb, blk[n][2], acc[n][2]);
-                            acc[n][3] = fmaf(sb, blk[n][3], acc[n][3]);
-                            blk[n][0] = blk[n][1] = blk[n][2] = blk[n][3] = 0.0f;
-                        }
+                    for (int m = 0; m < 4; ++m) {
+                        f[m] = byte_centered(lo, m);
+                        f[4 + m] = byte_centered(hi, m);
                     }
+                    if (SMODE == 2) {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) f[m] *= ((m >> 1) & 1) ? sb : sa;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) A[q] = pack_bf2(f[2 * q], f[2 * q + 1]);
+                }
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xa[n][0]);
+                    // kstep j uses activation words 2j, 2j+1 of the lane's run
+                    if (SMODE == 1)
+                        mma_bf16(blk[n], A, xw[2 * j], xw[2 * j + 1]);
+                    else
+                        mma_bf16(acc[n], A, xw[2 * j], xw[2 * j + 1]);
                 }
             }
-        }
+        };
+        // end of a scale chunk (SMODE 1): undo the fold, scale, accumulate
+        auto apply = [&](const ScaleRaw<SF32> sc, const float* csc) {
+            float sa, sb;
+            sc.get(sa, sb);
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            float v[4] = {acc[n][0], acc[n][1], acc[n][2], acc[n][3]};
-            if (SMODE == 0) {
-                v[0] *= s0;
-                v[1] *= s0;
-                v[2] *= s1;
-                v[3] *= s1;
+            for (int n = 0; n < NT; ++n) {
+                if (FOLD) {
+                    const float2 t = *reinterpret_cast<const float2*>(csc + 8 * n);
+                    blk[n][0] = fmaf(-kFoldOffset, t.x, blk[n][0]);
+                    blk[n][1] = fmaf(-kFoldOffset, t.y, blk[n][1]);
+                    blk[n][2] = fmaf(-kFoldOffset, t.x, blk[n][2]);
+                    blk[n][3] = fmaf(-kFoldOffset, t.y, blk[n][3]);
+                }
+                acc[n][0] = fmaf(sa, blk[n][0], acc[n][0]);
+                acc[n][1] = fmaf(sa, blk[n][1], acc[n][1]);
+                acc[n][2] = fmaf(sb, blk[n][2], acc[n][2]);
+                acc[n][3] = fmaf(sb, blk[n][3], acc[n][3]);
+                blk[n][0] = blk[n][1] = blk[n][2] = blk[n][3] = 0.0f;
             }
-            epilogue(a, rt, r0, c, seg0, M, p0 + 8 * n, v, split, true);
+        };
+
+        if (active) {
+            const uint8_t* wn = wp + D * GS;                      // loads run D groups ahead
+            const uint8_t* xp = xs + r0 * rs + (KG / 4) * c * 2;  // this lane's run, group 0
+            const float* csp = cs + 2 * c;                        // chunk 0, tokens 2c, 2c+1
+            ScaleRaw<SF32> scur = sr[0];
+            int g = 0;  // group relative to g_lo
+            // steady rounds: every prefetch is in range
+            for (; g + 2 * D <= ng; g += D) {
+#pragma unroll
+                for (int i = 0; i < D; ++i) {
+                    const uint4 w = wr[i];
+                    wr[i] = ld_stream(wn + i * GS);
+                    if (SMODE != 0 && i % P == 0) {
+                        scur = sr[i / P];
+                        sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + D));
+                    }
+                    group(w, xp + i * KG * 2, scur);
+                    if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
+                }
+                wn += D * GS;
+                xp += D * KG * 2;
+                csp += (D / P) * ROWS;
+            }
+            // drain round: prefetch only what remains
+            if (g + D <= ng) {
+#pragma unroll
+                for (int i = 0; i < D; ++i) {
+                    const uint4 w = wr[i];
+                    const bool more = g + i + D < ng;
+                    if (more) wr[i] = ld_stream(wn + i * GS);
+                    if (SMODE != 0 && i % P == 0) {
+                        scur = sr[i / P];
+                        if (more) sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + D));
+                    }
+                    group(w, xp + i * KG * 2, scur);
+                    if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
+                }
+                g += D;
+                xp += D * KG * 2;
+                csp += (D / P) * ROWS;
+            }
+            // tail: fewer than D groups left, all loaded
+#pragma unroll
+            for (int i = 0; i < D; ++i) {
+                if (g + i < ng) {
+                    if (SMODE != 0 && i % P == 0) scur = sr[i / P];
+                    group(wr[i], xp + i * KG * 2, scur);
+                    if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
+                }
+            }
+
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                float v[4] = {acc[n][0], acc[n][1], acc[n][2], acc[n][3]};
+                if (SMODE == 0) {
+                    if (FOLD) {
+                        const float2 t = *reinterpret_cast<const float2*>(cs + 8 * n + 2 * c);
+                        v[0] = fmaf(-kFoldOffset, t.x, v[0]);
+                        v[1] = fmaf(-kFoldOffset, t.y, v[1]);
+                        v[2] = fmaf(-kFoldOffset, t.x, v[2]);
+                        v[3] = fmaf(-kFoldOffset, t.y, v[3]);
+                    }
+                    v[0] *= s0;
+                    v[1] *= s0;
+                    v[2] *= s1;
+                    v[3] *= s1;
+                }
+                epilogue(a, rt, r0, c, seg0, M, p0 + 8 * n, v, split, true);
+            }
         }
+        __syncthreads();  // the next pass restages xs
     }
 }
 
@@ -367,7 +556,9 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
     const int r0 = lane >> 2, c = lane & 3;
     const int e = blockIdx.y, split = blockIdx.z;
     const int64_t nrt = a.N / kTileRows;
-    const int64_t rt = (int64_t)blockIdx.x * kWarps + warp;
+    const int64_t nrb = padded_rows(a.N) / kBlockRows;
+    const int64_t rb = blockIdx.x;
+    const int64_t rt = rb * kTilesPerBlock + warp;
     if (rt >= nrt) return;
     const int64_t seg0 = a.offsets[e];
     const int M = a.offsets[e + 1] - int(seg0);
@@ -376,8 +567,10 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
     const int64_t nsb = a.block_size > 0 ? a.K / a.block_size : 1;
     int64_t g_lo, g_hi;
     split_range(ngr, a.splits, split, 1, g_lo, g_hi);
-    const uint8_t* wtile = a.W + ((int64_t)e * nrt + rt) * ngr * kUnitBytes + lane * 16;
-    const int64_t sbase = ((int64_t)e * nrt + rt) * nsb * 16 + 2 * r0;
+    const uint8_t* wtile =
+        a.W + (((int64_t)e * nrb + rb) * ngr * kTilesPerBlock + warp) * kUnitBytes + lane * 16;
+    constexpr int64_t kGroupStride = (int64_t)kTilesPerBlock * kUnitBytes;
+    const int64_t sbase = (((int64_t)e * nrb + rb) * nsb * kTilesPerBlock + warp) * 16 + 2 * r0;
     const float* act = (const float*)a.act;
     const bool sf32 = !a.scale_bf16;
 
@@ -394,7 +587,7 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
 #pragma unroll
         for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = 0.0f;
         for (int64_t g = g_lo; g < g_hi; ++g) {
-            const uint4 w = *reinterpret_cast<const uint4*>(wtile + g * kUnitBytes);
+            const uint4 w = *reinterpret_cast<const uint4*>(wtile + g * kGroupStride);
             const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
             // decode the lane's 2 x KL codes into (row, actual k) order
             float q[2][KL];
@@ -415,8 +608,8 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
                     }
             }
             const int64_t b = a.block_size > 0 ? (g * KG + KL * c) / a.block_size : 0;
-            const float sa = load_scale(a.S, sbase + b * 16, sf32);
-            const float sb = load_scale(a.S, sbase + b * 16 + 1, sf32);
+            const float sa = load_scale(a.S, sbase + b * 128, sf32);
+            const float sb = load_scale(a.S, sbase + b * 128 + 1, sf32);
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
                 float pa = 0.0f, pb = 0.0f;
@@ -459,23 +652,82 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
     }
 }
 
-template <int BITS, int SMODE, bool SF32>
-cudaError_t launch_nt(const FfnArgs& a, dim3 grid, cudaStream_t st) {
-    switch (a.nt) {
-        case 1: ffn_decode_kernel<BITS, SMODE, SF32, 1><<<grid, kWarps * 32, 0, st>>>(a); break;
-        case 2: ffn_decode_kernel<BITS, SMODE, SF32, 2><<<grid, kWarps * 32, 0, st>>>(a); break;
-        default: ffn_decode_kernel<BITS, SMODE, SF32, 4><<<grid, kWarps * 32, 0, st>>>(a); break;
-    }
+template <int BITS, int SMODE, bool SF32, int NT, int P>
+cudaError_t launch_one(const FfnArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
+    ffn_decode_kernel<BITS, SMODE, SF32, NT, P><<<grid, kWarps * 32, smem, st>>>(a);
     return cudaGetLastError();
 }
 
-template <int BITS, int SMODE>
-cudaError_t launch_sf(const FfnArgs& a, dim3 grid, cudaStream_t st) {
-    return a.scale_bf16 ? launch_nt<BITS, SMODE, false>(a, grid, st)
-                        : launch_nt<BITS, SMODE, true>(a, grid, st);
+template <int BITS, int SMODE, bool SF32, int P>
+cudaError_t launch_nt(const FfnArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
+    switch (a.nt) {
+        case 1: return launch_one<BITS, SMODE, SF32, 1, P>(a, grid, smem, st);
+        case 2: return launch_one<BITS, SMODE, SF32, 2, P>(a, grid, smem, st);
+        default: return launch_one<BITS, SMODE, SF32, 4, P>(a, grid, smem, st);
+    }
+}
+
+template <int BITS, int SMODE, int P>
+cudaError_t launch_sf(const FfnArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
+    return a.scale_bf16 ? launch_nt<BITS, SMODE, false, P>(a, grid, smem, st)
+                        : launch_nt<BITS, SMODE, true, P>(a, grid, smem, st);
+}
+
+template <int BITS, int SMODE, bool SF32, int P>
+cudaError_t raise_smem_nt() {
+    const int lim = int(kDecodeSmemLimit);
+    cudaError_t e = cudaFuncSetAttribute(ffn_decode_kernel<BITS, SMODE, SF32, 1, P>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ffn_decode_kernel<BITS, SMODE, SF32, 2, P>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ffn_decode_kernel<BITS, SMODE, SF32, 4, P>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    return e;
+}
+
+template <int BITS, int SMODE, int P>
+cudaError_t raise_smem_sf() {
+    cudaError_t e = raise_smem_nt<BITS, SMODE, false, P>();
+    return e == cudaSuccess ? raise_smem_nt<BITS, SMODE, true, P>() : e;
+}
+
+// groups per scale application for SMODE 1
+int chunk_groups(int bits, int block_size) {
+    const int gpb = block_size / kgroup_of(bits);
+    return gpb >= kRing ? kRing : gpb;
 }
 
 }  // namespace
+
+int64_t decode_smem_bytes(int64_t K, int bits, int block_size, int splits, int nt) {
+    const int kg = kgroup_of(bits);
+    const int64_t ngr = K / kg;
+    const int64_t gpb = (block_size >= kg) ? block_size / kg : 1;
+    const int64_t nblk = (ngr + gpb - 1) / gpb;
+    const int64_t per = (nblk + splits - 1) / splits;
+    const int64_t groups = std::min<int64_t>(ngr, per * gpb);
+    const int64_t sums = (block_size >= kg) ? groups / chunk_groups(bits, block_size) : 1;
+    return int64_t(8) * nt * (staged_row_bytes(groups * kg) + 4 * sums);
+}
+
+cudaError_t prepare_ffn_decode() {
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = raise_smem_sf<4, 0, 1>();
+    if (e == cudaSuccess) e = raise_smem_sf<4, 1, 1>();
+    if (e == cudaSuccess) e = raise_smem_sf<4, 1, 2>();
+    if (e == cudaSuccess) e = raise_smem_sf<4, 1, 4>();
+    if (e == cudaSuccess) e = raise_smem_sf<4, 1, 8>();
+    if (e == cudaSuccess) e = raise_smem_sf<4, 2, 1>();
+    if (e == cudaSuccess) e = raise_smem_sf<8, 0, 1>();
+    if (e == cudaSuccess) e = raise_smem_sf<8, 1, 1>();
+    if (e == cudaSuccess) e = raise_smem_sf<8, 1, 2>();
+    if (e == cudaSuccess) e = raise_smem_sf<8, 1, 4>();
+    if (e == cudaSuccess) e = raise_smem_sf<8, 1, 8>();
+    if (e == cudaSuccess) e = raise_smem_sf<8, 2, 1>();
+    return e;
+}
 
 int scale_mode(int bits, int block_size) {
     if (block_size == 0) return 0;
@@ -483,22 +735,29 @@ int scale_mode(int bits, int block_size) {
 }
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st) {
-    const int64_t nrt = a.N / kTileRows;
-    dim3 grid(unsigned((nrt + kWarps - 1) / kWarps), unsigned(a.E), unsigned(a.splits));
+    dim3 grid(unsigned(padded_rows(a.N) / kBlockRows), unsigned(a.E), unsigned(a.splits));
+    const size_t smem = size_t(decode_smem_bytes(a.K, a.bits, a.block_size, a.splits, a.nt));
+    if (smem > kDecodeSmemLimit) return cudaErrorInvalidConfiguration;
     const int sm = scale_mode(a.bits, a.block_size);
+    const int P = sm == 1 ? chunk_groups(a.bits, a.block_size) : 1;
     if (a.bits == 4) {
-        if (sm == 0) return launch_sf<4, 0>(a, grid, st);
-        if (sm == 1) return launch_sf<4, 1>(a, grid, st);
-        return launch_sf<4, 2>(a, grid, st);
+        if (sm == 0) return launch_sf<4, 0, 1>(a, grid, smem, st);
+        if (sm == 2) return launch_sf<4, 2, 1>(a, grid, smem, st);
+        if (P == 1) return launch_sf<4, 1, 1>(a, grid, smem, st);
+        if (P == 2) return launch_sf<4, 1, 2>(a, grid, smem, st);
+        if (P == 4) return launch_sf<4, 1, 4>(a, grid, smem, st);
+        return launch_sf<4, 1, 8>(a, grid, smem, st);
     }
-    if (sm == 0) return launch_sf<8, 0>(a, grid, st);
-    if (sm == 1) return launch_sf<8, 1>(a, grid, st);
-    return launch_sf<8, 2>(a, grid, st);
+    if (sm == 0) return launch_sf<8, 0, 1>(a, grid, smem, st);
+    if (sm == 2) return launch_sf<8, 2, 1>(a, grid, smem, st);
+    if (P == 1) return launch_sf<8, 1, 1>(a, grid, smem, st);
+    if (P == 2) return launch_sf<8, 1, 2>(a, grid, smem, st);
+    if (P == 4) return launch_sf<8, 1, 4>(a, grid, smem, st);
+    return launch_sf<8, 1, 8>(a, grid, smem, st);
 }
 
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st) {
-    const int64_t nrt = a.N / kTileRows;
-    dim3 grid(unsigned((nrt + kWarps - 1) / kWarps), unsigned(a.E), unsigned(a.splits));
+    dim3 grid(unsigned(padded_rows(a.N) / kBlockRows), unsigned(a.E), unsigned(a.splits));
     if (a.bits == 4)
         ffn_simt_kernel<4><<<grid, kWarps * 32, 0, st>>>(a);
     else

@@ -35,24 +35,30 @@ __device__ __forceinline__ uint32_t code_at(const uint8_t* rowp, int64_t k, int 
 }
 
 // One thread writes the 16 bytes of one lane of one (row tile, k-group) unit.
+// Units are ordered [E][N/128 row blocks][K/KG groups][8 row tiles]; row tiles
+// past N (the padded tail of the last block) are written as zero codes.
 __global__ void pack_codes_kernel(PackArgs a) {
     const int64_t nrt = a.N / kTileRows;
+    const int64_t nrb = (nrt + kTilesPerBlock - 1) / kTilesPerBlock;
     const int kg = kgroup_of(a.bits);
     const int64_t ngr = a.K / kg;
-    const int64_t total = a.E * nrt * ngr * 32;
+    const int64_t total = a.E * nrb * ngr * kTilesPerBlock * 32;
     const int64_t src_rows = source_rows(a.mode, a.N, a.I);
     const int64_t row_bytes = a.K * a.bits / 8;
     for (int64_t id = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; id < total;
          id += (int64_t)gridDim.x * blockDim.x) {
         const int lane = int(id & 31);
         int64_t rest = id >> 5;
+        const int64_t tib = rest % kTilesPerBlock;
+        rest /= kTilesPerBlock;
         const int64_t g = rest % ngr;
         rest /= ngr;
-        const int64_t rt = rest % nrt;
-        const int64_t e = rest / nrt;
+        const int64_t rb = rest % nrb;
+        const int64_t e = rest / nrb;
+        const int64_t rt = rb * kTilesPerBlock + tib;
         const int r0 = lane >> 2, c = lane & 3;
-        uint32_t words[4];
-        if (a.bits == 4) {
+        uint32_t words[4] = {0u, 0u, 0u, 0u};
+        if (rt < nrt && a.bits == 4) {
             // word j, nibble p: row r0 + 8*(p&1), k = 64g + 16c + 4j + 2*((p>>1)&1) + (p>>2)
             for (int j = 0; j < 4; ++j) {
                 uint32_t w = 0;
@@ -66,7 +72,7 @@ __global__ void pack_codes_kernel(PackArgs a) {
                 }
                 words[j] = w;
             }
-        } else {
+        } else if (rt < nrt) {
             // kstep j (8 bytes), byte m: pair q = m/2 -> row r0 + 8*(q&1),
             // k = 32g + 8c + 4j + 2*(q>>1) + (m&1)
             for (int j = 0; j < 2; ++j) {
@@ -91,20 +97,33 @@ __global__ void pack_codes_kernel(PackArgs a) {
     }
 }
 
+// Scales: [E][N/128 row blocks][K/bs or 1][8 row tiles][16], the 16 entries
+// of a row tile in lane order (r0, r0 + 8) pairs; padded tiles hold zeros.
 __global__ void pack_scales_kernel(PackArgs a) {
     const int64_t nrt = a.N / kTileRows;
+    const int64_t nrb = (nrt + kTilesPerBlock - 1) / kTilesPerBlock;
     const int64_t nsb = a.block_size > 0 ? a.K / a.block_size : 1;
-    const int64_t total = a.E * nrt * nsb * 16;
+    const int64_t total = a.E * nrb * nsb * kTilesPerBlock * 16;
     const int64_t src_rows = source_rows(a.mode, a.N, a.I);
     for (int64_t id = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; id < total;
          id += (int64_t)gridDim.x * blockDim.x) {
         const int pos = int(id & 15);
         int64_t rest = id >> 4;
+        const int64_t tib = rest % kTilesPerBlock;
+        rest /= kTilesPerBlock;
         const int64_t b = rest % nsb;
         rest /= nsb;
-        const int64_t rt = rest % nrt;
-        const int64_t e = rest / nrt;
+        const int64_t rb = rest % nrb;
+        const int64_t e = rest / nrb;
+        const int64_t rt = rb * kTilesPerBlock + tib;
         const int rr = (pos >> 1) + 8 * (pos & 1);
+        if (rt >= nrt) {
+            if (a.scale_bf16)
+                ((uint16_t*)a.s_dst)[id] = 0;
+            else
+                ((float*)a.s_dst)[id] = 0.0f;
+            continue;
+        }
         const SrcRow s = source_row(a.mode, rt, rr, a.I);
         const int64_t src_idx = (e * src_rows + s.row) * nsb + b;
         if (a.scale_bf16) {
@@ -144,10 +163,11 @@ int grid_for(int64_t n, int threads) {
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t st) {
     const int th = 256;
-    const int64_t ncode = a.E * (a.N / kTileRows) * (a.K / kgroup_of(a.bits)) * 32;
+    const int64_t nrb = padded_rows(a.N) / kBlockRows;
+    const int64_t ncode = a.E * nrb * (a.K / kgroup_of(a.bits)) * kTilesPerBlock * 32;
     pack_codes_kernel<<<grid_for(ncode, th), th, 0, st>>>(a);
     const int64_t nsb = a.block_size > 0 ? a.K / a.block_size : 1;
-    pack_scales_kernel<<<grid_for(a.E * (a.N / kTileRows) * nsb * 16, th), th, 0, st>>>(a);
+    pack_scales_kernel<<<grid_for(a.E * nrb * nsb * kTilesPerBlock * 16, th), th, 0, st>>>(a);
     if (a.b_dst) pack_bias_kernel<<<grid_for(a.E * a.N, th), th, 0, st>>>(a);
     return cudaGetLastError();
 }

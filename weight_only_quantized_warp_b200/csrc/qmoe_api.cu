@@ -30,18 +30,24 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     p.path = bf16 ? kPathDecode : kPathSimt;
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size;
     if (p.path == kPathDecode) {
+        const int bits = c.expert_weight_bits, bs = c.block_size;
         const int64_t per_expert = ceil_div(std::max<int64_t>(p.R, 1), E);
         p.nt = per_expert <= 8 ? 1 : (per_expert <= 16 ? 2 : 4);
+        // FC1 runs unsplit; keep its staged rows small enough for two CTAs per SM
+        while (p.nt > 1 && decode_smem_bytes(H, bits, bs, 1, p.nt) > kDecodeSmemTarget) p.nt /= 2;
         // enough FC2 warps (one per 16-row tile per touched expert per split)
         // to give every SM several resident warps
         const int64_t touched = std::min<int64_t>(E, std::max<int64_t>(p.R, 1));
         const int64_t warps = touched * (H / kTileRows);
         const int64_t want = kSms * 48;
-        const int64_t ngr = I / kgroup_of(c.expert_weight_bits);
+        const int64_t ngr = I / kgroup_of(bits);
         int64_t s = ceil_div(want, warps);
         s = std::min<int64_t>(s, 8);
+        while (s < ngr && decode_smem_bytes(I, bits, bs, int(s), p.nt) > kDecodeSmemTarget) ++s;
         s = std::min<int64_t>(s, ngr);
         p.fc2_splits = int(std::max<int64_t>(s, 1));
+        p.ok = decode_smem_bytes(H, bits, bs, 1, p.nt) <= int64_t(kDecodeSmemLimit) &&
+               decode_smem_bytes(I, bits, bs, p.fc2_splits, p.nt) <= int64_t(kDecodeSmemLimit);
     }
     p.launches = 5;
     const size_t R = size_t(p.R);
@@ -207,6 +213,7 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return cuda_fail(h, err, "cudaGetDevice");
     err = prepare_route_permute();
+    if (err == cudaSuccess) err = prepare_ffn_decode();
     if (err != cudaSuccess) return cuda_fail(h, err, "prepare kernels");
 
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size, N1 = h->n1;
@@ -219,11 +226,12 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
     void *s1 = nullptr, *s2 = nullptr;
     float *b1 = nullptr, *b2 = nullptr;
     auto alloc = [&](void** p, size_t n) { return cudaMalloc(p, n < 16 ? 16 : n); };
-    if ((err = alloc((void**)&w1, size_t(E * N1 * H * bits / 8))) != cudaSuccess ||
-        (err = alloc(&s1, size_t(E * N1 * nsb1) * ssz)) != cudaSuccess ||
+    const int64_t P1 = padded_rows(N1), P2 = padded_rows(H);
+    if ((err = alloc((void**)&w1, size_t(E * P1 * H * bits / 8))) != cudaSuccess ||
+        (err = alloc(&s1, size_t(E * P1 * nsb1) * ssz)) != cudaSuccess ||
         (any_b1 && (err = alloc((void**)&b1, size_t(E * N1) * 4)) != cudaSuccess) ||
-        (err = alloc((void**)&w2, size_t(E * H * I * bits / 8))) != cudaSuccess ||
-        (err = alloc(&s2, size_t(E * H * nsb2) * ssz)) != cudaSuccess ||
+        (err = alloc((void**)&w2, size_t(E * P2 * I * bits / 8))) != cudaSuccess ||
+        (err = alloc(&s2, size_t(E * P2 * nsb2) * ssz)) != cudaSuccess ||
         (c.has_fc2_bias && (err = alloc((void**)&b2, size_t(E * H) * 4)) != cudaSuccess)) {
         free_pack(w1, s1, b1, w2, s2, b2);
         cudaGetLastError();
@@ -312,6 +320,8 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     if (reinterpret_cast<uintptr_t>(workspace) & 255)
         return fail(h, QMOE_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
     const Plan p = make_plan(*h, T);
+    if (!p.ok)
+        return fail(h, QMOE_UNSUPPORTED, "no kernel configuration fits this shape (hidden_size too large)");
     if (workspace_bytes < p.total)
         return fail(h, QMOE_INVALID_ARGUMENT, "workspace too small: %zu < %zu", workspace_bytes,
                     p.total);

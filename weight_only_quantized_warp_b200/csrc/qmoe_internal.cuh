@@ -10,32 +10,40 @@
 #include <mutex>
 #include <string>
 
-#include "../../include/qmoe.h"
+#include "qmoe.h"
 
 namespace qmoe {
 
 // ---------------------------------------------------------------------------
 // Packed weight layout ("fragment order").
 //
-// A weight W[N, K] of one expert (N output rows, K reduction) is stored as
-// [N/16 row tiles][K/KG k-groups][32 lanes][16 bytes], KG = 64 for 4-bit and
-// 32 for 8-bit codes, so one (row tile, k-group) unit is 512 contiguous bytes
-// and one row tile is contiguous along K. Lane L owns rows r0 = L/4 and
-// r0 + 8 of the tile and the k sub-range [KG/4 * (L%4), KG/4 * (L%4 + 1)) of
-// the group: exactly the operand fragments of an m16n8k16 bf16 MMA whose k
-// axis is permuted consistently for weights and activations (see
-// decode_fragments in ffn_decode.cu). Bytes are the page's codes, re-laid,
-// never decoded: the pack has the same size as the input.
+// A weight W[N, K] of one expert (N output rows, K reduction) is cut into row
+// tiles of 16 rows and k-groups of KG (64 for 4-bit codes, 32 for 8-bit). One
+// (row tile, k-group) unit is 512 bytes: lane L of a warp owns rows r0 = L/4
+// and r0 + 8 of the tile and the k sub-range [KG/4 * (L%4), KG/4 * (L%4 + 1))
+// of the group, 16 bytes -- exactly the operand fragments of an m16n8k16 bf16
+// MMA whose k axis is permuted the same way for weights and activations (see
+// ffn_decode.cu). Units are ordered [N/128 row blocks][K/KG groups][8 row
+// tiles], so a 128-row x KG slab (one tensor-core stage) is one contiguous
+// 4 KB run and a row tile walks K with a 4 KB stride. N is padded to a
+// multiple of 128 with zero codes. Bytes are the page's codes, re-laid,
+// never decoded.
 //
 // FC1 of a gated FFN is re-laid so that row tile t holds gate rows
 // i = 8t..8t+7 in its first 8 rows and the matching up rows in its last 8,
 // whatever the input layout (fused interleaved, fused concatenated, or fc1 +
-// fc3). Scales follow as [N/16][K/bs or 1][16] with the 16 entries in lane
-// order (r0, r0 + 8) pairs; biases as fp32 in packed row order.
+// fc3). Scales follow as [N/128][K/bs or 1][8 row tiles][16] with the 16
+// entries of a tile in lane order (r0, r0 + 8) pairs; biases as fp32 in
+// packed row order.
 // ---------------------------------------------------------------------------
 constexpr int kTileRows = 16;
+constexpr int kTilesPerBlock = 8;
+constexpr int kBlockRows = kTileRows * kTilesPerBlock;  // 128
 constexpr int kUnitBytes = 512;
 __host__ __device__ constexpr int kgroup_of(int bits) { return bits == 4 ? 64 : 32; }
+__host__ __device__ constexpr int64_t padded_rows(int64_t n) {
+    return (n + kBlockRows - 1) / kBlockRows * kBlockRows;
+}
 
 // Hot-path selection.
 enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2 };
@@ -46,6 +54,7 @@ struct Plan {
     int nt = 1;          // 8-token MMA n-tiles handled per pass (decode path)
     int fc2_splits = 1;  // split-K factor of FC2 (partials reduced by the combine)
     int launches = 0;
+    bool ok = true;      // a kernel configuration exists for this shape
     size_t off_idx = 0, off_w = 0, off_inv = 0, off_perm = 0, off_offsets = 0, off_status = 0,
            off_h = 0, off_o = 0, total = 0;
 };
@@ -124,6 +133,12 @@ struct FfnArgs {
     int nt;
 };
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
+// Shared memory of one decode CTA (staged activation rows) and its limit;
+// prepare_ffn_decode() raises the kernels' limit on the current device.
+constexpr size_t kDecodeSmemLimit = 200 * 1024;
+constexpr int64_t kDecodeSmemTarget = 112 * 1024;  // two CTAs per SM
+int64_t decode_smem_bytes(int64_t K, int bits, int block_size, int splits, int nt);
+cudaError_t prepare_ffn_decode();
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
 
 // Router-weighted combine with fc2 bias and shared output; sums the FC2

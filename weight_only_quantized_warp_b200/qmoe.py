@@ -15,7 +15,8 @@ import os
 from typing import Optional
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libqmoe.so")
+# QMOE_LIB may point at another build of the same library (same ABI).
+LIB_PATH = os.environ.get("QMOE_LIB") or os.path.join(HERE, "libqmoe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libqmoe.so is not built (run weight_only_quantized_warp_b200/build.py or "
