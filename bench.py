@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="mixtral_decode")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", type=int, default=None,
+                    help="force the expert-FFN kernels: 1 weight-streaming, 2 tcgen05 (default: by shape)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0,
                     help="tokens in the CPU-baseline sample (0: whole batch, capped by time)")
@@ -230,7 +232,7 @@ def run_ours(args):
         other = gen.make_inputs(dataclasses_replace(cfg), seed + 1000 * rank, **kw)
         inp.x, inp.logits, inp.shared = other.x, other.logits, other.shared
 
-    m = qmoe.QMoE(cfg, dev)
+    m = qmoe.QMoE(cfg, dev, path=args.path)
     m.set_weights_from(inp)
     x = qmoe.to_device(inp.x, dev)
     lg = qmoe.to_device(inp.logits, dev)
@@ -296,7 +298,9 @@ def run_ours(args):
         dist.barrier()
     per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(launches)]
                            for i in range(K)]).mean(axis=0)
-    names = ["route", "permute", "fc1", "fc2", "combine"][:launches]
+    path = qmoe.qmoe_path_for(h, T)
+    names = (["route", "permute", "gather", "fc1", "fc2", "combine"] if path == qmoe.PATH_TC
+             else ["route", "permute", "fc1", "fc2", "combine"])[:launches]
 
     # ---- end to end through the public call, host buffers, copies inside
     x_h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu())
@@ -350,18 +354,32 @@ def run_ours(args):
         return 0
 
     peaks, peaks_kind = load_peaks()
-    fc1_ms = float(per_kernel[2])
+    kms = dict(zip(names, [float(v) for v in per_kernel]))
+    fc1_ms = kms["fc1"]
     step_ms = ms / K
     tokens = T * world * K
     value = tokens / (ms / 1e3)
-    # dominant kernel by algorithmic work: FC1 (gate + up rows) here
+    # dominant kernel by algorithmic work: FC1 (gate + up rows); its bound is
+    # the slower of its bytes at HBM bandwidth and its FLOPs at bf16 peak
     hbm_peak = float(peaks["hbm_gbs"])
-    achieved = alg["fc1_bytes"] / (fc1_ms / 1e3) / 1e9
-    tr = traffic_record("fc1_decode_" + args.workload)
-    roofline = {"bound": "hbm", "kernel": "ffn_decode_kernel (FC1 + SwiGLU)",
-                "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                "peak_kind": peaks_kind, "traffic": tr["bytes_per_launch"] if tr else None,
-                "algorithmic_bytes": alg["fc1_bytes"], "avg_launch_ms": fc1_ms}
+    tc_peak = float(peaks["bf16_tflops"])
+    fc1_flops = 2.0 * cfg.T * cfg.k * (cfg.n1 + (cfg.I if cfg.has_fc3 else 0)) * cfg.H
+    t_hbm = alg["fc1_bytes"] / (hbm_peak * 1e9)
+    t_tc = fc1_flops / (tc_peak * 1e12)
+    kname = "ffn_tc_kernel (FC1 + SwiGLU)" if path == qmoe.PATH_TC else "ffn_decode_kernel (FC1 + SwiGLU)"
+    tr = traffic_record(("fc1_tc_" if path == qmoe.PATH_TC else "fc1_decode_") + args.workload)
+    if t_hbm >= t_tc:
+        achieved = alg["fc1_bytes"] / (fc1_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "algorithmic_bytes": alg["fc1_bytes"]}
+    else:
+        achieved = fc1_flops / (fc1_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": achieved / tc_peak, "algorithmic_flops": fc1_flops}
+    roofline.update({"kernel": kname, "peak_kind": peaks_kind + (" (burst bf16)" if roofline["bound"] == "tensor" else ""),
+                     "traffic": tr["bytes_per_launch"] if tr else None, "avg_launch_ms": fc1_ms,
+                     "roofline_frac_of_step": max(alg["total_bytes"] / (hbm_peak * 1e9),
+                                                  alg["flops"] / (tc_peak * 1e12)) / (ms / K / 1e3)})
     whole = alg["total_bytes"] / (step_ms / 1e3) / 1e9
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -372,7 +390,7 @@ def run_ours(args):
             "step": {"hbm_gbs": whole, "tflops": alg["flops"] / (step_ms / 1e3) / 1e12,
                      "hbm_frac": whole / hbm_peak, "experts_touched": alg["touched"],
                      "algorithmic_bytes": alg["total_bytes"],
-                     "kernel_ms": dict(zip(names, [float(v) for v in per_kernel]))},
+                     "kernel_ms": kms, "path": path},
             "cpu_baseline": cpu,
             "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

@@ -223,6 +223,17 @@ QMOE_API const char* qmoe_status_string(qmoe_status s);
  * the handle. */
 QMOE_API const char* qmoe_last_error(const qmoe_handle* h);
 
+/* Tunable options (qmoe_set_option). QMOE_OPT_PATH selects the expert-FFN
+ * kernels for bf16 activations: -1 (default) chooses by shape, 1 forces the
+ * weight-streaming decode kernels, 2 the tcgen05 grouped GEMM. fp32
+ * activations always take the fp32 path (0). */
+enum { QMOE_OPT_PATH = 1 };
+
+/* qmoe_set_option -- set a tunable option on the handle. QMOE_INVALID_ARGUMENT
+ * for an unknown option or value. Not thread-safe against concurrent
+ * qmoe_forward calls on the same handle. */
+QMOE_API qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t value);
+
 /* The forward path qmoe_forward takes for T tokens: 0 = fp32 SIMT path,
  * 1 = weight-streaming decode path (mma.sync), 2 = tcgen05 grouped GEMM.
  * -1 for a NULL handle. */

@@ -43,11 +43,13 @@ class GpuRun:
     path: int
 
 
-def run_gpu(inp: gen.MoEInputs, device="cuda:0", repeat: int = 1) -> GpuRun:
+def run_gpu(inp: gen.MoEInputs, device="cuda:0", repeat: int = 1, path=None) -> GpuRun:
+    """path: None (chosen by shape), 1 (weight-streaming kernels) or 2
+    (tcgen05 grouped GEMM); ignored for fp32 activations."""
     import torch
     from weight_only_quantized_warp_b200 import qmoe
     c = inp.cfg
-    m = qmoe.QMoE(c, device)
+    m = qmoe.QMoE(c, device, path=path if c.act_dtype == gen.DT_BF16 else None)
     m.set_weights_from(inp)
     x = qmoe.to_device(inp.x, device)
     lg = qmoe.to_device(inp.logits, device)
@@ -68,6 +70,8 @@ def run_gpu(inp: gen.MoEInputs, device="cuda:0", repeat: int = 1) -> GpuRun:
     hid = torch.empty((max(R, 1), c.I), dtype=x.dtype, device=device)
     qmoe.qmoe_debug_hidden(m.handle, T, ws, hid)
     torch.cuda.synchronize()
+    status = qmoe.qmoe_read_device_status(m.handle, ws)
+    assert status == qmoe.QMOE_OK, f"device status {status}"
     path = qmoe.qmoe_path_for(m.handle, T)
     return GpuRun(to_numpy(y), idx.cpu().numpy(), w.cpu().numpy(), off.cpu().numpy(),
                   perm.cpu().numpy()[:R], inv.cpu().numpy(), to_numpy(hid)[:R], path)

@@ -70,11 +70,18 @@ CASES = {
 }
 
 
+PATH_DECODE, PATH_TC = 1, 2
+
+
+@pytest.mark.parametrize("path", [PATH_DECODE, PATH_TC], ids=["decode", "tc"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_parity_small(cuda_device, name):
+def test_parity_small(cuda_device, name, path):
     cfg = _cfg(**CASES[name])
+    if cfg.act_dtype == gen.DT_F32 and path == PATH_TC:
+        pytest.skip("fp32 activations always take the fp32 path")
     inp = gen.make_inputs(cfg, seed=100 + list(CASES).index(name), bias_std=0.1)
-    g = run_gpu(inp)
+    g = run_gpu(inp, path=path)
+    assert g.path == (0 if cfg.act_dtype == gen.DT_F32 else path)
     check_full(inp, g)
 
 
@@ -113,11 +120,12 @@ def test_zero_tokens_is_a_noop(cuda_device):
     torch.cuda.synchronize()
 
 
-def test_repeated_forward_is_bitwise_deterministic(cuda_device):
+@pytest.mark.parametrize("path", [PATH_DECODE, PATH_TC], ids=["decode", "tc"])
+def test_repeated_forward_is_bitwise_deterministic(cuda_device, path):
     cfg = _cfg(T=50, bits=4, block_size=128, H=384, I=640)
     inp = gen.make_inputs(cfg, seed=8)
-    a = run_gpu(inp)
-    b = run_gpu(inp, repeat=3)
+    a = run_gpu(inp, path=path)
+    b = run_gpu(inp, repeat=3, path=path)
     np.testing.assert_array_equal(a.y, b.y)
     np.testing.assert_array_equal(a.hidden, b.hidden)
 
@@ -146,16 +154,17 @@ def _sample(T, n=8, seed=0):
     return np.sort(rng.choice(T, size=min(n, T), replace=False))
 
 
+@pytest.mark.parametrize("path", [None, PATH_DECODE, PATH_TC], ids=["auto", "decode", "tc"])
 @pytest.mark.parametrize("name", ["mixtral_decode", "gpt_oss", "deepseek"])
-def test_full_size_configs(cuda_device, name):
+def test_full_size_configs(cuda_device, name, path):
     cfg, seed, kw = gen.workload(name)
     inp = gen.make_inputs(cfg, seed, **kw)
-    g = run_gpu(inp)
+    g = run_gpu(inp, path=path)
     tokens = np.arange(cfg.T) if cfg.T <= 8 else _sample(cfg.T)
     check_sampled(inp, g, tokens)
 
 
-@pytest.mark.parametrize("bits,T", [(4, 1), (4, 16), (8, 1), (8, 128)])
+@pytest.mark.parametrize("bits,T", [(4, 1), (4, 16), (8, 1), (8, 128), (4, 1024)])
 def test_sweep_configs(cuda_device, bits, T):
     cfg, seed, kw = gen.sweep(bits, T)
     inp = gen.make_inputs(cfg, seed, **kw)

@@ -327,13 +327,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
                 }
             }
         }
-        // stage the activation rows of tokens p0 .. p0 + ROWS - 1 (clamped)
-        for (int i = tid; i < ROWS * chunks; i += blockDim.x) {
-            const int row = i / chunks;
-            const int ch = i - row * chunks;
+        // stage the activation rows of tokens p0 .. p0 + ROWS - 1 (clamped):
+        // one warp per row, lanes over its 16-byte chunks
+        for (int row = warp; row < ROWS; row += kWarps) {
             const int tok = min(p0 + row, M - 1);
             const int64_t srow = a.rowmap ? a.rowmap[seg0 + tok] : seg0 + tok;
-            cp_async16(xs + row * rs + ch * 16, act + srow * a.K + g_lo * KG + ch * 8);
+            const __nv_bfloat16* src = act + srow * a.K + g_lo * KG;
+            uint8_t* dst = xs + row * rs;
+            for (int ch = lane; ch < chunks; ch += 32) cp_async16(dst + ch * 16, src + ch * 8);
         }
         cp_async_wait_all();
         __syncthreads();
@@ -482,13 +483,12 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
             for (; g + 2 * D <= ng; g += D) {
 #pragma unroll
                 for (int i = 0; i < D; ++i) {
-                    const uint4 w = wr[i];
+                    // use slot i, then refill it (no register copy of the old value)
+                    if (SMODE != 0 && i % P == 0) scur = sr[i / P];
+                    group(wr[i], xp + i * KG * 2, scur);
                     wr[i] = ld_stream(wn + i * GS);
-                    if (SMODE != 0 && i % P == 0) {
-                        scur = sr[i / P];
-                        sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + D));
-                    }
-                    group(w, xp + i * KG * 2, scur);
+                    if (SMODE != 0 && i % P == P - 1)
+                        sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + 1 - P + D));
                     if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
                 }
                 wn += D * GS;
@@ -499,14 +499,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
             if (g + D <= ng) {
 #pragma unroll
                 for (int i = 0; i < D; ++i) {
-                    const uint4 w = wr[i];
-                    const bool more = g + i + D < ng;
-                    if (more) wr[i] = ld_stream(wn + i * GS);
-                    if (SMODE != 0 && i % P == 0) {
-                        scur = sr[i / P];
-                        if (more) sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + D));
-                    }
-                    group(w, xp + i * KG * 2, scur);
+                    if (SMODE != 0 && i % P == 0) scur = sr[i / P];
+                    group(wr[i], xp + i * KG * 2, scur);
+                    if (g + i + D < ng) wr[i] = ld_stream(wn + i * GS);
+                    if (SMODE != 0 && i % P == P - 1 && g + i + 1 - P + D < ng)
+                        sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + 1 - P + D));
                     if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
                 }
                 g += D;

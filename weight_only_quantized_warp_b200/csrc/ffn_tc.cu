@@ -1,0 +1,716 @@
+// ffn_tc.cu -- expert FFN layers on the 5th-generation tensor cores
+// (tcgen05.mma with TMEM accumulators), sm_100a.
+//
+// Each linear is y = x @ dequant(W).T + b ("QLinearWoQ" page, class summary)
+// over the rows routed to one expert; the packed weights are decoded one
+// 128 x 64 tile at a time inside the GEMM mainloop and never written out
+// dense in global memory ("ClikaRT::nn::QMoEWoQ", class description: each
+// expert weight decodes one block at a time inside the GEMM dot). FC1 applies
+// the QMoE page's gated activation in its epilogue.
+//
+// Operand roles ("swap AB"): the MMA's M dimension is 128 weight rows, its N
+// dimension the routed tokens of one expert (a multiple of 16, up to 256), so
+// a small expert segment wastes no tensor work on padding rows.
+//
+// Warp roles of one persistent CTA (448 threads, one CTA per SM):
+//   warps 0-7   dequantise: packed codes (shared) -> bf16 A tile in the
+//               128-byte-swizzled K-major layout the MMA descriptor reads
+//   warp 8      producer: one bulk copy of the packed 128 x 64 tile (4 KB
+//               int4, 8 KB int8), one of its scales, one TMA tile of the
+//               activations (N rows x 64 bf16, 128-byte swizzle)
+//   warp 9      allocates TMEM and issues tcgen05.mma from one thread
+//   warps 10-13 epilogue: TMEM -> registers (tcgen05.ld), scale / bias /
+//               activation, global stores
+// Stages cycle through an S-deep ring guarded by mbarriers (full: copies
+// landed; deq: A tile written; empty: the MMAs reading the stage are done);
+// two TMEM accumulators let the epilogue of one work item overlap the
+// mainloop of the next. Every wait is bounded: after about two seconds the
+// kernel records QMOE_TIMEOUT in the workspace status word, every role
+// leaves its loop, and the CTA frees its TMEM and exits.
+//
+// Scales: a K-block scale is multiplied into the decoded weight (one bf16
+// rounding of (q - z) * s); per-column scales (block_size 0) leave exact
+// integer weights in the MMA and are applied in fp32 in the epilogue.
+#include <cuda.h>
+
+#include "qmoe_internal.cuh"
+
+namespace qmoe {
+namespace {
+
+constexpr int kDeqWarps = 8;
+constexpr int kWarpProd = 8;
+constexpr int kWarpMma = 9;
+constexpr int kWarpEpi0 = 10;
+constexpr int kTcThreads = 14 * 32;
+constexpr int kBK = 64;                           // k per stage
+constexpr int kATile = kBlockRows * kBK * 2;      // 16 KB of bf16
+constexpr int kScaleBytesMax = 4 * kTilesPerBlock * 16 * 4;  // 4 blocks of fp32 pairs
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+struct TcArgs {
+    const uint8_t* W;
+    const void* S;
+    const float* bias;       // FC1, packed row order, or nullptr
+    const int32_t* offsets;  // [E + 1]
+    void* out;               // FC1: h [R, I] bf16; FC2: partials [splits, R, N] fp32
+    int32_t* status;         // workspace status word
+    int64_t N, K, R;
+    int E, block_size, gated, is_fc1, act_type;
+    float alpha, beta, limit;
+    int splits, scale_bf16, bn;
+};
+
+// ------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return uint32_t(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.b32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on a phase parity. Returns false (after raising the CTA's
+// abort flag and the workspace status) when the wait gives up or another role
+// already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = now_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try(bar, parity)) return true;
+        if ((spin & 255u) == 0u) {
+            if (*abort_flag) return false;
+            if (now_ns() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                atomicExch(status, int32_t(QMOE_TIMEOUT));
+                return false;
+            }
+        }
+    }
+}
+
+// Wait by a whole warp: every lane polls, and the warp continues only if all
+// lanes saw the phase complete (a timeout in any lane stops the whole warp).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+    const bool ok = mbar_wait(bar, parity, abort_flag, status);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                       uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3}], [%4];" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
+// 1024 bytes stacked along M/N (stride 1024), version 1 for sm_100.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t(1) << 16;             // leading offset: unused for swizzled K-major
+    d |= uint64_t(1024 >> 4) << 32;     // stride offset between 8-row atoms
+    d |= uint64_t(1) << 46;             // descriptor version
+    d |= uint64_t(2) << 61;             // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: kind::f16, bf16 A and B (K-major), fp32 D, M = 128.
+__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// --------------------------------------------------------------- arithmetic
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bf2_bcast(float s) {
+    __nv_bfloat162 r = __float2bfloat162_rn(s);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
+__device__ __forceinline__ float act_plain(int t, float a) {
+    switch (t) {
+        case QMOE_ACT_RELU: return fmaxf(a, 0.0f);
+        case QMOE_ACT_GELU: return 0.5f * a * (1.0f + erff(a * 0.70710678118654752f));
+        case QMOE_ACT_SILU: return a * sigmoidf_(a);
+        default: return a;
+    }
+}
+__device__ __forceinline__ float act_gated(int t, float g, float u, float alpha, float beta,
+                                           float limit) {
+    if (t == QMOE_ACT_SWIGLU) {
+        g = fminf(g, limit);
+        u = fminf(fmaxf(u, -limit), limit);
+        return (u + beta) * g * sigmoidf_(alpha * g);
+    }
+    return act_plain(t, g) * u;
+}
+
+// Byte offset of element (row, k) inside an A tile: 8-row atoms of 1024 bytes,
+// 16-byte chunks of a 128-byte row XOR-swizzled by the row's index in its atom.
+__device__ __forceinline__ uint32_t a_off(int row, int k) {
+    return uint32_t((row >> 3) * 1024 + (row & 7) * 128 + ((((k >> 3) ^ (row & 7))) << 4) + (k & 7) * 2);
+}
+
+// ------------------------------------------------------------ work items
+struct Item {
+    int e, rb, tt, split;
+    int64_t seg0;
+    int M;      // rows routed to the expert
+    int rows;   // rows of this token tile
+    int ks_lo, ks_hi;
+};
+
+// Items are ordered expert, row block, token tile, split, so CTAs working on
+// neighbouring items share weight blocks in L2.
+__device__ __forceinline__ Item item_at(int i, const int* prefix, const TcArgs& a, int nrb, int nks) {
+    int lo = 0, hi = a.E;  // largest e with prefix[e] <= i
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= i) lo = mid; else hi = mid;
+    }
+    Item it;
+    it.e = lo;
+    it.seg0 = a.offsets[lo];
+    it.M = a.offsets[lo + 1] - int(it.seg0);
+    const int ntt = (it.M + a.bn - 1) / a.bn;
+    int rem = i - prefix[lo];
+    const int per_rb = ntt * a.splits;
+    it.rb = rem / per_rb;
+    rem -= it.rb * per_rb;
+    it.tt = rem / a.splits;
+    it.split = rem - it.tt * a.splits;
+    it.rows = min(a.bn, it.M - it.tt * a.bn);
+    it.ks_lo = int((int64_t(it.split) * nks) / a.splits);
+    it.ks_hi = int((int64_t(it.split + 1) * nks) / a.splits);
+    return it;
+}
+
+template <int BITS, bool PERCOL, int BNMAX, int STAGES>
+struct TcCfg {
+    static constexpr int kPacked = kBlockRows * kBK * BITS / 8;  // 4 KB or 8 KB
+    static constexpr int kB = BNMAX * 128;
+    static constexpr int kStage = kATile + kB + kPacked + kScaleBytesMax;
+    static constexpr int kTmemCols = (2 * BNMAX < 32) ? 32 : 2 * BNMAX;
+    static constexpr int kBarOff = STAGES * kStage;
+    static constexpr int kSmem = kBarOff + 1024 + 4 * 260 + 1024;  // barriers, prefix, align slack
+};
+
+template <int BITS, bool PERCOL, int BNMAX, int STAGES>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    ffn_tc_kernel(const __grid_constant__ CUtensorMap bmap, const TcArgs a) {
+    using C = TcCfg<BITS, PERCOL, BNMAX, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    uint8_t* bar_area = smem + C::kBarOff;
+    uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
+    uint64_t* deq = full + STAGES;
+    uint64_t* empty = deq + STAGES;
+    uint64_t* accf = empty + STAGES;
+    uint64_t* acce = accf + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* prefix = reinterpret_cast<int*>(tmem_slot + 4);  // [E + 1]
+
+    const int nrb = int(padded_rows(a.N) / kBlockRows);
+    const int nks = int(a.K / kBK);
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&deq[s]), kDeqWarps);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&accf[b]), 1);
+            mbar_init(smem_u32(&acce[b]), 4);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {  // item counts per expert, exclusive prefix
+        int carry = 0;
+        for (int e0 = 0; e0 < a.E; e0 += 32) {
+            const int e = e0 + lane;
+            int v = 0;
+            if (e < a.E) {
+                const int M = a.offsets[e + 1] - a.offsets[e];
+                v = ((M + a.bn - 1) / a.bn) * nrb * a.splits;
+            }
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (e < a.E) prefix[e] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) prefix[a.E] = carry;
+    }
+    if (warp == kWarpMma) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(C::kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int total = prefix[a.E];
+    const int nsb = a.block_size > 0 ? int(a.K / a.block_size) : 1;
+    const int ssz = a.scale_bf16 ? 2 : 4;
+    // scale blocks covered by one 64-k stage, and the stage's scale bytes
+    const int sblk = PERCOL ? 0 : (a.block_size >= kBK ? 1 : kBK / a.block_size);
+    const uint32_t sbytes = uint32_t(sblk * kTilesPerBlock * 16 * ssz);
+
+    if (warp == kWarpProd) {
+        // ------------------------------------------------------- producer
+        if (lane == 0) {
+            int st = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+                const Item it = item_at(i, prefix, a, nrb, nks);
+                const int ngr = int(a.K / kgroup_of(BITS));
+                for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
+                    if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                    uint8_t* sb = smem + st * C::kStage;
+                    const uint32_t fb = smem_u32(&full[st]);
+                    mbar_expect_tx(fb, uint32_t(C::kPacked + C::kB) + sbytes);
+                    const int g = ks * (kBK / kgroup_of(BITS));  // first k-group of the stage
+                    const uint8_t* src = a.W + ((int64_t(it.e) * nrb + it.rb) * ngr + g) * int64_t(kTilesPerBlock) * kUnitBytes;
+                    bulk_g2s(smem_u32(sb + kATile + C::kB), src, C::kPacked, fb);
+                    if (!PERCOL) {
+                        const int b0 = (ks * kBK) / a.block_size;
+                        const int64_t sidx = ((int64_t(it.e) * nrb + it.rb) * nsb + b0) * kTilesPerBlock * 16;
+                        const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(a.S) + sidx * ssz;
+                        bulk_g2s(smem_u32(sb + kATile + C::kB + C::kPacked), ssrc, sbytes, fb);
+                    }
+                    tma_2d(smem_u32(sb + kATile), &bmap, ks * kBK, int(it.seg0) + it.tt * a.bn, fb);
+                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int st = 0, acc = 0;
+            uint32_t ph = 0, aph = 0;
+            bool ok = true;
+            for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+                const Item it = item_at(i, prefix, a, nrb, nks);
+                const int n = ((it.rows + 15) / 16) * 16;
+                const uint32_t idesc = idesc_bf16(n);
+                if (!mbar_wait(smem_u32(&acce[acc]), aph ^ 1u, abort_flag, a.status)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + uint32_t(acc * BNMAX);
+                for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
+                    if (!mbar_wait(smem_u32(&deq[st]), ph, abort_flag, a.status) ||
+                        !mbar_wait(smem_u32(&full[st]), ph, abort_flag, a.status)) { ok = false; break; }
+                    tc_fence_after();
+                    uint8_t* sb = smem + st * C::kStage;
+                    const uint64_t ad = desc_sw128(smem_u32(sb));
+                    const uint64_t bd = desc_sw128(smem_u32(sb + kATile));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)  // 32 bytes of K per MMA
+                        mma_bf16_ss(d, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc,
+                                    (ks > it.ks_lo || kk > 0) ? 1u : 0u);
+                    mma_commit(smem_u32(&empty[st]));
+                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&accf[acc]));
+                if (++acc == 2) { acc = 0; aph ^= 1u; }
+            }
+        }
+    } else if (warp < kDeqWarps) {
+        // ------------------------------------------------------- dequantise
+        int st = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        const uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u, kBias4 = 0x43084308u;
+        for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+            const Item it = item_at(i, prefix, a, nrb, nks);
+            for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
+                if (!warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status)) { ok = false; break; }
+                uint8_t* sb = smem + st * C::kStage;
+                const uint8_t* pk = sb + kATile + C::kB;
+                const uint8_t* sc = pk + C::kPacked;
+                constexpr int CHUNKS = (BITS == 4 ? 1 : 2);
+#pragma unroll
+                for (int q = 0; q < CHUNKS; ++q) {
+                    const int id = tid + q * (kDeqWarps * 32);
+                    const int gg = id >> 8;           // k-group inside the stage (int8: 0 or 1)
+                    const int tile = (id >> 5) & 7;
+                    const int ln = id & 31;
+                    const int r0 = ln >> 2, c = ln & 3;
+                    const int row0 = tile * 16 + r0, row1 = row0 + 8;
+                    const uint4 w = *reinterpret_cast<const uint4*>(pk + id * 16);
+                    // the lane's k range inside the stage
+                    const int k0 = BITS == 4 ? 16 * c : 32 * gg + 8 * c;
+                    uint32_t sa2 = 0, sb2 = 0;
+                    if (!PERCOL) {
+                        const int blk = a.block_size >= kBK ? 0 : k0 / a.block_size;
+                        const int si = (blk * kTilesPerBlock + tile) * 16 + 2 * r0;
+                        float sa, sbv;
+                        if (a.scale_bf16) {
+                            const uint32_t raw = *reinterpret_cast<const uint32_t*>(sc + si * 2);
+                            sa = __uint_as_float(raw << 16);
+                            sbv = __uint_as_float(raw & 0xFFFF0000u);
+                        } else {
+                            const float2 f = *reinterpret_cast<const float2*>(sc + si * 4);
+                            sa = f.x;
+                            sbv = f.y;
+                        }
+                        sa2 = bf2_bcast(sa);
+                        sb2 = bf2_bcast(sbv);
+                    }
+                    if (BITS == 4) {
+                        // 4 k-steps x 4 registers; register p of step j holds rows
+                        // (r0, r0+8, r0, r0+8)[p] at k offsets 4j + (0,0,2,2)[p] (+1)
+                        uint32_t r0v[8], r1v[8];
+                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t A[4];
+                            A[0] = bf2_sub((wv[j] & kMask) | kMagic, kBias4);
+                            A[1] = bf2_sub(((wv[j] >> 4) & kMask) | kMagic, kBias4);
+                            A[2] = bf2_sub(((wv[j] >> 8) & kMask) | kMagic, kBias4);
+                            A[3] = bf2_sub(((wv[j] >> 12) & kMask) | kMagic, kBias4);
+                            if (!PERCOL) {
+                                A[0] = bf2_mul(A[0], sa2);
+                                A[2] = bf2_mul(A[2], sa2);
+                                A[1] = bf2_mul(A[1], sb2);
+                                A[3] = bf2_mul(A[3], sb2);
+                            }
+                            r0v[2 * j] = A[0];      // row0, k 4j, 4j+1
+                            r0v[2 * j + 1] = A[2];  // row0, k 4j+2, 4j+3
+                            r1v[2 * j] = A[1];
+                            r1v[2 * j + 1] = A[3];
+                        }
+                        *reinterpret_cast<uint4*>(sb + a_off(row0, k0)) = make_uint4(r0v[0], r0v[1], r0v[2], r0v[3]);
+                        *reinterpret_cast<uint4*>(sb + a_off(row0, k0 + 8)) = make_uint4(r0v[4], r0v[5], r0v[6], r0v[7]);
+                        *reinterpret_cast<uint4*>(sb + a_off(row1, k0)) = make_uint4(r1v[0], r1v[1], r1v[2], r1v[3]);
+                        *reinterpret_cast<uint4*>(sb + a_off(row1, k0 + 8)) = make_uint4(r1v[4], r1v[5], r1v[6], r1v[7]);
+                    } else {
+                        // 2 k-steps of 8 bytes; byte pair q of a step holds rows
+                        // (r0, r0+8, r0, r0+8)[q] at k offsets 4j + (0,0,2,2)[q] (+1).
+                        // A byte b is q - 128 = (b & 127) - (b >= 128 ? 0 : 128): OR the low
+                        // 7 bits into bf16 128.0 and subtract 256.0 or 128.0 (0x4380 with
+                        // the exponent bit flipped by the byte's top bit), both exact.
+                        uint32_t r0v[4], r1v[4];
+                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            uint32_t A[4];
+#pragma unroll
+                            for (int qq = 0; qq < 4; ++qq) {
+                                const uint32_t word = wv[2 * j + (qq >> 1)];
+                                // bytes (0,1) or (2,3) of the word into the low byte of each half
+                                const uint32_t pr = __byte_perm(word, 0u, (qq & 1) ? 0x4342u : 0x4140u);
+                                const uint32_t lo = (pr & 0x007F007Fu) | 0x43004300u;
+                                const uint32_t hi = (pr & 0x00800080u) ^ 0x43804380u;
+                                A[qq] = bf2_sub(lo, hi);
+                            }
+                            if (!PERCOL) {
+                                A[0] = bf2_mul(A[0], sa2);
+                                A[2] = bf2_mul(A[2], sa2);
+                                A[1] = bf2_mul(A[1], sb2);
+                                A[3] = bf2_mul(A[3], sb2);
+                            }
+                            r0v[2 * j] = A[0];
+                            r0v[2 * j + 1] = A[2];
+                            r1v[2 * j] = A[1];
+                            r1v[2 * j + 1] = A[3];
+                        }
+                        *reinterpret_cast<uint4*>(sb + a_off(row0, k0)) = make_uint4(r0v[0], r0v[1], r0v[2], r0v[3]);
+                        *reinterpret_cast<uint4*>(sb + a_off(row1, k0)) = make_uint4(r1v[0], r1v[1], r1v[2], r1v[3]);
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&deq[st]));
+                if (++st == STAGES) { st = 0; ph ^= 1u; }
+            }
+        }
+    } else if (warp >= kWarpEpi0) {
+        // ------------------------------------------------------- epilogue
+        const int qd = warp & 3;  // TMEM lane quarter this warp may read
+        const int row = qd * 32 + lane;
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int i = blockIdx.x; i < total; i += gridDim.x) {
+            const Item it = item_at(i, prefix, a, nrb, nks);
+            if (!warp_wait(smem_u32(&accf[acc]), aph, abort_flag, a.status)) break;
+            tc_fence_after();
+            const int64_t prow = int64_t(it.rb) * kBlockRows + row;  // packed row in the expert
+            const bool valid = prow < a.N;
+            float s = 1.0f;
+            if (PERCOL && valid) {
+                const int tile = row >> 4, rr = row & 15;
+                const int64_t si = ((int64_t(it.e) * nrb + it.rb) * kTilesPerBlock + tile) * 16 + (rr & 7) * 2 + (rr >> 3);
+                s = a.scale_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.S)[si])
+                                 : reinterpret_cast<const float*>(a.S)[si];
+            }
+            const float bias = (a.bias && valid) ? a.bias[int64_t(it.e) * a.N + prow] : 0.0f;
+            const uint32_t tbase = tmem + (uint32_t(qd * 32) << 16) + uint32_t(acc * BNMAX);
+            const int ncol = ((it.rows + 15) / 16) * 16;
+            for (int c0 = 0; c0 < ncol; c0 += 16) {
+                float v[16];
+                tmem_ld16(tbase + uint32_t(c0), v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int col = c0 + j;
+                    const float val = fmaf(v[j], s, bias);
+                    const bool in = col < it.rows;
+                    const int64_t p = it.seg0 + int64_t(it.tt) * a.bn + col;  // permuted row
+                    if (a.is_fc1) {
+                        if (a.gated) {
+                            const float up = __shfl_down_sync(0xffffffffu, val, 8);
+                            if (in && valid && (row & 15) < 8) {
+                                const int64_t I = a.N / 2;
+                                const int64_t ii = (prow >> 4) * 8 + (row & 7);
+                                reinterpret_cast<__nv_bfloat16*>(a.out)[p * I + ii] =
+                                    __float2bfloat16_rn(act_gated(a.act_type, val, up, a.alpha, a.beta, a.limit));
+                            }
+                        } else if (in && valid) {
+                            reinterpret_cast<__nv_bfloat16*>(a.out)[p * a.N + prow] =
+                                __float2bfloat16_rn(act_plain(a.act_type, val));
+                        }
+                    } else if (in && valid) {
+                        reinterpret_cast<float*>(a.out)[(int64_t(it.split) * a.R + p) * a.N + prow] = val;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acce[acc]));
+            if (++acc == 2) { acc = 0; aph ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols));
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int BITS, bool PERCOL, int BNMAX>
+struct Launch {
+    static constexpr int kStage = TcCfg<BITS, PERCOL, BNMAX, 1>::kStage;
+    static constexpr int kStages = ((220 * 1024) / kStage) > 8 ? 8 : ((220 * 1024) / kStage);
+    using C = TcCfg<BITS, PERCOL, BNMAX, kStages>;
+    static cudaError_t prepare() {
+        return cudaFuncSetAttribute(ffn_tc_kernel<BITS, PERCOL, BNMAX, kStages>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    }
+    static cudaError_t run(const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t st) {
+        ffn_tc_kernel<BITS, PERCOL, BNMAX, kStages><<<grid, kTcThreads, C::kSmem, st>>>(map, a);
+        return cudaGetLastError();
+    }
+};
+
+template <int BITS, bool PERCOL>
+cudaError_t dispatch_bn(int bnmax, const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t st) {
+    switch (bnmax) {
+        case 16: return Launch<BITS, PERCOL, 16>::run(map, a, grid, st);
+        case 32: return Launch<BITS, PERCOL, 32>::run(map, a, grid, st);
+        case 64: return Launch<BITS, PERCOL, 64>::run(map, a, grid, st);
+        case 128: return Launch<BITS, PERCOL, 128>::run(map, a, grid, st);
+        default: return Launch<BITS, PERCOL, 256>::run(map, a, grid, st);
+    }
+}
+
+template <int BITS, bool PERCOL>
+cudaError_t prepare_bits() {
+    cudaError_t e = Launch<BITS, PERCOL, 16>::prepare();
+    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 32>::prepare();
+    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 64>::prepare();
+    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 128>::prepare();
+    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 256>::prepare();
+    return e;
+}
+
+__global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm,
+                                   uint4* __restrict__ xp, int64_t R, int64_t row_vecs) {
+    const int64_t total = R * row_vecs;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t p = i / row_vecs, v = i - p * row_vecs;
+        xp[i] = x[int64_t(perm[p]) * row_vecs + v];
+    }
+}
+
+}  // namespace
+
+cudaError_t prepare_ffn_tc() {
+    cudaError_t e = prepare_bits<4, false>();
+    if (e == cudaSuccess) e = prepare_bits<4, true>();
+    if (e == cudaSuccess) e = prepare_bits<8, false>();
+    if (e == cudaSuccess) e = prepare_bits<8, true>();
+    return e;
+}
+
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm, void* xp, int64_t R, int64_t row_bytes,
+                               cudaStream_t st) {
+    if (R == 0) return cudaSuccess;
+    const int64_t vecs = row_bytes / 16;
+    int64_t blocks = (R * vecs + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    gather_rows_kernel<<<unsigned(blocks), 256, 0, st>>>(reinterpret_cast<const uint4*>(x), perm,
+                                                       reinterpret_cast<uint4*>(xp), R, vecs);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ffn_tc(const FfnArgs& f, int bn, int32_t* status, cudaStream_t st) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    int bnmax = 16;
+    while (bnmax < bn) bnmax *= 2;
+    if (bnmax > 256) return cudaErrorInvalidValue;
+    // activations: [rows, K] bf16; rows = R (permuted rows)
+    const int64_t rows = f.R;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {cuuint64_t(f.K), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(f.K * 2)};
+    const cuuint32_t box[2] = {cuuint32_t(kBK), cuuint32_t(bnmax)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(f.act), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    TcArgs a{};
+    a.W = f.W;
+    a.S = f.S;
+    a.bias = f.bias;
+    a.offsets = f.offsets;
+    a.out = f.out;
+    a.status = status;
+    a.N = f.N;
+    a.K = f.K;
+    a.R = f.R;
+    a.E = f.E;
+    a.block_size = f.block_size;
+    a.gated = f.gated;
+    a.is_fc1 = f.is_fc1;
+    a.act_type = f.act_type;
+    a.alpha = f.alpha;
+    a.beta = f.beta;
+    a.limit = f.limit;
+    a.splits = f.splits;
+    a.scale_bf16 = f.scale_bf16;
+    a.bn = bn;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const bool percol = f.block_size == 0;
+    if (f.bits == 4)
+        return percol ? dispatch_bn<4, true>(bnmax, map, a, sms, st) : dispatch_bn<4, false>(bnmax, map, a, sms, st);
+    return percol ? dispatch_bn<8, true>(bnmax, map, a, sms, st) : dispatch_bn<8, false>(bnmax, map, a, sms, st);
+}
+
+}  // namespace qmoe

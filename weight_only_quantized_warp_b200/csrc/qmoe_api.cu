@@ -27,17 +27,22 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     p.T = T;
     p.R = T * c.k;
     const bool bf16 = c.act_dtype == QMOE_DTYPE_BF16;
-    p.path = bf16 ? kPathDecode : kPathSimt;
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size;
+    const int bits = c.expert_weight_bits, bs = c.block_size;
+    const int64_t per_expert = ceil_div(std::max<int64_t>(p.R, 1), E);
+    if (!bf16)
+        p.path = kPathSimt;
+    else if (h.path_override == kPathDecode || h.path_override == kPathTc)
+        p.path = h.path_override;
+    else
+        p.path = per_expert <= kDecodeRowsPerExpert ? kPathDecode : kPathTc;
+    const int64_t touched = std::min<int64_t>(E, std::max<int64_t>(p.R, 1));
     if (p.path == kPathDecode) {
-        const int bits = c.expert_weight_bits, bs = c.block_size;
-        const int64_t per_expert = ceil_div(std::max<int64_t>(p.R, 1), E);
         p.nt = per_expert <= 8 ? 1 : (per_expert <= 16 ? 2 : 4);
         // FC1 runs unsplit; keep its staged rows small enough for two CTAs per SM
         while (p.nt > 1 && decode_smem_bytes(H, bits, bs, 1, p.nt) > kDecodeSmemTarget) p.nt /= 2;
         // enough FC2 warps (one per 16-row tile per touched expert per split)
         // to give every SM several resident warps
-        const int64_t touched = std::min<int64_t>(E, std::max<int64_t>(p.R, 1));
         const int64_t warps = touched * (H / kTileRows);
         const int64_t want = kSms * 48;
         const int64_t ngr = I / kgroup_of(bits);
@@ -48,8 +53,19 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         p.fc2_splits = int(std::max<int64_t>(s, 1));
         p.ok = decode_smem_bytes(H, bits, bs, 1, p.nt) <= int64_t(kDecodeSmemLimit) &&
                decode_smem_bytes(I, bits, bs, p.fc2_splits, p.nt) <= int64_t(kDecodeSmemLimit);
+    } else if (p.path == kPathTc) {
+        int bn = 16;
+        while (bn < 256 && bn < per_expert) bn *= 2;
+        if (per_expert >= 64) bn = 256;
+        p.bn = bn;
+        // FC2 work items: touched experts x 128-row blocks x token tiles;
+        // split K until every SM has about two items
+        const int64_t items = touched * (padded_rows(H) / kBlockRows) * std::max<int64_t>(1, ceil_div(per_expert, bn));
+        int64_t s = 1;
+        while (items * s < 2 * kSms && s < 8 && s * 2 <= I / 64) s *= 2;
+        p.fc2_splits = int(s);
     }
-    p.launches = 5;
+    p.launches = p.path == kPathTc ? 6 : 5;
     const size_t R = size_t(p.R);
     const size_t act = bf16 ? 2 : 4;
     size_t off = 0;
@@ -60,6 +76,7 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     p.off_perm = off;    off = align256(off + R * 4);
     p.off_offsets = off; off = align256(off + size_t(E + 1) * 4);
     p.off_h = off;       off = align256(off + R * size_t(I) * act);
+    p.off_xperm = off;   off = align256(off + (p.path == kPathTc ? R * size_t(H) * act : 0));
     p.off_o = off;       off = align256(off + size_t(p.fc2_splits) * R * size_t(H) * 4);
     p.total = off;
     return p;
@@ -214,6 +231,7 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
     if (err != cudaSuccess) return cuda_fail(h, err, "cudaGetDevice");
     err = prepare_route_permute();
     if (err == cudaSuccess) err = prepare_ffn_decode();
+    if (err == cudaSuccess) err = prepare_ffn_tc();
     if (err != cudaSuccess) return cuda_fail(h, err, "prepare kernels");
 
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size, N1 = h->n1;
@@ -286,6 +304,17 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
     h->bound = true;
     h->last_error.clear();
     return QMOE_OK;
+}
+
+qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t value) {
+    if (!h) return QMOE_INVALID_ARGUMENT;
+    if (option == QMOE_OPT_PATH) {
+        if (value != -1 && value != kPathDecode && value != kPathTc)
+            return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_PATH must be -1, 1 or 2");
+        h->path_override = int(value);
+        return QMOE_OK;
+    }
+    return fail(h, QMOE_INVALID_ARGUMENT, "unknown option %d", int(option));
 }
 
 size_t qmoe_workspace_size(const qmoe_handle* h, int64_t T) {
@@ -395,11 +424,23 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     f2.gated = 0;
     f2.is_fc1 = 0;
     f2.splits = p.fc2_splits;
+    int32_t* status = (int32_t*)(ws + p.off_status);
+    if (p.path == kPathTc) {
+        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+        void* xp = ws + p.off_xperm;
+        if ((err = launch_gather_rows(x, perm, xp, p.R, c.hidden_size * 2, st)) != cudaSuccess)
+            return cuda_fail(h, err, "gather");
+        f1.act = xp;
+    }
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-    err = p.path == kPathSimt ? launch_ffn_simt(f1, st) : launch_ffn_decode(f1, st);
+    err = p.path == kPathSimt ? launch_ffn_simt(f1, st)
+          : p.path == kPathTc ? launch_ffn_tc(f1, p.bn, status, st)
+                              : launch_ffn_decode(f1, st);
     if (err != cudaSuccess) return cuda_fail(h, err, "fc1");
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-    err = p.path == kPathSimt ? launch_ffn_simt(f2, st) : launch_ffn_decode(f2, st);
+    err = p.path == kPathSimt ? launch_ffn_simt(f2, st)
+          : p.path == kPathTc ? launch_ffn_tc(f2, p.bn, status, st)
+                              : launch_ffn_decode(f2, st);
     if (err != cudaSuccess) return cuda_fail(h, err, "fc2");
     CombineArgs ca{};
     ca.o = o;

@@ -55,8 +55,9 @@ struct Plan {
     int fc2_splits = 1;  // split-K factor of FC2 (partials reduced by the combine)
     int launches = 0;
     bool ok = true;      // a kernel configuration exists for this shape
+    int bn = 0;          // token tile of the tensor-core path
     size_t off_idx = 0, off_w = 0, off_inv = 0, off_perm = 0, off_offsets = 0, off_status = 0,
-           off_h = 0, off_o = 0, total = 0;
+           off_h = 0, off_o = 0, off_xperm = 0, total = 0;
 };
 
 }  // namespace qmoe
@@ -73,6 +74,7 @@ struct qmoe_handle {
     void* s2 = nullptr;
     float* b2 = nullptr;  // [E, H] fp32, nullptr when no fc2 bias
     int device = -1;
+    int path_override = -1;  // QMOE_OPT_PATH; -1 = choose by shape
     mutable std::mutex mu;
     mutable std::string last_error;
 };
@@ -137,9 +139,19 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
 // prepare_ffn_decode() raises the kernels' limit on the current device.
 constexpr size_t kDecodeSmemLimit = 200 * 1024;
 constexpr int64_t kDecodeSmemTarget = 112 * 1024;  // two CTAs per SM
+// Rows per expert up to which the weight-streaming kernels are chosen.
+constexpr int64_t kDecodeRowsPerExpert = 16;
 int64_t decode_smem_bytes(int64_t K, int bits, int block_size, int splits, int nt);
 cudaError_t prepare_ffn_decode();
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
+
+// Tensor-core (tcgen05) expert FFN layer over the segments; bn = token tile.
+// prepare_ffn_tc() raises the kernels' shared-memory limit on the current
+// device. launch_gather_rows copies the routed rows of x into segment order.
+cudaError_t prepare_ffn_tc();
+cudaError_t launch_ffn_tc(const FfnArgs& a, int bn, int32_t* status, cudaStream_t st);
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm, void* xp, int64_t R, int64_t row_bytes,
+                               cudaStream_t st);
 
 // Router-weighted combine with fc2 bias and shared output; sums the FC2
 // split partials in fixed order.

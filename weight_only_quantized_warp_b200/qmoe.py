@@ -34,7 +34,9 @@ PATH_SIMT, PATH_DECODE, PATH_TC = 0, 1, 2
 EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forward",
            "qmoe_forward_profiled",
            "qmoe_debug_routing", "qmoe_debug_hidden", "qmoe_read_device_status", "qmoe_destroy",
-           "qmoe_status_string", "qmoe_last_error", "qmoe_path_for", "qmoe_launches_for")
+           "qmoe_status_string", "qmoe_last_error", "qmoe_path_for", "qmoe_launches_for",
+           "qmoe_set_option")
+QMOE_OPT_PATH = 1
 
 
 class qmoe_config(ctypes.Structure):
@@ -76,6 +78,8 @@ lib.qmoe_last_error.restype = ctypes.c_char_p
 lib.qmoe_last_error.argtypes = [_vp]
 lib.qmoe_path_for.restype = ctypes.c_int32
 lib.qmoe_path_for.argtypes = [_vp, _i64]
+lib.qmoe_set_option.restype = ctypes.c_int
+lib.qmoe_set_option.argtypes = [_vp, ctypes.c_int32, _i64]
 lib.qmoe_launches_for.restype = ctypes.c_int32
 lib.qmoe_launches_for.argtypes = [_vp, _i64]
 
@@ -181,6 +185,10 @@ def qmoe_path_for(h, T: int) -> int:
     return int(lib.qmoe_path_for(h, T))
 
 
+def qmoe_set_option(h, option: int, value: int):
+    _check(lib.qmoe_set_option(h, option, value), h)
+
+
 def qmoe_launches_for(h, T: int) -> int:
     return int(lib.qmoe_launches_for(h, T))
 
@@ -202,12 +210,14 @@ def to_device(a, device):
 class QMoE:
     """One QMoE operator instance on one GPU (marshalling around the C ABI)."""
 
-    def __init__(self, cfg, device=None):
+    def __init__(self, cfg, device=None, path=None):
         import torch
         self.cfg = cfg
         self.device = torch.device(device or "cuda")
         self.handle = qmoe_create(make_config(cfg))
         self._ws = None
+        if path is not None:
+            qmoe_set_option(self.handle, QMOE_OPT_PATH, path)
 
     def __del__(self):
         h = getattr(self, "handle", None)
