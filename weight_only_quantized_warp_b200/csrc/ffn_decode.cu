@@ -15,11 +15,10 @@
 //
 // Fragments. For an m16n8k16 MMA, lane L holds A rows r0 = L/4 and r0 + 8 at
 // k positions 2c, 2c+1, 2c+8, 2c+9 (c = L%4) and B column r0 at the same k
-// positions. Because the dot product does not depend on the order of k, the
-// packed layout assigns lane column c the 16 consecutive actual k
-// [16c, 16c + 16) of each 64-wide group (int4; 8 of each 32-wide group for
-// int8), spread over 4 (2) MMA k-steps. The lane's activations for a group are
-// then one contiguous 32-byte (16-byte) run, and its weights one 16-byte load.
+// positions. The packed layout maps those positions of k-step j to the actual
+// k values 16j + 4c + {0, 1} and 16j + 4c + {2, 3} (the dot product does not
+// depend on the order of k), so the lane's activations for one k-step are one
+// 8-byte run and its weights for a whole k-group one 16-byte load.
 //
 // Int-to-bf16 decode, derived from the IEEE-754 bf16 layout (1 sign, 8
 // exponent, 7 mantissa bits): the word 0x4300 is 128.0 and its mantissa's unit
@@ -236,9 +235,9 @@ struct ScaleRaw<true> {
 };
 
 // Bytes of one staged activation row for a k range of kr elements: bf16
-// values plus 16 bytes of padding, which spreads the 8 rows a warp reads at
-// one time over all 32 shared-memory banks.
-__host__ __device__ constexpr int64_t staged_row_bytes(int64_t kr) { return kr * 2 + 16; }
+// values plus 32 bytes of padding, so the 8-byte reads of 4 rows x 4 lanes
+// that one phase of a warp's load serves land in distinct shared-memory banks.
+__host__ __device__ constexpr int64_t staged_row_bytes(int64_t kr) { return kr * 2 + 32; }
 
 // Zero-point folding (int4, scale after the MMA). With A = 128 + q (the code
 // OR-ed into bf16 128.0, no subtraction), sum_k (q - 8) x_k equals
@@ -306,10 +305,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
     const int64_t sb0 = (((int64_t)e * nrb + rb) * nsb * kTilesPerBlock + warp) * 16 + 2 * r0;
     const void* sbase = SF32 ? (const void*)((const float*)a.S + sb0)
                              : (const void*)((const __nv_bfloat16*)a.S + sb0);
-    const int kc = SMODE == 2 ? (KG / 4) * c : 0;
-    auto sidx = [&](int ga) -> int {
-        return SMODE == 1 ? (ga >> lg_gpb) * 128 : ((ga * KG + kc) >> lg_bs) * 128;
-    };
+    // SMODE 1: scale index of absolute group ga; SMODE 2: of k-step j of ga
+    auto sidx = [&](int ga) -> int { return (ga >> lg_gpb) * 128; };
+    auto sidx_step = [&](int ga, int j) -> int { return ((ga * KG + 16 * j + 4 * c) >> lg_bs) * 128; };
     const __nv_bfloat16* act = (const __nv_bfloat16*)a.act;
 
     float s0 = 1.0f, s1 = 1.0f;  // per-column scales
@@ -323,7 +321,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
             for (int i = 0; i < D; ++i) {
                 if (i < ng) {
                     wr[i] = ld_stream(wp + i * GS);
-                    if (SMODE != 0 && i % P == 0) sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + i));
+                    if (SMODE == 1 && i % P == 0) sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + i));
                 }
             }
         }
@@ -388,19 +386,19 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
 
         // one k-group: decode the lane's 16 bytes, 4 (int4) or 2 (int8) MMA
         // k-steps per token tile. xg is this lane's activation run of the group.
-        auto group = [&](const uint4 w, const uint8_t* xg, const ScaleRaw<SF32> sc) {
-            uint4 xa[NT][2];
+        auto group = [&](const uint4 w, const uint8_t* xg, const ScaleRaw<SF32> sc, int ga) {
+            uint2 xa[NT][KSTEPS];  // per k-step: activation pairs at 16j+4c, 16j+4c+2
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                xa[n][0] = *reinterpret_cast<const uint4*>(xg + n * 8 * rs);
-                if (BITS == 4) xa[n][1] = *reinterpret_cast<const uint4*>(xg + n * 8 * rs + 16);
-            }
-            float sa = 1.0f, sb = 1.0f;
-            if (SMODE == 2) sc.get(sa, sb);
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int j = 0; j < KSTEPS; ++j)
+                    xa[n][j] = *reinterpret_cast<const uint2*>(xg + n * 8 * rs + j * 32);
             const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int j = 0; j < KSTEPS; ++j) {
                 uint32_t A[4];
+                float sa = 1.0f, sb = 1.0f;  // SMODE 2: scales of this k-step's block
+                if (SMODE == 2) ScaleRaw<SF32>::load(sbase, sidx_step(ga, j)).get(sa, sb);
                 if (BITS == 4) {
                     if (FOLD) {
                         constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;
@@ -443,12 +441,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
                 }
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
-                    const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xa[n][0]);
-                    // kstep j uses activation words 2j, 2j+1 of the lane's run
                     if (SMODE == 1)
-                        mma_bf16(blk[n], A, xw[2 * j], xw[2 * j + 1]);
+                        mma_bf16(blk[n], A, xa[n][j].x, xa[n][j].y);
                     else
-                        mma_bf16(acc[n], A, xw[2 * j], xw[2 * j + 1]);
+                        mma_bf16(acc[n], A, xa[n][j].x, xa[n][j].y);
                 }
             }
         };
@@ -475,7 +471,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
 
         if (active) {
             const uint8_t* wn = wp + D * GS;                      // loads run D groups ahead
-            const uint8_t* xp = xs + r0 * rs + (KG / 4) * c * 2;  // this lane's run, group 0
+            const uint8_t* xp = xs + r0 * rs + 8 * c;  // this lane's first pair, group 0
             const float* csp = cs + 2 * c;                        // chunk 0, tokens 2c, 2c+1
             ScaleRaw<SF32> scur = sr[0];
             int g = 0;  // group relative to g_lo
@@ -484,10 +480,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
 #pragma unroll
                 for (int i = 0; i < D; ++i) {
                     // use slot i, then refill it (no register copy of the old value)
-                    if (SMODE != 0 && i % P == 0) scur = sr[i / P];
-                    group(wr[i], xp + i * KG * 2, scur);
+                    if (SMODE == 1 && i % P == 0) scur = sr[i / P];
+                    group(wr[i], xp + i * KG * 2, scur, int(g_lo) + g + i);
                     wr[i] = ld_stream(wn + i * GS);
-                    if (SMODE != 0 && i % P == P - 1)
+                    if (SMODE == 1 && i % P == P - 1)
                         sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + 1 - P + D));
                     if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
                 }
@@ -499,10 +495,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
             if (g + D <= ng) {
 #pragma unroll
                 for (int i = 0; i < D; ++i) {
-                    if (SMODE != 0 && i % P == 0) scur = sr[i / P];
-                    group(wr[i], xp + i * KG * 2, scur);
+                    if (SMODE == 1 && i % P == 0) scur = sr[i / P];
+                    group(wr[i], xp + i * KG * 2, scur, int(g_lo) + g + i);
                     if (g + i + D < ng) wr[i] = ld_stream(wn + i * GS);
-                    if (SMODE != 0 && i % P == P - 1 && g + i + 1 - P + D < ng)
+                    if (SMODE == 1 && i % P == P - 1 && g + i + 1 - P + D < ng)
                         sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + 1 - P + D));
                     if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
                 }
@@ -514,8 +510,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
 #pragma unroll
             for (int i = 0; i < D; ++i) {
                 if (g + i < ng) {
-                    if (SMODE != 0 && i % P == 0) scur = sr[i / P];
-                    group(wr[i], xp + i * KG * 2, scur);
+                    if (SMODE == 1 && i % P == 0) scur = sr[i / P];
+                    group(wr[i], xp + i * KG * 2, scur, int(g_lo) + g + i);
                     if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
                 }
             }
@@ -578,7 +574,7 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
         for (int n = 0; n < 8; ++n) {
             const int tok = min(p0 + n, M - 1);
             const int64_t row = a.rowmap ? a.rowmap[seg0 + tok] : seg0 + tok;
-            xrow[n] = act + row * a.K + KL * c;
+            xrow[n] = act + row * a.K;
         }
         float acc[8][2];
 #pragma unroll
@@ -588,6 +584,7 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
             const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
             // decode the lane's 2 x KL codes into (row, actual k) order
             float q[2][KL];
+            // q[row][4j + t] is the code at k = 16j + 4c + t of row r0 (+8)
             if (BITS == 4) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
@@ -604,24 +601,27 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
                             byte_centered(wv[2 * j + (m >> 2)], m & 3);
                     }
             }
-            const int64_t b = a.block_size > 0 ? (g * KG + KL * c) / a.block_size : 0;
-            const float sa = load_scale(a.S, sbase + b * 128, sf32);
-            const float sb = load_scale(a.S, sbase + b * 128 + 1, sf32);
+            // the lane's k values span several blocks when block_size < KG: one
+            // scale per 4-wide run (block_size >= 16 keeps each run in one block)
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                float pa = 0.0f, pb = 0.0f;
+            for (int j = 0; j < KL / 4; ++j) {
+                const int64_t kk = g * KG + 16 * j + 4 * c;
+                const int64_t b = a.block_size > 0 ? kk / a.block_size : 0;
+                const float sa = load_scale(a.S, sbase + b * 128, sf32);
+                const float sb = load_scale(a.S, sbase + b * 128 + 1, sf32);
 #pragma unroll
-                for (int v4 = 0; v4 < KL / 4; ++v4) {
-                    const float4 xv = *reinterpret_cast<const float4*>(xrow[n] + g * KG + 4 * v4);
+                for (int n = 0; n < 8; ++n) {
+                    const float4 xv = *reinterpret_cast<const float4*>(xrow[n] + kk);
                     const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+                    float pa = 0.0f, pb = 0.0f;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        pa = fmaf(q[0][4 * v4 + u], xs[u], pa);
-                        pb = fmaf(q[1][4 * v4 + u], xs[u], pb);
+                        pa = fmaf(q[0][4 * j + u], xs[u], pa);
+                        pb = fmaf(q[1][4 * j + u], xs[u], pb);
                     }
+                    acc[n][0] = fmaf(sa, pa, acc[n][0]);
+                    acc[n][1] = fmaf(sb, pb, acc[n][1]);
                 }
-                acc[n][0] = fmaf(sa, pa, acc[n][0]);
-                acc[n][1] = fmaf(sb, pb, acc[n][1]);
             }
         }
         // reduce over the 4 lanes of a row pair (lane bits 0-1)

@@ -9,24 +9,31 @@
 // the QMoE page's gated activation in its epilogue.
 //
 // Operand roles ("swap AB"): the MMA's M dimension is 128 weight rows, its N
-// dimension the routed tokens of one expert (a multiple of 16, up to 256), so
+// dimension the routed tokens of one expert (a multiple of 16, up to 128), so
 // a small expert segment wastes no tensor work on padding rows.
 //
-// Warp roles of one persistent CTA (448 threads, one CTA per SM):
-//   warps 0-7   dequantise: packed codes (shared) -> bf16 A tile in the
-//               128-byte-swizzled K-major layout the MMA descriptor reads
+// Warp roles of one persistent CTA (576 threads, one CTA per SM):
+//   warps 0-7   dequantise: packed codes (shared) -> bf16 A tile written
+//               straight into tensor memory (tcgen05.st), one 16-row tile per
+//               warp; the A operand never touches shared memory
 //   warp 8      producer: one bulk copy of the packed 128 x 64 tile (4 KB
-//               int4, 8 KB int8), one of its scales, one TMA tile of the
-//               activations (N rows x 64 bf16, 128-byte swizzle)
-//   warp 9      allocates TMEM and issues tcgen05.mma from one thread
-//   warps 10-13 epilogue: TMEM -> registers (tcgen05.ld), scale / bias /
-//               activation, global stores
+//               int4, 8 KB int8), one of its scales, and 64-row TMA boxes of
+//               the activations (bf16, 128-byte swizzle), as many as the tile
+//               has rows
+//   warp 9      allocates TMEM and issues tcgen05.mma (A from TMEM, B from
+//               shared memory) from one thread
+//   warps 10-17 epilogue: TMEM -> registers (tcgen05.ld), scale / bias /
+//               activation, global stores; two warps per TMEM lane quarter
 // Stages cycle through an S-deep ring guarded by mbarriers (full: copies
-// landed; deq: A tile written; empty: the MMAs reading the stage are done);
-// two TMEM accumulators let the epilogue of one work item overlap the
+// landed; deq: A tile written to TMEM; empty: the MMAs reading the stage are
+// done); two TMEM accumulators let the epilogue of one work item overlap the
 // mainloop of the next. Every wait is bounded: after about two seconds the
 // kernel records QMOE_TIMEOUT in the workspace status word, every role
 // leaves its loop, and the CTA frees its TMEM and exits.
+//
+// The packed layout puts lane (r0 = L/4, c = L%4) of a 16-row tile on rows r0
+// and r0 + 8 and k = 16j + 4c + {0..3}: after decoding, its registers are
+// exactly the 16x256b tensor-memory store fragment of k-step j.
 //
 // Scales: a K-block scale is multiplied into the decoded weight (one bf16
 // rounding of (q - z) * s); per-column scales (block_size 0) leave exact
@@ -42,9 +49,10 @@ constexpr int kDeqWarps = 8;
 constexpr int kWarpProd = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpEpi0 = 10;
-constexpr int kTcThreads = 14 * 32;
-constexpr int kBK = 64;                           // k per stage
-constexpr int kATile = kBlockRows * kBK * 2;      // 16 KB of bf16
+constexpr int kEpiWarps = 8;
+constexpr int kTcThreads = (kWarpEpi0 + kEpiWarps) * 32;  // 576
+constexpr int kBK = 64;                                    // k per stage
+constexpr int kAStageCols = kBK / 2;                       // TMEM columns of one A tile
 constexpr int kScaleBytesMax = 4 * kTilesPerBlock * 16 * 4;  // 4 blocks of fp32 pairs
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
@@ -191,6 +199,35 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_st16x256_x4(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16x256_x2(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// MMA with A read from tensor memory (128 lanes = rows, 2 bf16 per column).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
 // --------------------------------------------------------------- arithmetic
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
     __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
@@ -207,7 +244,8 @@ __device__ __forceinline__ uint32_t bf2_bcast(float s) {
     return *reinterpret_cast<uint32_t*>(&r);
 }
 
-__device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
+// fast sigmoid: the result is rounded to bf16 right after
+__device__ __forceinline__ float sigmoidf_(float v) { return __fdividef(1.0f, 1.0f + __expf(-v)); }
 __device__ __forceinline__ float act_plain(int t, float a) {
     switch (t) {
         case QMOE_ACT_RELU: return fmaxf(a, 0.0f);
@@ -224,12 +262,6 @@ __device__ __forceinline__ float act_gated(int t, float g, float u, float alpha,
         return (u + beta) * g * sigmoidf_(alpha * g);
     }
     return act_plain(t, g) * u;
-}
-
-// Byte offset of element (row, k) inside an A tile: 8-row atoms of 1024 bytes,
-// 16-byte chunks of a 128-byte row XOR-swizzled by the row's index in its atom.
-__device__ __forceinline__ uint32_t a_off(int row, int k) {
-    return uint32_t((row >> 3) * 1024 + (row & 7) * 128 + ((((k >> 3) ^ (row & 7))) << 4) + (k & 7) * 2);
 }
 
 // ------------------------------------------------------------ work items
@@ -268,12 +300,17 @@ __device__ __forceinline__ Item item_at(int i, const int* prefix, const TcArgs& 
 
 template <int BITS, bool PERCOL, int BNMAX, int STAGES>
 struct TcCfg {
-    static constexpr int kPacked = kBlockRows * kBK * BITS / 8;  // 4 KB or 8 KB
-    static constexpr int kB = BNMAX * 128;
-    static constexpr int kStage = kATile + kB + kPacked + kScaleBytesMax;
-    static constexpr int kTmemCols = (2 * BNMAX < 32) ? 32 : 2 * BNMAX;
+    static constexpr int kBoxRows = BNMAX < 64 ? BNMAX : 64;       // rows of one activation TMA box
+    static constexpr int kPacked = kBlockRows * kBK * BITS / 8;    // 4 KB or 8 KB
+    static constexpr int kB = BNMAX * 128;                         // activation tile
+    static constexpr int kStage = kB + kPacked + kScaleBytesMax;   // multiple of 1024
+    static constexpr int kACol0 = 2 * BNMAX;                       // A tiles after the accumulators
+    static constexpr int kTmemCols = 512;
+    static_assert(kACol0 + STAGES * kAStageCols <= kTmemCols, "TMEM budget");
     static constexpr int kBarOff = STAGES * kStage;
-    static constexpr int kSmem = kBarOff + 1024 + 4 * 260 + 1024;  // barriers, prefix, align slack
+    // barriers, prefix table, alignment slack; at least 120 KB so one CTA per SM
+    static constexpr int kSmemUse = kBarOff + 1024 + 4 * 260 + 1024;
+    static constexpr int kSmem = kSmemUse > 120 * 1024 ? kSmemUse : 120 * 1024;
 };
 
 template <int BITS, bool PERCOL, int BNMAX, int STAGES>
@@ -305,7 +342,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&accf[b]), 1);
-            mbar_init(smem_u32(&acce[b]), 4);
+            mbar_init(smem_u32(&acce[b]), kEpiWarps);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -353,24 +390,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int st = 0;
             uint32_t ph = 0;
             bool ok = true;
+            const int ngr = int(a.K / kgroup_of(BITS));
             for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
                 const Item it = item_at(i, prefix, a, nrb, nks);
-                const int ngr = int(a.K / kgroup_of(BITS));
+                const int nbox = (it.rows + C::kBoxRows - 1) / C::kBoxRows;
+                const uint32_t bytes = uint32_t(C::kPacked + nbox * C::kBoxRows * 128) + sbytes;
                 for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
                     if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
                     uint8_t* sb = smem + st * C::kStage;
                     const uint32_t fb = smem_u32(&full[st]);
-                    mbar_expect_tx(fb, uint32_t(C::kPacked + C::kB) + sbytes);
+                    mbar_expect_tx(fb, bytes);
                     const int g = ks * (kBK / kgroup_of(BITS));  // first k-group of the stage
-                    const uint8_t* src = a.W + ((int64_t(it.e) * nrb + it.rb) * ngr + g) * int64_t(kTilesPerBlock) * kUnitBytes;
-                    bulk_g2s(smem_u32(sb + kATile + C::kB), src, C::kPacked, fb);
+                    const uint8_t* src =
+                        a.W + ((int64_t(it.e) * nrb + it.rb) * ngr + g) * int64_t(kTilesPerBlock) * kUnitBytes;
+                    bulk_g2s(smem_u32(sb + C::kB), src, C::kPacked, fb);
                     if (!PERCOL) {
                         const int b0 = (ks * kBK) / a.block_size;
                         const int64_t sidx = ((int64_t(it.e) * nrb + it.rb) * nsb + b0) * kTilesPerBlock * 16;
                         const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(a.S) + sidx * ssz;
-                        bulk_g2s(smem_u32(sb + kATile + C::kB + C::kPacked), ssrc, sbytes, fb);
+                        bulk_g2s(smem_u32(sb + C::kB + C::kPacked), ssrc, sbytes, fb);
                     }
-                    tma_2d(smem_u32(sb + kATile), &bmap, ks * kBK, int(it.seg0) + it.tt * a.bn, fb);
+                    const int y0 = int(it.seg0) + it.tt * a.bn;
+                    for (int b = 0; b < nbox; ++b)
+                        tma_2d(smem_u32(sb + b * C::kBoxRows * 128), &bmap, ks * kBK, y0 + b * C::kBoxRows, fb);
                     if (++st == STAGES) { st = 0; ph ^= 1u; }
                 }
             }
@@ -392,12 +434,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (!mbar_wait(smem_u32(&deq[st]), ph, abort_flag, a.status) ||
                         !mbar_wait(smem_u32(&full[st]), ph, abort_flag, a.status)) { ok = false; break; }
                     tc_fence_after();
-                    uint8_t* sb = smem + st * C::kStage;
-                    const uint64_t ad = desc_sw128(smem_u32(sb));
-                    const uint64_t bd = desc_sw128(smem_u32(sb + kATile));
+                    const uint32_t at = tmem + uint32_t(C::kACol0 + st * kAStageCols);
+                    const uint64_t bd = desc_sw128(smem_u32(smem + st * C::kStage));
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)  // 32 bytes of K per MMA
-                        mma_bf16_ss(d, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc,
+                    for (int kk = 0; kk < kBK / 16; ++kk)  // 16 k per MMA: 8 A columns, 32 B of B
+                        mma_bf16_ts(d, at + uint32_t(8 * kk), bd + uint64_t(2 * kk), idesc,
                                     (ks > it.ks_lo || kk > 0) ? 1u : 0u);
                     mma_commit(smem_u32(&empty[st]));
                     if (++st == STAGES) { st = 0; ph ^= 1u; }
@@ -409,6 +450,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp < kDeqWarps) {
         // ------------------------------------------------------- dequantise
+        // warp w writes row tile t = 2*(w%4) + w/4 (TMEM lanes 16t..16t+15,
+        // inside the lane quarter w%4 it may access)
+        const int tile = 2 * (warp & 3) + (warp >> 2);
+        const int r0 = lane >> 2, c = lane & 3;
+        const uint32_t lane_addr = uint32_t(16 * tile) << 16;
         int st = 0;
         uint32_t ph = 0;
         bool ok = true;
@@ -417,101 +463,73 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const Item it = item_at(i, prefix, a, nrb, nks);
             for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
                 if (!warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status)) { ok = false; break; }
-                uint8_t* sb = smem + st * C::kStage;
-                const uint8_t* pk = sb + kATile + C::kB;
+                const uint8_t* sb = smem + st * C::kStage;
+                const uint8_t* pk = sb + C::kB;
                 const uint8_t* sc = pk + C::kPacked;
-                constexpr int CHUNKS = (BITS == 4 ? 1 : 2);
+                const uint32_t at = tmem + lane_addr + uint32_t(C::kACol0 + st * kAStageCols);
+                constexpr int GROUPS = kBK / kgroup_of(BITS);  // 1 (int4) or 2 (int8)
 #pragma unroll
-                for (int q = 0; q < CHUNKS; ++q) {
-                    const int id = tid + q * (kDeqWarps * 32);
-                    const int gg = id >> 8;           // k-group inside the stage (int8: 0 or 1)
-                    const int tile = (id >> 5) & 7;
-                    const int ln = id & 31;
-                    const int r0 = ln >> 2, c = ln & 3;
-                    const int row0 = tile * 16 + r0, row1 = row0 + 8;
-                    const uint4 w = *reinterpret_cast<const uint4*>(pk + id * 16);
-                    // the lane's k range inside the stage
-                    const int k0 = BITS == 4 ? 16 * c : 32 * gg + 8 * c;
-                    uint32_t sa2 = 0, sb2 = 0;
-                    if (!PERCOL) {
-                        const int blk = a.block_size >= kBK ? 0 : k0 / a.block_size;
-                        const int si = (blk * kTilesPerBlock + tile) * 16 + 2 * r0;
-                        float sa, sbv;
-                        if (a.scale_bf16) {
-                            const uint32_t raw = *reinterpret_cast<const uint32_t*>(sc + si * 2);
-                            sa = __uint_as_float(raw << 16);
-                            sbv = __uint_as_float(raw & 0xFFFF0000u);
-                        } else {
-                            const float2 f = *reinterpret_cast<const float2*>(sc + si * 4);
-                            sa = f.x;
-                            sbv = f.y;
-                        }
-                        sa2 = bf2_bcast(sa);
-                        sb2 = bf2_bcast(sbv);
-                    }
-                    if (BITS == 4) {
-                        // 4 k-steps x 4 registers; register p of step j holds rows
-                        // (r0, r0+8, r0, r0+8)[p] at k offsets 4j + (0,0,2,2)[p] (+1)
-                        uint32_t r0v[8], r1v[8];
-                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                for (int gg = 0; gg < GROUPS; ++gg) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(pk + ((gg * kTilesPerBlock + tile) * 32 + lane) * 16);
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                    constexpr int KSTEPS = kgroup_of(BITS) / 16;
+                    uint32_t r[4 * KSTEPS];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint32_t A[4];
+                    for (int j = 0; j < KSTEPS; ++j) {
+                        uint32_t A[4];  // (r0, k 0-1), (r0+8, k 0-1), (r0, k 2-3), (r0+8, k 2-3)
+                        if (BITS == 4) {
                             A[0] = bf2_sub((wv[j] & kMask) | kMagic, kBias4);
                             A[1] = bf2_sub(((wv[j] >> 4) & kMask) | kMagic, kBias4);
                             A[2] = bf2_sub(((wv[j] >> 8) & kMask) | kMagic, kBias4);
                             A[3] = bf2_sub(((wv[j] >> 12) & kMask) | kMagic, kBias4);
-                            if (!PERCOL) {
-                                A[0] = bf2_mul(A[0], sa2);
-                                A[2] = bf2_mul(A[2], sa2);
-                                A[1] = bf2_mul(A[1], sb2);
-                                A[3] = bf2_mul(A[3], sb2);
-                            }
-                            r0v[2 * j] = A[0];      // row0, k 4j, 4j+1
-                            r0v[2 * j + 1] = A[2];  // row0, k 4j+2, 4j+3
-                            r1v[2 * j] = A[1];
-                            r1v[2 * j + 1] = A[3];
-                        }
-                        *reinterpret_cast<uint4*>(sb + a_off(row0, k0)) = make_uint4(r0v[0], r0v[1], r0v[2], r0v[3]);
-                        *reinterpret_cast<uint4*>(sb + a_off(row0, k0 + 8)) = make_uint4(r0v[4], r0v[5], r0v[6], r0v[7]);
-                        *reinterpret_cast<uint4*>(sb + a_off(row1, k0)) = make_uint4(r1v[0], r1v[1], r1v[2], r1v[3]);
-                        *reinterpret_cast<uint4*>(sb + a_off(row1, k0 + 8)) = make_uint4(r1v[4], r1v[5], r1v[6], r1v[7]);
-                    } else {
-                        // 2 k-steps of 8 bytes; byte pair q of a step holds rows
-                        // (r0, r0+8, r0, r0+8)[q] at k offsets 4j + (0,0,2,2)[q] (+1).
-                        // A byte b is q - 128 = (b & 127) - (b >= 128 ? 0 : 128): OR the low
-                        // 7 bits into bf16 128.0 and subtract 256.0 or 128.0 (0x4380 with
-                        // the exponent bit flipped by the byte's top bit), both exact.
-                        uint32_t r0v[4], r1v[4];
-                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            uint32_t A[4];
+                        } else {
+                            // byte b holds q - 128 = (b & 127) - (b < 128 ? 128 : 0): OR the
+                            // low 7 bits into bf16 128.0 and subtract 256.0 or 128.0 (0x4380
+                            // with its exponent bit flipped by the byte's top bit), exactly
 #pragma unroll
                             for (int qq = 0; qq < 4; ++qq) {
                                 const uint32_t word = wv[2 * j + (qq >> 1)];
-                                // bytes (0,1) or (2,3) of the word into the low byte of each half
                                 const uint32_t pr = __byte_perm(word, 0u, (qq & 1) ? 0x4342u : 0x4140u);
                                 const uint32_t lo = (pr & 0x007F007Fu) | 0x43004300u;
                                 const uint32_t hi = (pr & 0x00800080u) ^ 0x43804380u;
                                 A[qq] = bf2_sub(lo, hi);
                             }
-                            if (!PERCOL) {
-                                A[0] = bf2_mul(A[0], sa2);
-                                A[2] = bf2_mul(A[2], sa2);
-                                A[1] = bf2_mul(A[1], sb2);
-                                A[3] = bf2_mul(A[3], sb2);
-                            }
-                            r0v[2 * j] = A[0];
-                            r0v[2 * j + 1] = A[2];
-                            r1v[2 * j] = A[1];
-                            r1v[2 * j + 1] = A[3];
                         }
-                        *reinterpret_cast<uint4*>(sb + a_off(row0, k0)) = make_uint4(r0v[0], r0v[1], r0v[2], r0v[3]);
-                        *reinterpret_cast<uint4*>(sb + a_off(row1, k0)) = make_uint4(r1v[0], r1v[1], r1v[2], r1v[3]);
+                        if (!PERCOL) {
+                            // scale block of this k-step (k = 64*ks + 32*gg + 16j + 4c + ...)
+                            const int kl = 32 * gg * (BITS == 8) + 16 * j + 4 * c;
+                            const int blk = a.block_size >= kBK ? 0 : kl / a.block_size;
+                            const int si = (blk * kTilesPerBlock + tile) * 16 + 2 * r0;
+                            float sa, sbv;
+                            if (a.scale_bf16) {
+                                const uint32_t raw = *reinterpret_cast<const uint32_t*>(sc + si * 2);
+                                sa = __uint_as_float(raw << 16);
+                                sbv = __uint_as_float(raw & 0xFFFF0000u);
+                            } else {
+                                const float2 f = *reinterpret_cast<const float2*>(sc + si * 4);
+                                sa = f.x;
+                                sbv = f.y;
+                            }
+                            const uint32_t sa2 = bf2_bcast(sa), sb2 = bf2_bcast(sbv);
+                            A[0] = bf2_mul(A[0], sa2);
+                            A[2] = bf2_mul(A[2], sa2);
+                            A[1] = bf2_mul(A[1], sb2);
+                            A[3] = bf2_mul(A[3], sb2);
+                        }
+                        // 16x256b fragment: (r0, col 2c), (r0, col 2c+1), (r0+8, col 2c), (r0+8, col 2c+1)
+                        r[4 * j + 0] = A[0];
+                        r[4 * j + 1] = A[2];
+                        r[4 * j + 2] = A[1];
+                        r[4 * j + 3] = A[3];
+                    }
+                    if (BITS == 4) {
+                        tmem_st16x256_x4(at, *reinterpret_cast<const uint32_t(*)[16]>(r));
+                    } else {
+                        tmem_st16x256_x2(at + uint32_t(16 * gg), *reinterpret_cast<const uint32_t(*)[8]>(r));
                     }
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&deq[st]));
                 if (++st == STAGES) { st = 0; ph ^= 1u; }
@@ -519,7 +537,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp >= kWarpEpi0) {
         // ------------------------------------------------------- epilogue
-        const int qd = warp & 3;  // TMEM lane quarter this warp may read
+        const int qd = warp & 3;                        // TMEM lane quarter this warp may read
+        const int half = (warp - kWarpEpi0) >> 2;       // which 16-column chunks it takes
         const int row = qd * 32 + lane;
         int acc = 0;
         uint32_t aph = 0;
@@ -531,15 +550,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const bool valid = prow < a.N;
             float s = 1.0f;
             if (PERCOL && valid) {
-                const int tile = row >> 4, rr = row & 15;
-                const int64_t si = ((int64_t(it.e) * nrb + it.rb) * kTilesPerBlock + tile) * 16 + (rr & 7) * 2 + (rr >> 3);
+                const int tl = row >> 4, rr = row & 15;
+                const int64_t si = ((int64_t(it.e) * nrb + it.rb) * kTilesPerBlock + tl) * 16 + (rr & 7) * 2 + (rr >> 3);
                 s = a.scale_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.S)[si])
                                  : reinterpret_cast<const float*>(a.S)[si];
             }
             const float bias = (a.bias && valid) ? a.bias[int64_t(it.e) * a.N + prow] : 0.0f;
             const uint32_t tbase = tmem + (uint32_t(qd * 32) << 16) + uint32_t(acc * BNMAX);
             const int ncol = ((it.rows + 15) / 16) * 16;
-            for (int c0 = 0; c0 < ncol; c0 += 16) {
+            for (int c0 = 16 * half; c0 < ncol; c0 += 32) {
                 float v[16];
                 tmem_ld16(tbase + uint32_t(c0), v);
 #pragma unroll
@@ -602,7 +621,9 @@ EncodeTiledFn encode_fn() {
 template <int BITS, bool PERCOL, int BNMAX>
 struct Launch {
     static constexpr int kStage = TcCfg<BITS, PERCOL, BNMAX, 1>::kStage;
-    static constexpr int kStages = ((220 * 1024) / kStage) > 8 ? 8 : ((220 * 1024) / kStage);
+    static constexpr int kByTmem = (512 - 2 * BNMAX) / kAStageCols;
+    static constexpr int kBySmem = (200 * 1024) / kStage;
+    static constexpr int kStages = kByTmem < kBySmem ? (kByTmem < 12 ? kByTmem : 12) : (kBySmem < 12 ? kBySmem : 12);
     using C = TcCfg<BITS, PERCOL, BNMAX, kStages>;
     static cudaError_t prepare() {
         return cudaFuncSetAttribute(ffn_tc_kernel<BITS, PERCOL, BNMAX, kStages>,
@@ -620,8 +641,7 @@ cudaError_t dispatch_bn(int bnmax, const CUtensorMap& map, const TcArgs& a, int 
         case 16: return Launch<BITS, PERCOL, 16>::run(map, a, grid, st);
         case 32: return Launch<BITS, PERCOL, 32>::run(map, a, grid, st);
         case 64: return Launch<BITS, PERCOL, 64>::run(map, a, grid, st);
-        case 128: return Launch<BITS, PERCOL, 128>::run(map, a, grid, st);
-        default: return Launch<BITS, PERCOL, 256>::run(map, a, grid, st);
+        default: return Launch<BITS, PERCOL, 128>::run(map, a, grid, st);
     }
 }
 
@@ -631,7 +651,6 @@ cudaError_t prepare_bits() {
     if (e == cudaSuccess) e = Launch<BITS, PERCOL, 32>::prepare();
     if (e == cudaSuccess) e = Launch<BITS, PERCOL, 64>::prepare();
     if (e == cudaSuccess) e = Launch<BITS, PERCOL, 128>::prepare();
-    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 256>::prepare();
     return e;
 }
 
@@ -671,13 +690,13 @@ cudaError_t launch_ffn_tc(const FfnArgs& f, int bn, int32_t* status, cudaStream_
     if (!enc) return cudaErrorNotSupported;
     int bnmax = 16;
     while (bnmax < bn) bnmax *= 2;
-    if (bnmax > 256) return cudaErrorInvalidValue;
+    if (bnmax > 128) return cudaErrorInvalidValue;
     // activations: [rows, K] bf16; rows = R (permuted rows)
     const int64_t rows = f.R;
     CUtensorMap map;
     const cuuint64_t dims[2] = {cuuint64_t(f.K), cuuint64_t(rows)};
     const cuuint64_t strides[1] = {cuuint64_t(f.K * 2)};
-    const cuuint32_t box[2] = {cuuint32_t(kBK), cuuint32_t(bnmax)};
+    const cuuint32_t box[2] = {cuuint32_t(kBK), cuuint32_t(bnmax < 64 ? bnmax : 64)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(f.act), dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -59,12 +59,12 @@ __global__ void pack_codes_kernel(PackArgs a) {
         const int r0 = lane >> 2, c = lane & 3;
         uint32_t words[4] = {0u, 0u, 0u, 0u};
         if (rt < nrt && a.bits == 4) {
-            // word j, nibble p: row r0 + 8*(p&1), k = 64g + 16c + 4j + 2*((p>>1)&1) + (p>>2)
+            // word j, nibble p: row r0 + 8*(p&1), k = 64g + 16j + 4c + 2*((p>>1)&1) + (p>>2)
             for (int j = 0; j < 4; ++j) {
                 uint32_t w = 0;
                 for (int p = 0; p < 8; ++p) {
                     const int rr = r0 + 8 * (p & 1);
-                    const int64_t k = g * 64 + 16 * c + 4 * j + 2 * ((p >> 1) & 1) + (p >> 2);
+                    const int64_t k = g * 64 + 16 * j + 4 * c + 2 * ((p >> 1) & 1) + (p >> 2);
                     const SrcRow s = source_row(a.mode, rt, rr, a.I);
                     const uint8_t* base = s.which ? a.src_up : a.src;
                     const uint8_t* rowp = base + (e * src_rows + s.row) * row_bytes;
@@ -74,7 +74,7 @@ __global__ void pack_codes_kernel(PackArgs a) {
             }
         } else if (rt < nrt) {
             // kstep j (8 bytes), byte m: pair q = m/2 -> row r0 + 8*(q&1),
-            // k = 32g + 8c + 4j + 2*(q>>1) + (m&1)
+            // k = 32g + 16j + 4c + 2*(q>>1) + (m&1)
             for (int j = 0; j < 2; ++j) {
                 for (int half = 0; half < 2; ++half) {
                     uint32_t w = 0;
@@ -82,7 +82,7 @@ __global__ void pack_codes_kernel(PackArgs a) {
                         const int m = half * 4 + mb;
                         const int q = m >> 1;
                         const int rr = r0 + 8 * (q & 1);
-                        const int64_t k = g * 32 + 8 * c + 4 * j + 2 * (q >> 1) + (m & 1);
+                        const int64_t k = g * 32 + 16 * j + 4 * c + 2 * (q >> 1) + (m & 1);
                         const SrcRow s = source_row(a.mode, rt, rr, a.I);
                         const uint8_t* base = s.which ? a.src_up : a.src;
                         const uint8_t* rowp = base + (e * src_rows + s.row) * row_bytes;

@@ -20,14 +20,16 @@ namespace qmoe {
 // A weight W[N, K] of one expert (N output rows, K reduction) is cut into row
 // tiles of 16 rows and k-groups of KG (64 for 4-bit codes, 32 for 8-bit). One
 // (row tile, k-group) unit is 512 bytes: lane L of a warp owns rows r0 = L/4
-// and r0 + 8 of the tile and the k sub-range [KG/4 * (L%4), KG/4 * (L%4 + 1))
-// of the group, 16 bytes -- exactly the operand fragments of an m16n8k16 bf16
-// MMA whose k axis is permuted the same way for weights and activations (see
-// ffn_decode.cu). Units are ordered [N/128 row blocks][K/KG groups][8 row
-// tiles], so a 128-row x KG slab (one tensor-core stage) is one contiguous
-// 4 KB run and a row tile walks K with a 4 KB stride. N is padded to a
-// multiple of 128 with zero codes. Bytes are the page's codes, re-laid,
-// never decoded.
+// and r0 + 8 of the tile and, with c = L%4, the k values 16j + 4c + {0..3}
+// of the group for j = 0 .. KG/16 - 1 -- 16 bytes. Word (int4) or word pair
+// (int8) j holds the codes of k-step j in the order of the m16n8k16 MMA A
+// fragment, which is also the register order of a 16x256b tensor-memory
+// store: registers (row r0, k 16j+4c+{0,1}), (row r0+8, same), (row r0,
+// k 16j+4c+{2,3}), (row r0+8, same). Units are ordered [N/128 row blocks]
+// [K/KG groups][8 row tiles], so a 128-row x KG slab (one tensor-core stage)
+// is one contiguous 4 KB run and a row tile walks K with a 4 KB stride. N is
+// padded to a multiple of 128 with zero codes. Bytes are the page's codes,
+// re-laid, never decoded.
 //
 // FC1 of a gated FFN is re-laid so that row tile t holds gate rows
 // i = 8t..8t+7 in its first 8 rows and the matching up rows in its last 8,
