@@ -212,6 +212,33 @@ QMOE_API qmoe_status qmoe_debug_hidden(const qmoe_handle* h, int64_t T, const vo
  */
 QMOE_API qmoe_status qmoe_read_device_status(const qmoe_handle* h, const void* workspace, void* stream);
 
+/*
+ * qmoe_forward_noalloc -- qmoe_forward without a caller workspace. (The
+ * operator pages have no counterpart; this is a deployment convenience.)
+ *
+ * For callers that cannot allocate device memory where they run the operator
+ * -- a plugin whose host framework owns all device memory and passes in only
+ * the input and output buffers, or a serving loop that must not allocate while
+ * it handles a request. The scratch is one fixed library-owned device array of
+ * qmoe_noalloc_scratch_bytes() bytes (8 MiB), which every GPU that loads the
+ * library holds until the process exits. Arguments are qmoe_forward's minus
+ * the workspace; a T whose qmoe_workspace_size exceeds the array returns
+ * QMOE_INVALID_ARGUMENT with the sizes in qmoe_last_error. Nothing is allocated
+ * or freed.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. All calls share the one array, which keeps the
+ * last call's contents: calls whose GPU work can overlap (other streams,
+ * other host threads) race on it and must be serialised by the caller.
+ */
+QMOE_API qmoe_status qmoe_forward_noalloc(const qmoe_handle* h, int64_t T, const void* x,
+                                          const void* router_logits, const void* shared_output,
+                                          void* y, void* stream);
+
+/* Size in bytes of the fixed scratch array behind qmoe_forward_noalloc. */
+QMOE_API size_t qmoe_noalloc_scratch_bytes(void);
+
 /* qmoe_destroy -- "ClikaRT::nn::QMoEWoQ", ~QMoEWoQ(): release the packed
  * weights and the handle. NULL is a no-op. */
 QMOE_API void qmoe_destroy(qmoe_handle* h);

@@ -35,7 +35,7 @@ EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forwa
            "qmoe_forward_profiled",
            "qmoe_debug_routing", "qmoe_debug_hidden", "qmoe_read_device_status", "qmoe_destroy",
            "qmoe_status_string", "qmoe_last_error", "qmoe_path_for", "qmoe_launches_for",
-           "qmoe_set_option")
+           "qmoe_set_option", "qmoe_forward_noalloc", "qmoe_noalloc_scratch_bytes")
 QMOE_OPT_PATH = 1
 
 
@@ -78,6 +78,10 @@ lib.qmoe_last_error.restype = ctypes.c_char_p
 lib.qmoe_last_error.argtypes = [_vp]
 lib.qmoe_path_for.restype = ctypes.c_int32
 lib.qmoe_path_for.argtypes = [_vp, _i64]
+lib.qmoe_forward_noalloc.restype = ctypes.c_int
+lib.qmoe_forward_noalloc.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp]
+lib.qmoe_noalloc_scratch_bytes.restype = _sz
+lib.qmoe_noalloc_scratch_bytes.argtypes = []
 lib.qmoe_set_option.restype = ctypes.c_int
 lib.qmoe_set_option.argtypes = [_vp, ctypes.c_int32, _i64]
 lib.qmoe_launches_for.restype = ctypes.c_int32
@@ -153,6 +157,17 @@ def qmoe_forward(h, T, x, router_logits, shared_output, y, workspace, workspace_
                             _ptr(workspace), workspace_bytes, _stream(stream)), h)
 
 
+def qmoe_forward_noalloc(h, T, x, router_logits, shared_output, y, stream=None):
+    """The forward with its scratch in the library's fixed device array (no
+    workspace argument, nothing allocated); see include/qmoe.h."""
+    _check(lib.qmoe_forward_noalloc(h, T, _ptr(x), _ptr(router_logits), _ptr(shared_output), _ptr(y),
+                                    _stream(stream)), h)
+
+
+def qmoe_noalloc_scratch_bytes() -> int:
+    return int(lib.qmoe_noalloc_scratch_bytes())
+
+
 def qmoe_forward_profiled(h, T, x, router_logits, shared_output, y, workspace, workspace_bytes,
                           events, stream=None):
     """``events``: torch.cuda.Event objects (timing enabled, already created by
@@ -221,8 +236,8 @@ class QMoE:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
-            qmoe_destroy(h)
+        if h and lib is not None:
+            lib.qmoe_destroy(h)
             self.handle = None
 
     def set_weights(self, fc1_w, fc1_s, fc2_w, fc2_s, fc1_b=None, fc2_b=None, fc3_w=None, fc3_s=None,
