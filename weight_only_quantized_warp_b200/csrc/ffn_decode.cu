@@ -68,6 +68,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A*B (accumulator input zero): starts a fresh partial without zeroing registers
+__device__ __forceinline__ void mma_bf16_zero(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
     __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
                                *reinterpret_cast<__nv_bfloat162*>(&b));
@@ -386,7 +396,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
 
         // one k-group: decode the lane's 16 bytes, 4 (int4) or 2 (int8) MMA
         // k-steps per token tile. xg is this lane's activation run of the group.
-        auto group = [&](const uint4 w, const uint8_t* xg, const ScaleRaw<SF32> sc, int ga) {
+        // first: this group opens a scale chunk (SMODE 1), so its first k-step
+        // writes the chunk partial instead of adding to it
+        auto group = [&](const uint4 w, const uint8_t* xg, const ScaleRaw<SF32> sc, int ga, bool first) {
             uint2 xa[NT][KSTEPS];  // per k-step: activation pairs at 16j+4c, 16j+4c+2
 #pragma unroll
             for (int n = 0; n < NT; ++n)
@@ -441,10 +453,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
                 }
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
-                    if (SMODE == 1)
-                        mma_bf16(blk[n], A, xa[n][j].x, xa[n][j].y);
-                    else
+                    if (SMODE == 1) {
+                        if (first && j == 0)
+                            mma_bf16_zero(blk[n], A, xa[n][j].x, xa[n][j].y);
+                        else
+                            mma_bf16(blk[n], A, xa[n][j].x, xa[n][j].y);
+                    } else {
                         mma_bf16(acc[n], A, xa[n][j].x, xa[n][j].y);
+                    }
                 }
             }
         };
@@ -465,7 +481,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
                 acc[n][1] = fmaf(sa, blk[n][1], acc[n][1]);
                 acc[n][2] = fmaf(sb, blk[n][2], acc[n][2]);
                 acc[n][3] = fmaf(sb, blk[n][3], acc[n][3]);
-                blk[n][0] = blk[n][1] = blk[n][2] = blk[n][3] = 0.0f;
             }
         };
 
@@ -473,19 +488,18 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
             const uint8_t* wn = wp + D * GS;                      // loads run D groups ahead
             const uint8_t* xp = xs + r0 * rs + 8 * c;  // this lane's first pair, group 0
             const float* csp = cs + 2 * c;                        // chunk 0, tokens 2c, 2c+1
-            ScaleRaw<SF32> scur = sr[0];
             int g = 0;  // group relative to g_lo
             // steady rounds: every prefetch is in range
             for (; g + 2 * D <= ng; g += D) {
 #pragma unroll
                 for (int i = 0; i < D; ++i) {
                     // use slot i, then refill it (no register copy of the old value)
-                    if (SMODE == 1 && i % P == 0) scur = sr[i / P];
-                    group(wr[i], xp + i * KG * 2, scur, int(g_lo) + g + i);
+                    group(wr[i], xp + i * KG * 2, sr[0], int(g_lo) + g + i, i % P == 0);
                     wr[i] = ld_stream(wn + i * GS);
-                    if (SMODE == 1 && i % P == P - 1)
+                    if (SMODE == 1 && i % P == P - 1) {
+                        apply(sr[i / P], csp + (i / P) * ROWS);
                         sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + 1 - P + D));
-                    if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
+                    }
                 }
                 wn += D * GS;
                 xp += D * KG * 2;
@@ -495,12 +509,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
             if (g + D <= ng) {
 #pragma unroll
                 for (int i = 0; i < D; ++i) {
-                    if (SMODE == 1 && i % P == 0) scur = sr[i / P];
-                    group(wr[i], xp + i * KG * 2, scur, int(g_lo) + g + i);
+                    group(wr[i], xp + i * KG * 2, sr[0], int(g_lo) + g + i, i % P == 0);
                     if (g + i + D < ng) wr[i] = ld_stream(wn + i * GS);
-                    if (SMODE == 1 && i % P == P - 1 && g + i + 1 - P + D < ng)
-                        sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + 1 - P + D));
-                    if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
+                    if (SMODE == 1 && i % P == P - 1) {
+                        apply(sr[i / P], csp + (i / P) * ROWS);
+                        if (g + i + 1 - P + D < ng)
+                            sr[i / P] = ScaleRaw<SF32>::load(sbase, sidx(int(g_lo) + g + i + 1 - P + D));
+                    }
                 }
                 g += D;
                 xp += D * KG * 2;
@@ -510,9 +525,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
 #pragma unroll
             for (int i = 0; i < D; ++i) {
                 if (g + i < ng) {
-                    if (SMODE == 1 && i % P == 0) scur = sr[i / P];
-                    group(wr[i], xp + i * KG * 2, scur, int(g_lo) + g + i);
-                    if (SMODE == 1 && i % P == P - 1) apply(scur, csp + (i / P) * ROWS);
+                    group(wr[i], xp + i * KG * 2, sr[0], int(g_lo) + g + i, i % P == 0);
+                    if (SMODE == 1 && i % P == P - 1) apply(sr[i / P], csp + (i / P) * ROWS);
                 }
             }
 
