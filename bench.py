@@ -44,7 +44,8 @@ def parse():
     ap.add_argument("--workload", default="mixtral_decode")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", type=int, default=None,
-                    help="force the expert-FFN kernels: 1 weight-streaming, 2 tcgen05 (default: by shape)")
+                    help="force the expert-FFN kernels: 1 mma.sync streaming, 2 tcgen05 GEMM, "
+                         "3 tcgen05 streaming (default: by shape)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0,
                     help="tokens in the CPU-baseline sample (0: whole batch, capped by time)")
@@ -217,7 +218,7 @@ def run_reference(args):
 def run_ours(args):
     import torch
     import torch.distributed as dist
-    from weight_only_quantized_warp_b200 import qmoe
+    from weight_only_quantized_warp_b200 import qmoe, replicas
 
     world, rank, local = dist_env()
     if world > 1:
@@ -226,11 +227,9 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    cfg, seed, kw = gen.workload(args.workload)
-    inp = gen.make_inputs(cfg, seed, **kw)
-    if world > 1 and rank > 0:  # each replica its own token batch, same weights
-        other = gen.make_inputs(dataclasses_replace(cfg), seed + 1000 * rank, **kw)
-        inp.x, inp.logits, inp.shared = other.x, other.logits, other.shared
+    # every replica: the same weights, its own token batch
+    inp = replicas.replica_inputs(args.workload, rank)
+    cfg = inp.cfg
 
     m = qmoe.QMoE(cfg, dev, path=args.path)
     m.set_weights_from(inp)
@@ -290,16 +289,13 @@ def run_ours(args):
     clk = clocks.stop()
     if clk is not None:
         clk["window"] = "timed region bracketed by 0.6 s / 0.4 s of the same forward"
-    ms = start.elapsed_time(stop)
+    ms = replicas.max_over_ranks([start.elapsed_time(stop)], dev)[0]
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(launches)]
                            for i in range(K)]).mean(axis=0)
     path = qmoe.qmoe_path_for(h, T)
-    names = (["route", "permute", "gather", "fc1", "fc2", "combine"] if path == qmoe.PATH_TC
+    names = (["route", "permute", "gather", "fc1", "fc2", "combine"] if path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE)
              else ["route", "permute", "fc1", "fc2", "combine"])[:launches]
 
     # ---- end to end through the public call, host buffers, copies inside
@@ -329,11 +325,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = replicas.max_over_ranks([e0.elapsed_time(e1)], dev)[0]
     h2d = x_h.numel() * x_h.element_size() + lg_h.numel() * lg_h.element_size() + (
         0 if sh_h is None else sh_h.numel() * sh_h.element_size())
     d2h = y_h.numel() * y_h.element_size()
@@ -357,8 +349,7 @@ def run_ours(args):
     kms = dict(zip(names, [float(v) for v in per_kernel]))
     fc1_ms = kms["fc1"]
     step_ms = ms / K
-    tokens = T * world * K
-    value = tokens / (ms / 1e3)
+    value = replicas.job_tokens_per_s(T, world, K, ms)
     # dominant kernel by algorithmic work: FC1 (gate + up rows); its bound is
     # the slower of its bytes at HBM bandwidth and its FLOPs at bf16 peak
     hbm_peak = float(peaks["hbm_gbs"])
@@ -366,8 +357,10 @@ def run_ours(args):
     fc1_flops = 2.0 * cfg.T * cfg.k * (cfg.n1 + (cfg.I if cfg.has_fc3 else 0)) * cfg.H
     t_hbm = alg["fc1_bytes"] / (hbm_peak * 1e9)
     t_tc = fc1_flops / (tc_peak * 1e12)
-    kname = "ffn_tc_kernel (FC1 + SwiGLU)" if path == qmoe.PATH_TC else "ffn_decode_kernel (FC1 + SwiGLU)"
-    tr = traffic_record(("fc1_tc_" if path == qmoe.PATH_TC else "fc1_decode_") + args.workload)
+    kname = {qmoe.PATH_TC: "ffn_tc_kernel (FC1 + SwiGLU)",
+             qmoe.PATH_TC_DECODE: "ffn_tc_decode_kernel (FC1 + SwiGLU)"}.get(path, "ffn_decode_kernel (FC1 + SwiGLU)")
+    tr = traffic_record({qmoe.PATH_TC: "fc1_tc_", qmoe.PATH_TC_DECODE: "fc1_tcdecode_"}.get(path, "fc1_decode_")
+                        + args.workload)
     if t_hbm >= t_tc:
         achieved = alg["fc1_bytes"] / (fc1_ms / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -392,17 +385,12 @@ def run_ours(args):
                      "algorithmic_bytes": alg["total_bytes"],
                      "kernel_ms": kms, "path": path},
             "cpu_baseline": cpu,
-            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": replicas.job_tokens_per_s(T, world, K, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches * K,
             "clocks": clk}
     print(json.dumps(line), flush=True)
     return 0
-
-
-def dataclasses_replace(cfg):
-    import dataclasses
-    return dataclasses.replace(cfg)
 
 
 def main():

@@ -252,8 +252,11 @@ QMOE_API const char* qmoe_last_error(const qmoe_handle* h);
 
 /* Tunable options (qmoe_set_option). QMOE_OPT_PATH selects the expert-FFN
  * kernels for bf16 activations: -1 (default) chooses by shape, 1 forces the
- * weight-streaming decode kernels, 2 the tcgen05 grouped GEMM. fp32
- * activations always take the fp32 path (0). */
+ * weight-streaming mma.sync kernels, 2 the tcgen05 grouped GEMM, 3 the
+ * tcgen05 streaming decode kernels (falls back to 1 for shapes they do not
+ * cover: more than 32 rows per expert, K not a multiple of 128, or a K range
+ * whose resident activations exceed 128 KB). fp32 activations always take
+ * the fp32 path (0). */
 enum { QMOE_OPT_PATH = 1 };
 
 /* qmoe_set_option -- set a tunable option on the handle. QMOE_INVALID_ARGUMENT
@@ -262,8 +265,8 @@ enum { QMOE_OPT_PATH = 1 };
 QMOE_API qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t value);
 
 /* The forward path qmoe_forward takes for T tokens: 0 = fp32 SIMT path,
- * 1 = weight-streaming decode path (mma.sync), 2 = tcgen05 grouped GEMM.
- * -1 for a NULL handle. */
+ * 1 = weight-streaming decode path (mma.sync), 2 = tcgen05 grouped GEMM,
+ * 3 = tcgen05 streaming decode. -1 for a NULL handle. */
 QMOE_API int32_t qmoe_path_for(const qmoe_handle* h, int64_t T);
 
 /* Number of kernel launches qmoe_forward enqueues for T tokens. */

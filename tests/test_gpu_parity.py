@@ -63,6 +63,14 @@ CASES = {
                    act=gen.ACT_SILU, normalize=False),
     "k_equals_E": dict(T=9, E=4, k=4),
     "t1": dict(T=1),
+    # shapes the streaming tensor-core kernels take (H, I multiples of 128)
+    "k128_int4_bs32_bias": dict(H=256, I=384, block_size=32, fusion=1, has_fc1_bias=True, has_fc2_bias=True),
+    "k128_int4_bs16_f32scales": dict(H=256, I=384, block_size=16, scale_dtype=gen.DT_F32),
+    "k128_int4_percol": dict(H=256, I=384, block_size=0),
+    "k128_int8_bs64_fc3": dict(H=256, I=384, bits=8, block_size=64, fusion=0, has_fc3=True,
+                               act=gen.ACT_SILU),
+    "k128_int8_percol_relu": dict(H=256, I=384, bits=8, block_size=0, fusion=0, act=gen.ACT_RELU),
+    "k128_t32_tile32": dict(H=256, I=384, T=96, E=8, k=2),
     "fp32_acts_int8": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, bits=8, block_size=32,
                            has_fc1_bias=True, has_fc2_bias=True, has_shared=True),
     "fp32_acts_percol_fc3": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_BF16, block_size=0,
@@ -70,18 +78,23 @@ CASES = {
 }
 
 
-PATH_DECODE, PATH_TC = 1, 2
+PATH_DECODE, PATH_TC, PATH_TC_DECODE = 1, 2, 3
 
 
-@pytest.mark.parametrize("path", [PATH_DECODE, PATH_TC], ids=["decode", "tc"])
+@pytest.mark.parametrize("path", [PATH_DECODE, PATH_TC, PATH_TC_DECODE], ids=["decode", "tc", "tcdecode"])
 @pytest.mark.parametrize("name", list(CASES))
 def test_parity_small(cuda_device, name, path):
     cfg = _cfg(**CASES[name])
-    if cfg.act_dtype == gen.DT_F32 and path == PATH_TC:
+    if cfg.act_dtype == gen.DT_F32 and path != PATH_DECODE:
         pytest.skip("fp32 activations always take the fp32 path")
     inp = gen.make_inputs(cfg, seed=100 + list(CASES).index(name), bias_std=0.1)
     g = run_gpu(inp, path=path)
-    assert g.path == (0 if cfg.act_dtype == gen.DT_F32 else path)
+    if cfg.act_dtype == gen.DT_F32:
+        assert g.path == 0
+    elif path == PATH_TC_DECODE:
+        assert g.path in (PATH_TC_DECODE, PATH_DECODE)
+    else:
+        assert g.path == path
     check_full(inp, g)
 
 
@@ -120,7 +133,7 @@ def test_zero_tokens_is_a_noop(cuda_device):
     torch.cuda.synchronize()
 
 
-@pytest.mark.parametrize("path", [PATH_DECODE, PATH_TC], ids=["decode", "tc"])
+@pytest.mark.parametrize("path", [PATH_DECODE, PATH_TC, PATH_TC_DECODE], ids=["decode", "tc", "tcdecode"])
 def test_repeated_forward_is_bitwise_deterministic(cuda_device, path):
     cfg = _cfg(T=50, bits=4, block_size=128, H=384, I=640)
     inp = gen.make_inputs(cfg, seed=8)
@@ -154,7 +167,7 @@ def _sample(T, n=8, seed=0):
     return np.sort(rng.choice(T, size=min(n, T), replace=False))
 
 
-@pytest.mark.parametrize("path", [None, PATH_DECODE, PATH_TC], ids=["auto", "decode", "tc"])
+@pytest.mark.parametrize("path", [None, PATH_DECODE, PATH_TC, PATH_TC_DECODE], ids=["auto", "decode", "tc", "tcdecode"])
 @pytest.mark.parametrize("name", ["mixtral_decode", "gpt_oss", "deepseek"])
 def test_full_size_configs(cuda_device, name, path):
     cfg, seed, kw = gen.workload(name)
@@ -164,9 +177,10 @@ def test_full_size_configs(cuda_device, name, path):
     check_sampled(inp, g, tokens)
 
 
+@pytest.mark.parametrize("path", [None, PATH_TC_DECODE], ids=["auto", "tcdecode"])
 @pytest.mark.parametrize("bits,T", [(4, 1), (4, 16), (8, 1), (8, 128), (4, 1024)])
-def test_sweep_configs(cuda_device, bits, T):
+def test_sweep_configs(cuda_device, bits, T, path):
     cfg, seed, kw = gen.sweep(bits, T)
     inp = gen.make_inputs(cfg, seed, **kw)
-    g = run_gpu(inp)
+    g = run_gpu(inp, path=path)
     check_sampled(inp, g, _sample(T, 4, seed))

@@ -30,13 +30,28 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size;
     const int bits = c.expert_weight_bits, bs = c.block_size;
     const int64_t per_expert = ceil_div(std::max<int64_t>(p.R, 1), E);
+    const int64_t touched = std::min<int64_t>(E, std::max<int64_t>(p.R, 1));
+    // streaming decode on the tensor cores: token tile 16 or 32, FC1 unsplit,
+    // FC2 split until every SM has work and each split's activations fit
+    const int tcd_bn = per_expert <= 16 ? 16 : 32;
+    int tcd_s2 = 1;
+    const int64_t max_s2 = std::max<int64_t>(1, I / 128);  // every split keeps >= one 128-k stage
+    while (tcd_s2 < max_s2 && (!tc_decode_fits(I, tcd_s2, tcd_bn) ||
+                               touched * (padded_rows(H) / kBlockRows) * tcd_s2 < 4 * kSms))
+        ++tcd_s2;
+    const bool tcd_ok = per_expert <= 32 && tc_decode_fits(H, 1, tcd_bn) && tc_decode_fits(I, tcd_s2, tcd_bn);
     if (!bf16)
         p.path = kPathSimt;
     else if (h.path_override == kPathDecode || h.path_override == kPathTc)
         p.path = h.path_override;
+    else if (h.path_override == kPathTcDecode)
+        p.path = tcd_ok ? kPathTcDecode : kPathDecode;
     else
         p.path = per_expert <= kDecodeRowsPerExpert ? kPathDecode : kPathTc;
-    const int64_t touched = std::min<int64_t>(E, std::max<int64_t>(p.R, 1));
+    if (p.path == kPathTcDecode) {
+        p.bn = tcd_bn;
+        p.fc2_splits = tcd_s2;
+    }
     if (p.path == kPathDecode) {
         p.nt = per_expert <= 8 ? 1 : (per_expert <= 16 ? 2 : 4);
         // FC1 runs unsplit; keep its staged rows small enough for two CTAs per SM
@@ -64,7 +79,7 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         while (items * s < 2 * kSms && s < 8 && s * 2 <= I / 64) s *= 2;
         p.fc2_splits = int(s);
     }
-    p.launches = p.path == kPathTc ? 6 : 5;
+    p.launches = (p.path == kPathTc || p.path == kPathTcDecode) ? 6 : 5;
     const size_t R = size_t(p.R);
     const size_t act = bf16 ? 2 : 4;
     size_t off = 0;
@@ -75,7 +90,8 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     p.off_perm = off;    off = align256(off + R * 4);
     p.off_offsets = off; off = align256(off + size_t(E + 1) * 4);
     p.off_h = off;       off = align256(off + R * size_t(I) * act);
-    p.off_xperm = off;   off = align256(off + (p.path == kPathTc ? R * size_t(H) * act : 0));
+    p.off_xperm = off;
+    off = align256(off + ((p.path == kPathTc || p.path == kPathTcDecode) ? R * size_t(H) * act : 0));
     p.off_o = off;       off = align256(off + size_t(p.fc2_splits) * R * size_t(H) * 4);
     p.total = off;
     return p;
@@ -308,8 +324,8 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
 qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t value) {
     if (!h) return QMOE_INVALID_ARGUMENT;
     if (option == QMOE_OPT_PATH) {
-        if (value != -1 && value != kPathDecode && value != kPathTc)
-            return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_PATH must be -1, 1 or 2");
+        if (value != -1 && value != kPathDecode && value != kPathTc && value != kPathTcDecode)
+            return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_PATH must be -1, 1, 2 or 3");
         h->path_override = int(value);
         return QMOE_OK;
     }
@@ -424,7 +440,7 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     f2.is_fc1 = 0;
     f2.splits = p.fc2_splits;
     int32_t* status = (int32_t*)(ws + p.off_status);
-    if (p.path == kPathTc) {
+    if (p.path == kPathTc || p.path == kPathTcDecode) {
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
         void* xp = ws + p.off_xperm;
         if ((err = launch_gather_rows(x, perm, xp, p.R, c.hidden_size * 2, st)) != cudaSuccess)
@@ -432,14 +448,16 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
         f1.act = xp;
     }
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-    err = p.path == kPathSimt ? launch_ffn_simt(f1, st)
-          : p.path == kPathTc ? launch_ffn_tc(f1, p.bn, status, st)
-                              : launch_ffn_decode(f1, st);
+    err = p.path == kPathSimt        ? launch_ffn_simt(f1, st)
+          : p.path == kPathTc        ? launch_ffn_tc(f1, p.bn, status, st)
+          : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f1, p.bn, status, st)
+                                     : launch_ffn_decode(f1, st);
     if (err != cudaSuccess) return cuda_fail(h, err, "fc1");
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-    err = p.path == kPathSimt ? launch_ffn_simt(f2, st)
-          : p.path == kPathTc ? launch_ffn_tc(f2, p.bn, status, st)
-                              : launch_ffn_decode(f2, st);
+    err = p.path == kPathSimt        ? launch_ffn_simt(f2, st)
+          : p.path == kPathTc        ? launch_ffn_tc(f2, p.bn, status, st)
+          : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f2, p.bn, status, st)
+                                     : launch_ffn_decode(f2, st);
     if (err != cudaSuccess) return cuda_fail(h, err, "fc2");
     CombineArgs ca{};
     ca.o = o;

@@ -48,7 +48,7 @@ __host__ __device__ constexpr int64_t padded_rows(int64_t n) {
 }
 
 // Hot-path selection.
-enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2 };
+enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2, kPathTcDecode = 3 };
 
 struct Plan {
     int path = kPathDecode;
@@ -152,6 +152,11 @@ cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
 // device. launch_gather_rows copies the routed rows of x into segment order.
 cudaError_t prepare_ffn_tc();
 cudaError_t launch_ffn_tc(const FfnArgs& a, int bn, int32_t* status, cudaStream_t st);
+// Tensor-core streaming decode (few rows per expert; activations resident in
+// shared memory): tc_decode_fits says whether a K range split `splits` ways
+// fits its resident-activation buffer for token tile bn.
+bool tc_decode_fits(int64_t K, int splits, int bn);
+cudaError_t launch_ffn_tc_decode(const FfnArgs& a, int bn, int32_t* status, cudaStream_t st);
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm, void* xp, int64_t R, int64_t row_bytes,
                                cudaStream_t st);
 

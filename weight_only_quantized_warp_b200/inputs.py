@@ -168,6 +168,26 @@ def make_inputs(cfg: MoEConfig, seed: int, logits: str = "normal",
     return inp
 
 
+def make_token_batch(cfg: MoEConfig, seed: int, logits: str = "normal",
+                     logit_std: float = 1.0, **_unused):
+    """Draw only the per-token tensors ``(x, router_logits, shared)`` for
+    ``cfg`` from their own seeded generator, with the same distributions as
+    :func:`make_inputs` (``shared`` is None unless ``cfg.has_shared``)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    T, H, E = cfg.T, cfg.H, cfg.E
+    x = _store(rng.standard_normal((T, H)), cfg.act_dtype)
+    if logits == "normal":
+        lg = rng.standard_normal((T, E)) * logit_std
+    elif logits == "uniform":
+        lg = rng.uniform(0.0, 1.0, size=(T, E))
+    elif logits == "zipf":
+        lg = zipf_gumbel_logits(rng, T, E, 1.1)
+    else:
+        raise ValueError(logits)
+    shared = _store(rng.standard_normal((T, H)), cfg.act_dtype) if cfg.has_shared else None
+    return x, _store(lg, cfg.act_dtype), shared
+
+
 # ---------------------------------------------------------------------------
 # Named workloads. Each is (config, seed, generator keyword arguments).
 # ---------------------------------------------------------------------------

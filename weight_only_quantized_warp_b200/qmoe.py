@@ -28,7 +28,7 @@ QMOE_OK, QMOE_INVALID_ARGUMENT, QMOE_NOT_BOUND, QMOE_UNSUPPORTED = 0, 1, 2, 3
 QMOE_CUDA_ERROR, QMOE_TIMEOUT, QMOE_OUT_OF_MEMORY = 4, 5, 6
 ACT_RELU, ACT_GELU, ACT_SILU, ACT_SWIGLU, ACT_IDENTITY = 0, 1, 2, 3, 4
 DTYPE_F32, DTYPE_BF16 = 0, 1
-PATH_SIMT, PATH_DECODE, PATH_TC = 0, 1, 2
+PATH_SIMT, PATH_DECODE, PATH_TC, PATH_TC_DECODE = 0, 1, 2, 3
 
 # Every function the header declares (checked against include/qmoe.h by the tests).
 EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forward",
