@@ -229,6 +229,69 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, ui
         "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// Single-issuer instructions from a converged warp: the whole warp runs the
+// issuing loop (so its control flow and operands stay warp-uniform) and the
+// instruction itself is predicated on one elected lane, with no branch.
+__device__ __forceinline__ uint32_t elect_one() {
+    uint32_t e;
+    asm volatile("{\n.reg .pred p;\nelect.sync _|p, 0xffffffff;\nselp.b32 %0, 1, 0, p;\n}" : "=r"(e));
+    return e;
+}
+
+__device__ __forceinline__ void mma_bf16_ts_e(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred p, q;\nsetp.ne.b32 p, %4, 0;\nsetp.ne.b32 q, %5, 0;\n"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e));
+}
+
+__device__ __forceinline__ void mma_commit_e(uint32_t bar, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %1, 0;\n"
+        "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}" ::"r"(bar),
+        "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx_e(uint32_t bar, uint32_t bytes, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %2, 0;\n"
+        "@q mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n}" ::"r"(bar),
+        "r"(bytes), "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s_e(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                           uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %4, 0;\n"
+        "@q cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar), "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_3d_e(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                         uint32_t bar, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %6, 0;\n"
+        "@q cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3, %4}], [%5];\n}" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar), "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_2d_e(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar,
+                                         uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %5, 0;\n"
+        "@q cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3}], [%4];\n}" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar), "r"(e)
+        : "memory");
+}
+
 // --------------------------------------------------------------- arithmetic
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
     __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
@@ -387,7 +450,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == kWarpProd) {
         // ------------------------------------------------------- producer
-        if (lane == 0) {
+        {
+            const uint32_t e = elect_one();
             int st = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -397,30 +461,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int nbox = (it.rows + C::kBoxRows - 1) / C::kBoxRows;
                 const uint32_t bytes = uint32_t(C::kPacked + nbox * C::kBoxRows * 128) + sbytes;
                 for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
-                    if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                    if (!warp_wait(smem_u32(&empty[st]), ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
                     uint8_t* sb = smem + st * C::kStage;
                     const uint32_t fb = smem_u32(&full[st]);
-                    mbar_expect_tx(fb, bytes);
+                    mbar_expect_tx_e(fb, bytes, e);
                     const int g = ks * (kBK / kgroup_of(BITS));  // first k-group of the stage
                     const uint8_t* src =
                         a.W + ((int64_t(it.e) * nrb + it.rb) * ngr + g) * int64_t(kTilesPerBlock) * kUnitBytes;
-                    bulk_g2s(smem_u32(sb + C::kB), src, C::kPacked, fb);
+                    bulk_g2s_e(smem_u32(sb + C::kB), src, C::kPacked, fb, e);
                     if (!PERCOL) {
                         const int b0 = (ks * kBK) / a.block_size;
                         const int64_t sidx = ((int64_t(it.e) * nrb + it.rb) * nsb + b0) * kTilesPerBlock * 16;
                         const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(a.S) + sidx * ssz;
-                        bulk_g2s(smem_u32(sb + C::kB + C::kPacked), ssrc, sbytes, fb);
+                        bulk_g2s_e(smem_u32(sb + C::kB + C::kPacked), ssrc, sbytes, fb, e);
                     }
                     const int y0 = int(it.seg0) + it.tt * a.bn;
                     for (int b = 0; b < nbox; ++b)
-                        tma_2d(smem_u32(sb + b * C::kBoxRows * 128), &bmap, ks * kBK, y0 + b * C::kBoxRows, fb);
+                        tma_2d_e(smem_u32(sb + b * C::kBoxRows * 128), &bmap, ks * kBK, y0 + b * C::kBoxRows, fb, e);
                     if (++st == STAGES) { st = 0; ph ^= 1u; }
                 }
             }
         }
     } else if (warp == kWarpMma) {
         // ------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        {
+            const uint32_t e = elect_one();
             int st = 0, acc = 0;
             uint32_t ph = 0, aph = 0;
             bool ok = true;
@@ -428,24 +493,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const Item it = item_at(i, prefix, a, nrb, nks);
                 const int n = ((it.rows + 15) / 16) * 16;
                 const uint32_t idesc = idesc_bf16(n);
-                if (!mbar_wait(smem_u32(&acce[acc]), aph ^ 1u, abort_flag, a.status)) break;
+                if (!warp_wait(smem_u32(&acce[acc]), aph ^ 1u, abort_flag, a.status)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + uint32_t(acc * BNMAX);
                 for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
-                    if (!mbar_wait(smem_u32(&deq[st]), ph, abort_flag, a.status) ||
-                        !mbar_wait(smem_u32(&full[st]), ph, abort_flag, a.status)) { ok = false; break; }
+                    if (!warp_wait(smem_u32(&deq[st]), ph, abort_flag, a.status) ||
+                        !warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t at = tmem + uint32_t(C::kACol0 + st * kAStageCols);
                     const uint64_t bd = desc_sw128(smem_u32(smem + st * C::kStage));
+                    const uint32_t acc0 = ks > it.ks_lo ? 1u : 0u;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)  // 16 k per MMA: 8 A columns, 32 B of B
-                        mma_bf16_ts(d, at + uint32_t(8 * kk), bd + uint64_t(2 * kk), idesc,
-                                    (ks > it.ks_lo || kk > 0) ? 1u : 0u);
-                    mma_commit(smem_u32(&empty[st]));
+                        mma_bf16_ts_e(d, at + uint32_t(8 * kk), bd + uint64_t(2 * kk), idesc, kk > 0 ? 1u : acc0, e);
+                    mma_commit_e(smem_u32(&empty[st]), e);
                     if (++st == STAGES) { st = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
-                mma_commit(smem_u32(&accf[acc]));
+                mma_commit_e(smem_u32(&accf[acc]), e);
                 if (++acc == 2) { acc = 0; aph ^= 1u; }
             }
         }
@@ -747,58 +812,6 @@ __device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int
         : "memory");
 }
 
-// Single-issuer instructions from a converged warp: the whole warp runs the
-// issuing loop (so its control flow and operands stay warp-uniform) and the
-// instruction itself is predicated on one elected lane, with no branch.
-__device__ __forceinline__ uint32_t elect_one() {
-    uint32_t e;
-    asm volatile("{\n.reg .pred p;\nelect.sync _|p, 0xffffffff;\nselp.b32 %0, 1, 0, p;\n}" : "=r"(e));
-    return e;
-}
-
-__device__ __forceinline__ void mma_bf16_ts_e(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                              uint32_t accumulate, uint32_t e) {
-    asm volatile(
-        "{\n.reg .pred p, q;\nsetp.ne.b32 p, %4, 0;\nsetp.ne.b32 q, %5, 0;\n"
-        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e));
-}
-
-__device__ __forceinline__ void mma_commit_e(uint32_t bar, uint32_t e) {
-    asm volatile(
-        "{\n.reg .pred q;\nsetp.ne.b32 q, %1, 0;\n"
-        "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}" ::"r"(bar),
-        "r"(e)
-        : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx_e(uint32_t bar, uint32_t bytes, uint32_t e) {
-    asm volatile(
-        "{\n.reg .pred q;\nsetp.ne.b32 q, %2, 0;\n"
-        "@q mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n}" ::"r"(bar),
-        "r"(bytes), "r"(e)
-        : "memory");
-}
-
-__device__ __forceinline__ void bulk_g2s_e(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
-                                           uint32_t e) {
-    asm volatile(
-        "{\n.reg .pred q;\nsetp.ne.b32 q, %4, 0;\n"
-        "@q cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
-            dst),
-        "l"(src), "r"(bytes), "r"(bar), "r"(e)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_3d_e(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
-                                         uint32_t bar, uint32_t e) {
-    asm volatile(
-        "{\n.reg .pred q;\nsetp.ne.b32 q, %6, 0;\n"
-        "@q cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
-        "{%2, %3, %4}], [%5];\n}" ::"r"(dst),
-        "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar), "r"(e)
-        : "memory");
-}
 
 template <int BITS, bool PERCOL, int BN>
 __global__ void __launch_bounds__(kDThreads, 1)
