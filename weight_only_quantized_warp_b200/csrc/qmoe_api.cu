@@ -36,10 +36,10 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     const int tcd_bn = per_expert <= 16 ? 16 : 32;
     int tcd_s2 = 1;
     const int64_t max_s2 = std::max<int64_t>(1, I / 128);  // every split keeps >= one 128-k stage
-    while (tcd_s2 < max_s2 && (!tc_decode_fits(I, tcd_s2, tcd_bn) ||
+    while (tcd_s2 < max_s2 && (!tc_decode_fits(I, tcd_s2, tcd_bn, bs) ||
                                touched * (padded_rows(H) / kBlockRows) * tcd_s2 < 4 * kSms))
         ++tcd_s2;
-    const bool tcd_ok = per_expert <= 32 && tc_decode_fits(H, 1, tcd_bn) && tc_decode_fits(I, tcd_s2, tcd_bn);
+    const bool tcd_ok = per_expert <= 32 && tc_decode_fits(H, 1, tcd_bn, bs) && tc_decode_fits(I, tcd_s2, tcd_bn, bs);
     if (!bf16)
         p.path = kPathSimt;
     else if (h.path_override == kPathDecode || h.path_override == kPathTc)

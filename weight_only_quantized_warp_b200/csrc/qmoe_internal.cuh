@@ -154,8 +154,10 @@ cudaError_t prepare_ffn_tc();
 cudaError_t launch_ffn_tc(const FfnArgs& a, int bn, int32_t* status, cudaStream_t st);
 // Tensor-core streaming decode (few rows per expert; activations resident in
 // shared memory): tc_decode_fits says whether a K range split `splits` ways
-// fits its resident-activation buffer for token tile bn.
-bool tc_decode_fits(int64_t K, int splits, int bn);
+// fits its resident-activation buffer for token tile bn, and whether the
+// block size is one the kernel takes (0, 32, 64 or >= 128).
+cudaError_t prepare_ffn_tc_decode();
+bool tc_decode_fits(int64_t K, int splits, int bn, int block_size);
 cudaError_t launch_ffn_tc_decode(const FfnArgs& a, int bn, int32_t* status, cudaStream_t st);
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm, void* xp, int64_t R, int64_t row_bytes,
                                cudaStream_t st);

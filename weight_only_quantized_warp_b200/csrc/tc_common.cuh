@@ -1,0 +1,333 @@
+// tc_common.cuh -- pieces shared by the tcgen05 expert-FFN kernels (sm_100a):
+// kernel arguments, mbarrier / bulk-copy / TMA / tcgen05 PTX wrappers, bf16x2
+// arithmetic, activations, work-item record and the tensor-map encoder entry
+// point. Everything is internal to the including translation unit.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "qmoe_internal.cuh"
+
+namespace qmoe {
+namespace {
+
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+struct TcArgs {
+    const uint8_t* W;
+    const void* S;
+    const float* bias;       // FC1, packed row order, or nullptr
+    const int32_t* offsets;  // [E + 1]
+    void* out;               // FC1: h [R, I] bf16; FC2: partials [splits, R, N] fp32
+    int32_t* status;         // workspace status word
+    int64_t N, K, R;
+    int E, block_size, gated, is_fc1, act_type;
+    float alpha, beta, limit;
+    int splits, scale_bf16, bn;
+    int ring, stage_bytes, sring;  // streaming decode: packed-ring slots, scale-slot bytes, scale-ring slots
+};
+
+// ------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return uint32_t(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+// Potentially blocking test: a warp whose phase is still open is suspended
+// (it issues nothing) until the phase completes or kSuspendNs pass.
+constexpr uint32_t kSuspendNs = 10000;
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.b32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Non-blocking test of a phase (no suspension when the phase is still open).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.b32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on a phase parity. Returns false (after raising the CTA's
+// abort flag and the workspace status) when the wait gives up or another role
+// already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = now_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try(bar, parity)) return true;
+        if ((spin & 15u) == 0u) {
+            if (*abort_flag) return false;
+            if (now_ns() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                atomicExch(status, int32_t(QMOE_TIMEOUT));
+                return false;
+            }
+        }
+    }
+}
+
+// Wait by a whole warp: every lane polls, and the warp continues only if all
+// lanes saw the phase complete (a timeout in any lane stops the whole warp).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+    const bool ok = mbar_wait(bar, parity, abort_flag, status);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                       uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3}], [%4];" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
+// 1024 bytes stacked along M/N (stride 1024), version 1 for sm_100.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t(1) << 16;             // leading offset: unused for swizzled K-major
+    d |= uint64_t(1024 >> 4) << 32;     // stride offset between 8-row atoms
+    d |= uint64_t(1) << 46;             // descriptor version
+    d |= uint64_t(2) << 61;             // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: kind::f16, bf16 A and B (K-major), fp32 D, M = 128.
+__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st16x256_x4(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16x256_x2(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// MMA with A read from tensor memory (128 lanes = rows, 2 bf16 per column).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Single-issuer instructions from a converged warp: the whole warp runs the
+// issuing loop (so its control flow and operands stay warp-uniform) and the
+// instruction itself is predicated on one elected lane, with no branch.
+__device__ __forceinline__ uint32_t elect_one() {
+    uint32_t e;
+    asm volatile("{\n.reg .pred p;\nelect.sync _|p, 0xffffffff;\nselp.b32 %0, 1, 0, p;\n}" : "=r"(e));
+    return e;
+}
+
+__device__ __forceinline__ void mma_bf16_ts_e(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred p, q;\nsetp.ne.b32 p, %4, 0;\nsetp.ne.b32 q, %5, 0;\n"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e));
+}
+
+__device__ __forceinline__ void mma_commit_e(uint32_t bar, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %1, 0;\n"
+        "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}" ::"r"(bar),
+        "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx_e(uint32_t bar, uint32_t bytes, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %2, 0;\n"
+        "@q mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n}" ::"r"(bar),
+        "r"(bytes), "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s_e(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                           uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %4, 0;\n"
+        "@q cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar), "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_3d_e(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                         uint32_t bar, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %6, 0;\n"
+        "@q cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3, %4}], [%5];\n}" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar), "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_2d_e(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar,
+                                         uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred q;\nsetp.ne.b32 q, %5, 0;\n"
+        "@q cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3}], [%4];\n}" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar), "r"(e)
+        : "memory");
+}
+
+// --------------------------------------------------------------- arithmetic
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bf2_bcast(float s) {
+    __nv_bfloat162 r = __float2bfloat162_rn(s);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// fast sigmoid: the result is rounded to bf16 right after
+__device__ __forceinline__ float sigmoidf_(float v) { return __fdividef(1.0f, 1.0f + __expf(-v)); }
+__device__ __forceinline__ float act_plain(int t, float a) {
+    switch (t) {
+        case QMOE_ACT_RELU: return fmaxf(a, 0.0f);
+        case QMOE_ACT_GELU: return 0.5f * a * (1.0f + erff(a * 0.70710678118654752f));
+        case QMOE_ACT_SILU: return a * sigmoidf_(a);
+        default: return a;
+    }
+}
+__device__ __forceinline__ float act_gated(int t, float g, float u, float alpha, float beta,
+                                           float limit) {
+    if (t == QMOE_ACT_SWIGLU) {
+        g = fminf(g, limit);
+        u = fminf(fmaxf(u, -limit), limit);
+        return (u + beta) * g * sigmoidf_(alpha * g);
+    }
+    return act_plain(t, g) * u;
+}
+
+// ------------------------------------------------------------ work items
+struct Item {
+    int e, rb, tt, split;
+    int64_t seg0;
+    int M;      // rows routed to the expert
+    int rows;   // rows of this token tile
+    int ks_lo, ks_hi;
+};
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+}  // namespace qmoe
