@@ -12,16 +12,17 @@
 // dimension the routed tokens of one expert (a multiple of 16, up to 128), so
 // a small expert segment wastes no tensor work on padding rows.
 //
-// Warp roles of one persistent CTA (576 threads, one CTA per SM):
+// Warp roles of one persistent CTA (608 threads, one CTA per SM):
 //   warps 0-7   dequantise: packed codes (shared) -> bf16 A tile written
 //               straight into tensor memory (tcgen05.st), one 16-row tile per
 //               warp; the A operand never touches shared memory
-//   warp 8      producer: one bulk copy of the packed 128 x 64 tile (4 KB
-//               int4, 8 KB int8), one of its scales, and 64-row TMA boxes of
-//               the activations (bf16, 128-byte swizzle), as many as the tile
-//               has rows
+//   warp 8      activation producer: 64-row TMA boxes of the activations
+//               (bf16, 128-byte swizzle), as many as the tile has rows
+//   warp 18     weight producer: one bulk copy of the packed 128 x 64 tile
+//               (4 KB int4, 8 KB int8) and one of its scales
 //   warp 9      allocates TMEM and issues tcgen05.mma (A from TMEM, B from
-//               shared memory) from one thread
+//               shared memory); producers and MMA run their loops as whole
+//               warps and predicate each issue on one elected lane
 //   warps 10-17 epilogue: TMEM -> registers (tcgen05.ld), scale / bias /
 //               activation, global stores; two warps per TMEM lane quarter
 // Stages cycle through an S-deep ring guarded by mbarriers (full: copies
@@ -51,7 +52,8 @@ constexpr int kWarpProd = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpEpi0 = 10;
 constexpr int kEpiWarps = 8;
-constexpr int kTcThreads = (kWarpEpi0 + kEpiWarps) * 32;  // 576
+constexpr int kWarpProd2 = kWarpEpi0 + kEpiWarps;          // second producer (weights)
+constexpr int kTcThreads = (kWarpProd2 + 1) * 32;           // 608
 constexpr int kBK = 64;                                    // k per stage
 constexpr int kAStageCols = kBK / 2;                       // TMEM columns of one A tile
 constexpr int kScaleBytesMax = 4 * kTilesPerBlock * 16 * 4;  // 4 blocks of fp32 pairs
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&full[s]), 2);  // one arrival per producer warp
             mbar_init(smem_u32(&deq[s]), kDeqWarps);
             mbar_init(smem_u32(&empty[s]), 1);
         }
@@ -166,38 +168,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int sblk = PERCOL ? 0 : (a.block_size >= kBK ? 1 : kBK / a.block_size);
     const uint32_t sbytes = uint32_t(sblk * kTilesPerBlock * 16 * ssz);
 
-    if (warp == kWarpProd) {
-        // ------------------------------------------------------- producer
-        {
-            const uint32_t e = elect_one();
-            int st = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            const int ngr = int(a.K / kgroup_of(BITS));
-            for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
-                const Item it = item_at(i, prefix, a, nrb, nks);
-                const int nbox = (it.rows + C::kBoxRows - 1) / C::kBoxRows;
-                const uint32_t bytes = uint32_t(C::kPacked + nbox * C::kBoxRows * 128) + sbytes;
-                for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
-                    if (!warp_wait(smem_u32(&empty[st]), ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
-                    uint8_t* sb = smem + st * C::kStage;
-                    const uint32_t fb = smem_u32(&full[st]);
-                    mbar_expect_tx_e(fb, bytes, e);
-                    const int g = ks * (kBK / kgroup_of(BITS));  // first k-group of the stage
-                    const uint8_t* src =
-                        a.W + ((int64_t(it.e) * nrb + it.rb) * ngr + g) * int64_t(kTilesPerBlock) * kUnitBytes;
-                    bulk_g2s_e(smem_u32(sb + C::kB), src, C::kPacked, fb, e);
-                    if (!PERCOL) {
-                        const int b0 = (ks * kBK) / a.block_size;
-                        const int64_t sidx = ((int64_t(it.e) * nrb + it.rb) * nsb + b0) * kTilesPerBlock * 16;
-                        const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(a.S) + sidx * ssz;
-                        bulk_g2s_e(smem_u32(sb + C::kB + C::kPacked), ssrc, sbytes, fb, e);
-                    }
-                    const int y0 = int(it.seg0) + it.tt * a.bn;
+    if (warp == kWarpProd || warp == kWarpProd2) {
+        // ------------------------------------------------------- producers
+        // warp kWarpProd: the activation boxes; warp kWarpProd2: the packed
+        // codes and their scales. Each arrives once on the stage's full barrier
+        // with its own byte count, so the two issue streams run side by side.
+        const bool acts = warp == kWarpProd;
+        const uint32_t e = elect_one();
+        int st = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        const int ngr = int(a.K / kgroup_of(BITS));
+        const int bs_log2 = PERCOL ? 0 : __ffs(a.block_size) - 1;
+        for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+            const Item it = item_at(i, prefix, a, nrb, nks);
+            const int nbox = (it.rows + C::kBoxRows - 1) / C::kBoxRows;
+            const uint32_t bytes = acts ? uint32_t(nbox * C::kBoxRows * 128) : uint32_t(C::kPacked) + sbytes;
+            const int y0 = int(it.seg0) + it.tt * a.bn;
+            const int64_t blk = int64_t(it.e) * nrb + it.rb;
+            for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
+                if (!warp_wait(smem_u32(&empty[st]), ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                uint8_t* sb = smem + st * C::kStage;
+                const uint32_t fb = smem_u32(&full[st]);
+                mbar_expect_tx_e(fb, bytes, e);
+                if (acts) {
                     for (int b = 0; b < nbox; ++b)
                         tma_2d_e(smem_u32(sb + b * C::kBoxRows * 128), &bmap, ks * kBK, y0 + b * C::kBoxRows, fb, e);
-                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                } else {
+                    const int g = ks * (kBK / kgroup_of(BITS));  // first k-group of the stage
+                    const uint8_t* src = a.W + (blk * ngr + g) * int64_t(kTilesPerBlock) * kUnitBytes;
+                    bulk_g2s_e(smem_u32(sb + C::kB), src, C::kPacked, fb, e);
+                    if (!PERCOL) {
+                        const int b0 = (ks * kBK) >> bs_log2;
+                        const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(a.S) +
+                                              (blk * nsb + b0) * int64_t(kTilesPerBlock * 16 * ssz);
+                        bulk_g2s_e(smem_u32(sb + C::kB + C::kPacked), ssrc, sbytes, fb, e);
+                    }
                 }
+                if (++st == STAGES) { st = 0; ph ^= 1u; }
             }
         }
     } else if (warp == kWarpMma) {
@@ -320,7 +328,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (++st == STAGES) { st = 0; ph ^= 1u; }
             }
         }
-    } else if (warp >= kWarpEpi0) {
+    } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + kEpiWarps) {
         // ------------------------------------------------------- epilogue
         const int qd = warp & 3;                        // TMEM lane quarter this warp may read
         const int half = (warp - kWarpEpi0) >> 2;       // which 16-column chunks it takes
