@@ -71,6 +71,11 @@ CASES = {
                                act=gen.ACT_SILU),
     "k128_int8_percol_relu": dict(H=256, I=384, bits=8, block_size=0, fusion=0, act=gen.ACT_RELU),
     "k128_t32_tile32": dict(H=256, I=384, T=96, E=8, k=2),
+    # more than 128 rows per expert: 256-wide token tiles on the tensor-core path
+    "wide_tile_int4_bs32_bias": dict(T=300, E=2, k=1, H=256, I=384, block_size=32, fusion=1, alpha=1.702,
+                                     beta=1.0, limit=7.0, has_fc1_bias=True, has_fc2_bias=True),
+    "wide_tile_int8_percol_fc3_shared": dict(T=520, E=4, k=2, H=256, I=384, bits=8, block_size=0, fusion=0,
+                                             has_fc3=True, act=gen.ACT_SILU, normalize=False, has_shared=True),
     "fp32_acts_int8": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, bits=8, block_size=32,
                            has_fc1_bias=True, has_fc2_bias=True, has_shared=True),
     "fp32_acts_percol_fc3": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_BF16, block_size=0,

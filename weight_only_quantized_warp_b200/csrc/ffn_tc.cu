@@ -57,30 +57,6 @@ constexpr int kTcThreads = (kWarpProd2 + 1) * 32;           // 608
 constexpr int kBK = 64;                                    // k per stage
 constexpr int kAStageCols = kBK / 2;                       // TMEM columns of one A tile
 constexpr int kScaleBytesMax = 4 * kTilesPerBlock * 16 * 4;  // 4 blocks of fp32 pairs
-// Items are ordered expert, row block, token tile, split, so CTAs working on
-// neighbouring items share weight blocks in L2.
-__device__ __forceinline__ Item item_at(int i, const int* prefix, const TcArgs& a, int nrb, int nks) {
-    int lo = 0, hi = a.E;  // largest e with prefix[e] <= i
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (prefix[mid] <= i) lo = mid; else hi = mid;
-    }
-    Item it;
-    it.e = lo;
-    it.seg0 = a.offsets[lo];
-    it.M = a.offsets[lo + 1] - int(it.seg0);
-    const int ntt = (it.M + a.bn - 1) / a.bn;
-    int rem = i - prefix[lo];
-    const int per_rb = ntt * a.splits;
-    it.rb = rem / per_rb;
-    rem -= it.rb * per_rb;
-    it.tt = rem / a.splits;
-    it.split = rem - it.tt * a.splits;
-    it.rows = min(a.bn, it.M - it.tt * a.bn);
-    it.ks_lo = int((int64_t(it.split) * nks) / a.splits);
-    it.ks_hi = int((int64_t(it.split + 1) * nks) / a.splits);
-    return it;
-}
 
 template <int BITS, bool PERCOL, int BNMAX, int STAGES>
 struct TcCfg {
@@ -339,61 +315,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const Item it = item_at(i, prefix, a, nrb, nks);
             if (!warp_wait(smem_u32(&accf[acc]), aph, abort_flag, a.status)) break;
             tc_fence_after();
-            const int64_t prow = int64_t(it.rb) * kBlockRows + row;  // packed row in the expert
-            const bool valid = prow < a.N;
-            float s = 1.0f;
-            if (PERCOL && valid) {
-                const int tl = row >> 4, rr = row & 15;
-                const int64_t si = ((int64_t(it.e) * nrb + it.rb) * kTilesPerBlock + tl) * 16 + (rr & 7) * 2 + (rr >> 3);
-                s = a.scale_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.S)[si])
-                                 : reinterpret_cast<const float*>(a.S)[si];
-            }
-            const float bias = (a.bias && valid) ? a.bias[int64_t(it.e) * a.N + prow] : 0.0f;
-            const uint32_t tbase = tmem + (uint32_t(qd * 32) << 16) + uint32_t(acc * BNMAX);
-            const int ncol = ((it.rows + 15) / 16) * 16;
-            const bool empty_k = it.ks_hi <= it.ks_lo;  // no MMA wrote the accumulator
-            const int64_t p0 = it.seg0 + int64_t(it.tt) * a.bn;  // permuted row of column 0
-            if (a.is_fc1 && a.gated) {
-                // tile rows 0-7 are gate rows, 8-15 the matching up rows (lane ^ 8):
-                // each lane of a pair finishes half of every 16 columns, so all
-                // lanes compute activations
-                const bool gate_lane = (lane & 8) == 0;
-                const int64_t I = a.N / 2;
-                __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(a.out) + p0 * I + (prow >> 4) * 8 + (row & 7);
-                for (int c0 = 16 * half; c0 < ncol; c0 += 32) {
-                    float v[16];
-                    tmem_ld16(tbase + uint32_t(c0), v);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = empty_k ? 0.0f : fmaf(v[j], s, bias);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float recv = __shfl_xor_sync(0xffffffffu, gate_lane ? v[j + 8] : v[j], 8);
-                        const float g = gate_lane ? v[j] : recv;
-                        const float u = gate_lane ? recv : v[j + 8];
-                        const int col = c0 + j + (gate_lane ? 0 : 8);
-                        if (col < it.rows && valid)
-                            hout[int64_t(col) * I] =
-                                __float2bfloat16_rn(act_gated(a.act_type, g, u, a.alpha, a.beta, a.limit));
-                    }
-                }
-            } else {
-                for (int c0 = 16 * half; c0 < ncol; c0 += 32) {
-                    float v[16];
-                    tmem_ld16(tbase + uint32_t(c0), v);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int col = c0 + j;
-                        const float val = empty_k ? 0.0f : fmaf(v[j], s, bias);
-                        if (col >= it.rows || !valid) continue;
-                        const int64_t p = p0 + col;  // permuted row
-                        if (a.is_fc1)
-                            reinterpret_cast<__nv_bfloat16*>(a.out)[p * a.N + prow] =
-                                __float2bfloat16_rn(act_plain(a.act_type, val));
-                        else
-                            reinterpret_cast<float*>(a.out)[(int64_t(it.split) * a.R + p) * a.N + prow] = val;
-                    }
-                }
-            }
+            tc_epilogue_item<PERCOL>(a, it, nrb, tmem + (uint32_t(qd * 32) << 16) + uint32_t(acc * BNMAX), row,
+                                     lane, 16 * half, 32);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&acce[acc]));
@@ -466,6 +389,7 @@ cudaError_t prepare_ffn_tc() {
     if (e == cudaSuccess) e = prepare_bits<8, false>();
     if (e == cudaSuccess) e = prepare_bits<8, true>();
     if (e == cudaSuccess) e = prepare_ffn_tc_decode();
+    if (e == cudaSuccess) e = prepare_ffn_tc_wide();
     return e;
 }
 
@@ -485,7 +409,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& f, int bn, int32_t* status, cudaStream_
     if (!enc) return cudaErrorNotSupported;
     int bnmax = 16;
     while (bnmax < bn) bnmax *= 2;
-    if (bnmax > 128) return cudaErrorInvalidValue;
+    if (bnmax > 128) return launch_ffn_tc_wide(f, bn, status, st);
     // activations: [rows, K] bf16; rows = R (permuted rows)
     const int64_t rows = f.R;
     CUtensorMap map;

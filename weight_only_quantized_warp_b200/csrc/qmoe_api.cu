@@ -70,7 +70,7 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
                decode_smem_bytes(I, bits, bs, p.fc2_splits, p.nt) <= int64_t(kDecodeSmemLimit);
     } else if (p.path == kPathTc) {
         int bn = 16;
-        while (bn < 128 && bn < per_expert) bn *= 2;
+        while (bn < 256 && bn < per_expert) bn *= 2;
         p.bn = bn;
         // FC2 work items: touched experts x 128-row blocks x token tiles;
         // split K until every SM has about two items

@@ -152,6 +152,9 @@ cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
 // device. launch_gather_rows copies the routed rows of x into segment order.
 cudaError_t prepare_ffn_tc();
 cudaError_t launch_ffn_tc(const FfnArgs& a, int bn, int32_t* status, cudaStream_t st);
+// Token tiles wider than 128 (up to 256): A tile in shared memory, N = 256 MMAs.
+cudaError_t prepare_ffn_tc_wide();
+cudaError_t launch_ffn_tc_wide(const FfnArgs& a, int bn, int32_t* status, cudaStream_t st);
 // Tensor-core streaming decode (few rows per expert; activations resident in
 // shared memory): tc_decode_fits says whether a K range split `splits` ways
 // fits its resident-activation buffer for token tile bn, and whether the

@@ -220,6 +220,14 @@ __device__ __forceinline__ void mma_bf16_ts_e(uint32_t tmem_d, uint32_t tmem_a, 
         "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e));
 }
 
+__device__ __forceinline__ void mma_bf16_ss_e(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate, uint32_t e) {
+    asm volatile(
+        "{\n.reg .pred p, q;\nsetp.ne.b32 p, %4, 0;\nsetp.ne.b32 q, %5, 0;\n"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e));
+}
+
 __device__ __forceinline__ void mma_commit_e(uint32_t bar, uint32_t e) {
     asm volatile(
         "{\n.reg .pred q;\nsetp.ne.b32 q, %1, 0;\n"
@@ -310,6 +318,95 @@ struct Item {
     int rows;   // rows of this token tile
     int ks_lo, ks_hi;
 };
+
+// Items are ordered expert, row block, token tile, split, so CTAs working on
+// neighbouring items share weight blocks in L2.
+__device__ __forceinline__ Item item_at(int i, const int* prefix, const TcArgs& a, int nrb, int nks) {
+    int lo = 0, hi = a.E;  // largest e with prefix[e] <= i
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= i) lo = mid; else hi = mid;
+    }
+    Item it;
+    it.e = lo;
+    it.seg0 = a.offsets[lo];
+    it.M = a.offsets[lo + 1] - int(it.seg0);
+    const int ntt = (it.M + a.bn - 1) / a.bn;
+    int rem = i - prefix[lo];
+    const int per_rb = ntt * a.splits;
+    it.rb = rem / per_rb;
+    rem -= it.rb * per_rb;
+    it.tt = rem / a.splits;
+    it.split = rem - it.tt * a.splits;
+    it.rows = min(a.bn, it.M - it.tt * a.bn);
+    it.ks_lo = int((int64_t(it.split) * nks) / a.splits);
+    it.ks_hi = int((int64_t(it.split + 1) * nks) / a.splits);
+    return it;
+}
+
+// Epilogue of one work item for the thread that owns accumulator lane `row`
+// (packed row rb*128 + row of the item's expert): columns c_first,
+// c_first + c_step, ... in chunks of 16 from the accumulator at TMEM address
+// tbase; scale (per-column mode), bias, activation and the store of h (FC1)
+// or of the split's fp32 partial (FC2).
+template <bool PERCOL>
+__device__ __forceinline__ void tc_epilogue_item(const TcArgs& a, const Item& it, int nrb, uint32_t tbase, int row,
+                                                 int lane, int c_first, int c_step) {
+    const int64_t prow = int64_t(it.rb) * kBlockRows + row;  // packed row in the expert
+    const bool valid = prow < a.N;
+    float s = 1.0f;
+    if (PERCOL && valid) {
+        const int tl = row >> 4, rr = row & 15;
+        const int64_t si = ((int64_t(it.e) * nrb + it.rb) * kTilesPerBlock + tl) * 16 + (rr & 7) * 2 + (rr >> 3);
+        s = a.scale_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.S)[si])
+                         : reinterpret_cast<const float*>(a.S)[si];
+    }
+    const float bias = (a.bias && valid) ? a.bias[int64_t(it.e) * a.N + prow] : 0.0f;
+    const int ncol = ((it.rows + 15) / 16) * 16;
+    const bool empty_k = it.ks_hi <= it.ks_lo;  // no MMA wrote the accumulator
+    const int64_t p0 = it.seg0 + int64_t(it.tt) * a.bn;  // permuted row of column 0
+    if (a.is_fc1 && a.gated) {
+        // tile rows 0-7 are gate rows, 8-15 the matching up rows (lane ^ 8):
+        // each lane of a pair finishes half of every 16 columns, so all
+        // lanes compute activations
+        const bool gate_lane = (lane & 8) == 0;
+        const int64_t I = a.N / 2;
+        __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(a.out) + p0 * I + (prow >> 4) * 8 + (row & 7);
+        for (int c0 = c_first; c0 < ncol; c0 += c_step) {
+            float v[16];
+            tmem_ld16(tbase + uint32_t(c0), v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = empty_k ? 0.0f : fmaf(v[j], s, bias);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float recv = __shfl_xor_sync(0xffffffffu, gate_lane ? v[j + 8] : v[j], 8);
+                const float g = gate_lane ? v[j] : recv;
+                const float u = gate_lane ? recv : v[j + 8];
+                const int col = c0 + j + (gate_lane ? 0 : 8);
+                if (col < it.rows && valid)
+                    hout[int64_t(col) * I] =
+                        __float2bfloat16_rn(act_gated(a.act_type, g, u, a.alpha, a.beta, a.limit));
+            }
+        }
+    } else {
+        for (int c0 = c_first; c0 < ncol; c0 += c_step) {
+            float v[16];
+            tmem_ld16(tbase + uint32_t(c0), v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int col = c0 + j;
+                const float val = empty_k ? 0.0f : fmaf(v[j], s, bias);
+                if (col >= it.rows || !valid) continue;
+                const int64_t p = p0 + col;  // permuted row
+                if (a.is_fc1)
+                    reinterpret_cast<__nv_bfloat16*>(a.out)[p * a.N + prow] =
+                        __float2bfloat16_rn(act_plain(a.act_type, val));
+                else
+                    reinterpret_cast<float*>(a.out)[(int64_t(it.split) * a.R + p) * a.N + prow] = val;
+            }
+        }
+    }
+}
 
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
