@@ -69,8 +69,11 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         p.ok = decode_smem_bytes(H, bits, bs, 1, p.nt) <= int64_t(kDecodeSmemLimit) &&
                decode_smem_bytes(I, bits, bs, p.fc2_splits, p.nt) <= int64_t(kDecodeSmemLimit);
     } else if (p.path == kPathTc) {
+        // token tile: the power of two covering the average segment with a
+        // third to spare, so that most experts take one tile (the weights of
+        // an expert are decoded once per tile)
         int bn = 16;
-        while (bn < 256 && bn < per_expert) bn *= 2;
+        while (bn < 256 && bn < ceil_div(4 * per_expert, 3)) bn *= 2;
         p.bn = bn;
         // FC2 work items: touched experts x 128-row blocks x token tiles;
         // split K until every SM has about two items
