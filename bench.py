@@ -155,10 +155,16 @@ def traffic_record(kernel_key):
         d = json.load(f).get(kernel_key)
     if not d:
         return None
-    src = os.path.join(ROOT, "weight_only_quantized_warp_b200", "csrc", d["source"])
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()[:16]
-    return d if digest == d.get("sha256_16") else None
+    return d if source_digest(d["source"]) == d.get("sha256_16") else None
+
+
+def source_digest(sources):
+    """First 16 hex digits of the sha256 over the named csrc files, in order."""
+    h = hashlib.sha256()
+    for name in ([sources] if isinstance(sources, str) else sources):
+        with open(os.path.join(ROOT, "weight_only_quantized_warp_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------- reference arm
@@ -295,8 +301,10 @@ def run_ours(args):
     per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(launches)]
                            for i in range(K)]).mean(axis=0)
     path = qmoe.qmoe_path_for(h, T)
-    names = (["route", "permute", "gather", "fc1", "fc2", "combine"] if path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE)
-             else ["route", "permute", "fc1", "fc2", "combine"])[:launches]
+    tc_path = path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE)
+    fused = launches == (5 if tc_path else 4)  # routing and permutation in one launch
+    names = ((["route_permute"] if fused else ["route", "permute"]) + (["gather"] if tc_path else [])
+             + ["fc1", "fc2", "combine"])
 
     # ---- end to end through the public call, host buffers, copies inside
     x_h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu())
@@ -357,10 +365,11 @@ def run_ours(args):
     fc1_flops = 2.0 * cfg.T * cfg.k * (cfg.n1 + (cfg.I if cfg.has_fc3 else 0)) * cfg.H
     t_hbm = alg["fc1_bytes"] / (hbm_peak * 1e9)
     t_tc = fc1_flops / (tc_peak * 1e12)
-    kname = {qmoe.PATH_TC: "ffn_tc_kernel (FC1 + SwiGLU)",
-             qmoe.PATH_TC_DECODE: "ffn_tc_decode_kernel (FC1 + SwiGLU)"}.get(path, "ffn_decode_kernel (FC1 + SwiGLU)")
-    tr = traffic_record({qmoe.PATH_TC: "fc1_tc_", qmoe.PATH_TC_DECODE: "fc1_tcdecode_"}.get(path, "fc1_decode_")
-                        + args.workload)
+    tile = qmoe.qmoe_token_tile_for(h, T)
+    kbase = ("ffn_tc_wide_kernel" if tile > 128 else "ffn_tc_kernel") if path == qmoe.PATH_TC else \
+        {qmoe.PATH_TC_DECODE: "ffn_tc_decode_kernel", qmoe.PATH_SIMT: "ffn_simt_kernel"}.get(path, "ffn_decode_kernel")
+    kname = kbase + " (FC1 + activation)"
+    tr = traffic_record("fc1_" + kbase + "_" + args.workload)
     if t_hbm >= t_tc:
         achieved = alg["fc1_bytes"] / (fc1_ms / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -383,7 +392,7 @@ def run_ours(args):
             "step": {"hbm_gbs": whole, "tflops": alg["flops"] / (step_ms / 1e3) / 1e12,
                      "hbm_frac": whole / hbm_peak, "experts_touched": alg["touched"],
                      "algorithmic_bytes": alg["total_bytes"],
-                     "kernel_ms": kms, "path": path},
+                     "kernel_ms": kms, "path": path, "token_tile": tile},
             "cpu_baseline": cpu,
             "e2e": {"value": replicas.job_tokens_per_s(T, world, K, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

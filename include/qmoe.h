@@ -269,8 +269,17 @@ QMOE_API qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t val
  * 3 = tcgen05 streaming decode. -1 for a NULL handle. */
 QMOE_API int32_t qmoe_path_for(const qmoe_handle* h, int64_t T);
 
-/* Number of kernel launches qmoe_forward enqueues for T tokens. */
+/* Number of kernel launches qmoe_forward enqueues for T tokens: routing and
+ * permutation (one launch for T <= 64, two above), the row gather (tensor-core
+ * paths), FC1, FC2 and the combine. 0 for T = 0. */
 QMOE_API int32_t qmoe_launches_for(const qmoe_handle* h, int64_t T);
+
+/* Token-tile width (the MMA N dimension, rows of one expert per work item)
+ * of the tensor-core paths for T tokens: 16..128 run the 128-wide tcgen05
+ * kernel with the decoded weights in TMEM, 256 the wide kernel with them in
+ * shared memory; 16 or 32 on path 3. 0 on paths 0 and 1, -1 for a NULL
+ * handle or T < 0. No counterpart on the pages: it only reports the plan. */
+QMOE_API int32_t qmoe_token_tile_for(const qmoe_handle* h, int64_t T);
 
 #ifdef __cplusplus
 }

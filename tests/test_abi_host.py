@@ -84,14 +84,30 @@ def test_create_accepts_and_plans_without_gpu(q):
         assert ws8 > q.qmoe_workspace_size(h, 1) and ws8 % 256 == 0
         assert q.qmoe_workspace_size(h, -1) == 0
         assert q.qmoe_path_for(h, 8) == q.PATH_DECODE
-        assert q.qmoe_launches_for(h, 8) == 5
+        assert q.qmoe_launches_for(h, 8) == 4     # route+permute, FC1, FC2, combine
+        assert q.qmoe_launches_for(h, 64) == 4
+        assert q.qmoe_launches_for(h, 65) == 6    # tensor-core path: route, permute, gather, ...
         assert q.qmoe_launches_for(h, 0) == 0
+        assert q.qmoe_token_tile_for(h, 8) == 0  # decode path: no token tile
+        assert q.qmoe_token_tile_for(h, -1) == -1
     finally:
         q.qmoe_destroy(h)
     hf = q.qmoe_create(_cfg(q, act_dtype=q.DTYPE_F32, scale_dtype=q.DTYPE_F32))
     assert q.qmoe_path_for(hf, 8) == q.PATH_SIMT
     q.qmoe_destroy(hf)
     q.qmoe_destroy(None)  # no-op
+
+
+@pytest.mark.parametrize("T,path,tile", [(8, 1, 0), (96, 2, 32), (384, 2, 128), (2048, 2, 256)])
+def test_plan_token_tile_covers_the_average_segment(q, T, path, tile):
+    # 8 experts, k = 2: T*2/8 rows per expert on average; the tile is the
+    # power of two covering 4/3 of that, at most 256
+    h = q.qmoe_create(_cfg(q))
+    try:
+        assert q.qmoe_path_for(h, T) == path
+        assert q.qmoe_token_tile_for(h, T) == tile
+    finally:
+        q.qmoe_destroy(h)
 
 
 def test_forward_before_set_weights_is_not_bound(q):

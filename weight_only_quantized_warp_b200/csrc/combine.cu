@@ -12,19 +12,28 @@
 namespace qmoe {
 namespace {
 
-__global__ void combine_kernel(const CombineArgs a) {
-    const int64_t hq = a.H / 4;
-    const int64_t total = a.T * hq;
-    for (int64_t id = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; id < total;
-         id += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = id / hq, m = (id % hq) * 4;
+constexpr int kCombineThreads = 256;
+constexpr int kCombineChunk = kCombineThreads * 4;  // elements of one row per block
+
+// One block per (token, 1024-element chunk of its row); each thread owns four
+// consecutive elements. The token's k routes are read once per block; the
+// loads of all k rows and splits are independent, so they are in flight
+// together.
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineArgs a) {
+    const float* __restrict__ o = a.o;
+    const int nchunk = int((a.H + kCombineChunk - 1) / kCombineChunk);
+    const int64_t nblk = a.T * nchunk;
+    for (int64_t b = blockIdx.x; b < nblk; b += gridDim.x) {
+        const int64_t t = b / nchunk;
+        const int64_t m = (b - t * nchunk) * kCombineChunk + 4 * threadIdx.x;
+        if (m >= a.H) continue;
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int j = 0; j < a.k; ++j) {
             const int64_t pos = a.inv[t * a.k + j];
             const float w = a.topk_w[t * a.k + j];
             float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             for (int s = 0; s < a.splits; ++s) {
-                const float4 p = *reinterpret_cast<const float4*>(a.o + ((int64_t)s * a.R + pos) * a.H + m);
+                const float4 p = __ldcs(reinterpret_cast<const float4*>(o + ((int64_t)s * a.R + pos) * a.H + m));
                 v[0] += p.x;
                 v[1] += p.y;
                 v[2] += p.z;
@@ -32,20 +41,22 @@ __global__ void combine_kernel(const CombineArgs a) {
             }
             if (a.b2) {
                 const int64_t e = a.topk_idx[t * a.k + j];
-                const float4 b = *reinterpret_cast<const float4*>(a.b2 + e * a.H + m);
-                v[0] += b.x;
-                v[1] += b.y;
-                v[2] += b.z;
-                v[3] += b.w;
+                const float4 bb = *reinterpret_cast<const float4*>(a.b2 + e * a.H + m);
+                v[0] += bb.x;
+                v[1] += bb.y;
+                v[2] += bb.z;
+                v[3] += bb.w;
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[q] = fmaf(w, v[q], acc[q]);
         }
         if (a.act_bf16) {
             if (a.shared) {
-                const __nv_bfloat16* s = (const __nv_bfloat16*)a.shared + t * a.H + m;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc[q] += __bfloat162float(s[q]);
+                const uint2 sv = *reinterpret_cast<const uint2*>((const __nv_bfloat16*)a.shared + t * a.H + m);
+                acc[0] += __uint_as_float(sv.x << 16);
+                acc[1] += __uint_as_float(sv.x & 0xFFFF0000u);
+                acc[2] += __uint_as_float(sv.y << 16);
+                acc[3] += __uint_as_float(sv.y & 0xFFFF0000u);
             }
             __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
             __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
@@ -55,14 +66,13 @@ __global__ void combine_kernel(const CombineArgs a) {
             *reinterpret_cast<uint2*>((__nv_bfloat16*)a.y + t * a.H + m) = out;
         } else {
             if (a.shared) {
-                const float4 s = *reinterpret_cast<const float4*>((const float*)a.shared + t * a.H + m);
-                acc[0] += s.x;
-                acc[1] += s.y;
-                acc[2] += s.z;
-                acc[3] += s.w;
+                const float4 sv = *reinterpret_cast<const float4*>((const float*)a.shared + t * a.H + m);
+                acc[0] += sv.x;
+                acc[1] += sv.y;
+                acc[2] += sv.z;
+                acc[3] += sv.w;
             }
-            *reinterpret_cast<float4*>((float*)a.y + t * a.H + m) =
-                make_float4(acc[0], acc[1], acc[2], acc[3]);
+            *reinterpret_cast<float4*>((float*)a.y + t * a.H + m) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         }
     }
 }
@@ -70,11 +80,10 @@ __global__ void combine_kernel(const CombineArgs a) {
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
-    const int threads = 256;
-    int64_t blocks = (a.T * (a.H / 4) + threads - 1) / threads;
+    if (a.T == 0) return cudaSuccess;
+    int64_t blocks = a.T * ((a.H + kCombineChunk - 1) / kCombineChunk);
     if (blocks > 148 * 16) blocks = 148 * 16;
-    if (blocks < 1) blocks = 1;
-    combine_kernel<<<unsigned(blocks), threads, 0, st>>>(a);
+    combine_kernel<<<unsigned(blocks), kCombineThreads, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -82,7 +82,8 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         while (items * s < 2 * kSms && s < 8 && s * 2 <= I / 64) s *= 2;
         p.fc2_splits = int(s);
     }
-    p.launches = (p.path == kPathTc || p.path == kPathTcDecode) ? 6 : 5;
+    p.fused_route = T <= kFusedRouteTokens;
+    p.launches = ((p.path == kPathTc || p.path == kPathTcDecode) ? 6 : 5) - (p.fused_route ? 1 : 0);
     const size_t R = size_t(p.R);
     const size_t act = bf16 ? 2 : 4;
     size_t off = 0;
@@ -350,6 +351,12 @@ int32_t qmoe_launches_for(const qmoe_handle* h, int64_t T) {
     return T == 0 ? 0 : make_plan(*h, T).launches;
 }
 
+int32_t qmoe_token_tile_for(const qmoe_handle* h, int64_t T) {
+    if (!h || T < 0) return -1;
+    const Plan p = make_plan(*h, T);
+    return (p.path == kPathTc || p.path == kPathTcDecode) ? p.bn : 0;
+}
+
 }  // extern "C"
 
 static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
@@ -396,15 +403,20 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     const int E = int(c.num_experts), k = int(c.k);
     const int bf16 = c.act_dtype == QMOE_DTYPE_BF16;
     cudaError_t err;
-    if ((err = cudaMemsetAsync(ws + p.off_status, 0, 16, st)) != cudaSuccess)
-        return cuda_fail(h, err, "status reset");
+    int32_t* status = (int32_t*)(ws + p.off_status);  // cleared by the first kernel
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-    if ((err = launch_route(router_logits, bf16, T, E, k, c.normalize_routing_weights, idx, tw, st)) !=
-        cudaSuccess)
-        return cuda_fail(h, err, "route");
-    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-    if ((err = launch_permute(idx, T, E, k, offsets, perm, inv, st)) != cudaSuccess)
-        return cuda_fail(h, err, "permute");
+    if (p.fused_route) {
+        if ((err = launch_route_permute(router_logits, bf16, T, E, k, c.normalize_routing_weights, idx, tw,
+                                        offsets, perm, inv, status, st)) != cudaSuccess)
+            return cuda_fail(h, err, "route+permute");
+    } else {
+        if ((err = launch_route(router_logits, bf16, T, E, k, c.normalize_routing_weights, idx, tw, status,
+                                st)) != cudaSuccess)
+            return cuda_fail(h, err, "route");
+        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+        if ((err = launch_permute(idx, T, E, k, offsets, perm, inv, st)) != cudaSuccess)
+            return cuda_fail(h, err, "permute");
+    }
 
     FfnArgs f1{};
     f1.W = h->w1;
@@ -442,7 +454,6 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     f2.gated = 0;
     f2.is_fc1 = 0;
     f2.splits = p.fc2_splits;
-    int32_t* status = (int32_t*)(ws + p.off_status);
     if (p.path == kPathTc || p.path == kPathTcDecode) {
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
         void* xp = ws + p.off_xperm;

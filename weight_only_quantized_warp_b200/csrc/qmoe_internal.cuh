@@ -58,6 +58,7 @@ struct Plan {
     int launches = 0;
     bool ok = true;      // a kernel configuration exists for this shape
     int bn = 0;          // token tile of the tensor-core path
+    bool fused_route = false;  // routing and permutation in one launch (few tokens)
     size_t off_idx = 0, off_w = 0, off_inv = 0, off_perm = 0, off_offsets = 0, off_status = 0,
            off_h = 0, off_o = 0, off_xperm = 0, total = 0;
 };
@@ -110,7 +111,12 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t st);
 
 // Top-k softmax routing: warp per token.
 cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
-                         int32_t* topk_idx, float* topk_w, cudaStream_t st);
+                         int32_t* topk_idx, float* topk_w, int32_t* status, cudaStream_t st);
+// Routing and permutation of at most kFusedRouteTokens tokens in one launch.
+constexpr int64_t kFusedRouteTokens = 64;
+cudaError_t launch_route_permute(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
+                                 int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm_tok,
+                                 int32_t* inv, int32_t* status, cudaStream_t st);
 
 // Histogram, scan and stable scatter into per-expert segments (one CTA).
 // prepare_route_permute() raises the permute kernel's shared-memory limit on

@@ -25,13 +25,10 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
     return v > bv || (v == bv && e < be);
 }
 
-// One warp per token.
-__global__ void route_kernel(const void* logits, int act_bf16, int64_t T, int E, int k,
-                             int normalize, int32_t* __restrict__ topk_idx,
-                             float* __restrict__ topk_w) {
-    const int lane = threadIdx.x & 31;
-    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    if (t >= T) return;
+// Route token t with one warp (lane = this thread's lane).
+__device__ __forceinline__ void route_token(const void* logits, int act_bf16, int64_t t, int E, int k,
+                                            int normalize, int32_t* __restrict__ topk_idx,
+                                            float* __restrict__ topk_w, int lane) {
     float v[kMaxPerLane];
     const int per = (E + 31) >> 5;
 #pragma unroll
@@ -95,16 +92,26 @@ __global__ void route_kernel(const void* logits, int act_bf16, int64_t T, int E,
     }
 }
 
+// One warp per token. Thread 0 also clears the workspace status word, which
+// no kernel of the forward has written yet.
+__global__ void route_kernel(const void* logits, int act_bf16, int64_t T, int E, int k,
+                             int normalize, int32_t* __restrict__ topk_idx,
+                             float* __restrict__ topk_w, int32_t* __restrict__ status) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    route_token(logits, act_bf16, t, E, k, normalize, topk_idx, topk_w, threadIdx.x & 31);
+}
+
 // One CTA of 1024 threads. Token chunks of 1024: for each chunk, warp-level
 // bit masks per expert give each (token, expert) pair its rank among the
 // chunk's earlier tokens; a running per-expert base carries across chunks.
 constexpr int kPermThreads = 1024;
 constexpr int kWarps = kPermThreads / 32;
 
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(
-    const int32_t* __restrict__ topk_idx, int64_t T, int E, int k, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv) {
-    extern __shared__ uint32_t sm[];
+__device__ __forceinline__ void permute_block(const int32_t* __restrict__ topk_idx, int64_t T, int E, int k,
+                                              int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok,
+                                              int32_t* __restrict__ inv, uint32_t* sm) {
     uint32_t* mask = sm;                   // [kWarps][E]
     uint32_t* wpre = mask + kWarps * E;    // [kWarps][E] exclusive prefix over warps
     int32_t* cnt = (int32_t*)(wpre + kWarps * E);  // [E]
@@ -171,15 +178,37 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
     }
 }
 
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t T, int E, int k, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv) {
+    extern __shared__ uint32_t sm[];
+    permute_block(topk_idx, T, E, k, offsets, perm_tok, inv, sm);
+}
+
+// Few tokens: one CTA routes them (a warp per token) and, after a barrier
+// that makes the top-k lists visible to the whole block, permutes them; one
+// launch instead of two. Thread 0 clears the workspace status word first.
+__global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
+    const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok,
+    int32_t* __restrict__ inv, int32_t* __restrict__ status) {
+    extern __shared__ uint32_t sm[];
+    if (threadIdx.x == 0) *status = 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int64_t t = warp; t < T; t += kWarps) route_token(logits, act_bf16, t, E, k, normalize, topk_idx, topk_w, lane);
+    __syncthreads();
+    permute_block(topk_idx, T, E, k, offsets, perm_tok, inv, sm);
+}
+
 }  // namespace
 
 cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
-                         int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+                         int32_t* topk_idx, float* topk_w, int32_t* status, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int threads = 256;
     const int64_t blocks = (T * 32 + threads - 1) / threads;
     route_kernel<<<unsigned(blocks), threads, 0, st>>>(logits, act_bf16, T, E, k, normalize,
-                                                       topk_idx, topk_w);
+                                                       topk_idx, topk_w, status);
     return cudaGetLastError();
 }
 
@@ -187,9 +216,22 @@ size_t permute_smem_bytes(int E) {
     return sizeof(uint32_t) * (2 * kWarps * E) + sizeof(int32_t) * (3 * E + 1);
 }
 
+cudaError_t launch_route_permute(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
+                                 int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm_tok,
+                                 int32_t* inv, int32_t* status, cudaStream_t st) {
+    route_permute_kernel<<<1, kPermThreads, permute_smem_bytes(E), st>>>(
+        logits, act_bf16, T, E, k, normalize, topk_idx, topk_w, offsets, perm_tok, inv, status);
+    return cudaGetLastError();
+}
+
+
 cudaError_t prepare_route_permute() {
-    return cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(permute_smem_bytes(256)));
+    cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(permute_smem_bytes(256)));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(route_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(permute_smem_bytes(256)));
+    return e;
 }
 
 cudaError_t launch_permute(const int32_t* topk_idx, int64_t T, int E, int k, int32_t* offsets,

@@ -35,6 +35,7 @@ EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forwa
            "qmoe_forward_profiled",
            "qmoe_debug_routing", "qmoe_debug_hidden", "qmoe_read_device_status", "qmoe_destroy",
            "qmoe_status_string", "qmoe_last_error", "qmoe_path_for", "qmoe_launches_for",
+           "qmoe_token_tile_for",
            "qmoe_set_option", "qmoe_forward_noalloc", "qmoe_noalloc_scratch_bytes")
 QMOE_OPT_PATH = 1
 
@@ -86,6 +87,8 @@ lib.qmoe_set_option.restype = ctypes.c_int
 lib.qmoe_set_option.argtypes = [_vp, ctypes.c_int32, _i64]
 lib.qmoe_launches_for.restype = ctypes.c_int32
 lib.qmoe_launches_for.argtypes = [_vp, _i64]
+lib.qmoe_token_tile_for.restype = ctypes.c_int32
+lib.qmoe_token_tile_for.argtypes = [_vp, _i64]
 
 
 class QMoEError(RuntimeError):
@@ -206,6 +209,10 @@ def qmoe_set_option(h, option: int, value: int):
 
 def qmoe_launches_for(h, T: int) -> int:
     return int(lib.qmoe_launches_for(h, T))
+
+
+def qmoe_token_tile_for(h, T: int) -> int:
+    return int(lib.qmoe_token_tile_for(h, T))
 
 
 # ------------------------------------------------------------- torch plumbing
