@@ -301,9 +301,9 @@ def run_ours(args):
     per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(launches)]
                            for i in range(K)]).mean(axis=0)
     path = qmoe.qmoe_path_for(h, T)
-    tc_path = path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE)
-    fused = launches == (5 if tc_path else 4)  # routing and permutation in one launch
-    names = ((["route_permute"] if fused else ["route", "permute"]) + (["gather"] if tc_path else [])
+    gather = path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE) or bool(cfg.apply_router_weight_on_input)
+    fused = launches - int(gather) - 3 == 1  # routing and permutation in one launch
+    names = ((["route_permute"] if fused else ["route", "permute"]) + (["gather"] if gather else [])
              + ["fc1", "fc2", "combine"])
 
     # ---- end to end through the public call, host buffers, copies inside

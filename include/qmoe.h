@@ -107,6 +107,25 @@ typedef struct qmoe_config {
     int32_t has_fc3_bias;
     int32_t use_sparse_mixer;     /* must be 0 */
     int32_t reserved;             /* must be 0 */
+    /* Routing options the "MoE" page names (n_group, topk_group,
+     * routed_scaling_factor, apply_router_weight_on_input) without formulas;
+     * readings:
+     *   grouped top-k -- the E experts form n_group consecutive groups of
+     *     E / n_group; a group's score is the largest raw logit among its
+     *     experts; the topk_group best groups are kept (ties to the lower group
+     *     id) and the k experts are the top-k by logit among their experts.
+     *     n_group 0 or 1: no grouping. Otherwise E % n_group == 0,
+     *     n_group <= 32, 1 <= topk_group <= n_group and
+     *     k <= topk_group * E / n_group.
+     *   routed_scaling_factor -- multiplies the router-weighted sum of the
+     *     expert outputs (not the shared output); 0 reads as 1.
+     *   apply_router_weight_on_input -- 1: the router weight scales the
+     *     expert's input row (rounded to the activation dtype) instead of its
+     *     output; the combine then sums the expert outputs unweighted. */
+    int32_t n_group;
+    int32_t topk_group;
+    float routed_scaling_factor;
+    int32_t apply_router_weight_on_input;
 } qmoe_config;
 
 typedef struct qmoe_handle qmoe_handle;

@@ -27,7 +27,10 @@ class _Cfg(ctypes.Structure):
                 ("block_size", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("fusion", ctypes.c_int32), ("normalize", ctypes.c_int32),
                 ("has_fc3", ctypes.c_int32), ("alpha", ctypes.c_double),
-                ("beta", ctypes.c_double), ("limit", ctypes.c_double)]
+                ("beta", ctypes.c_double), ("limit", ctypes.c_double),
+                ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
+                ("apply_router_weight_on_input", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_double)]
 
 
 def _load():
@@ -83,13 +86,14 @@ def dequant(packed: np.ndarray, scales: np.ndarray, N: int, K: int, bits: int,
     return w
 
 
-def route(logits: np.ndarray, k: int, normalize: bool):
+def route(logits: np.ndarray, k: int, normalize: bool, n_group: int = 0, topk_group: int = 0):
     lg = to_f64(logits)
     T, E = lg.shape
     idx = np.empty((T, k), dtype=np.int32)
     w = np.empty((T, k), dtype=np.float64)
     _load().oracle_route(_p(lg, _f64p), ctypes.c_int64(T), ctypes.c_int64(E), ctypes.c_int64(k),
-                         ctypes.c_int32(int(normalize)), _p(idx, _i32p), _p(w, _f64p))
+                         ctypes.c_int32(int(normalize)), ctypes.c_int32(n_group), ctypes.c_int32(topk_group),
+                         _p(idx, _i32p), _p(w, _f64p))
     return idx, w
 
 
@@ -133,7 +137,10 @@ def forward(inp, tokens: Optional[Sequence[int]] = None, want_h: bool = False) -
     cfg = _Cfg(T=T, H=c.H, I=c.I, E=c.E, k=c.k, bits=c.bits, block_size=c.block_size,
                act=c.act, fusion=c.fusion, normalize=int(c.normalize), has_fc3=int(c.has_fc3),
                alpha=float(c.alpha), beta=float(c.beta),
-               limit=float(c.limit) if c.limit is not None else math.inf)
+               limit=float(c.limit) if c.limit is not None else math.inf,
+               n_group=int(c.n_group), topk_group=int(c.topk_group),
+               apply_router_weight_on_input=int(c.apply_router_weight_on_input),
+               routed_scaling_factor=float(c.routed_scaling_factor) if c.routed_scaling_factor else 1.0)
     y = np.empty((T, c.H), dtype=np.float64)
     idx = np.empty((T, c.k), dtype=np.int32)
     w = np.empty((T, c.k), dtype=np.float64)

@@ -32,6 +32,18 @@
  *   - fusion 1: gate = even rows, up = odd rows; fusion 2: gate = first I
  *     rows, up = last I rows; fusion 0 with fc3: gate = fc1, up = fc3.
  *
+ * Routing options the "MoE" page names without formulas (n_group,
+ * topk_group, routed_scaling_factor, apply_router_weight_on_input), read as:
+ *   - grouped top-k: the E experts form n_group consecutive groups of
+ *     E / n_group; a group's score is the largest raw logit among its
+ *     experts; the topk_group groups with the highest scores are kept (ties
+ *     to the lower group id) and the k experts are the top-k by logit among
+ *     the kept groups' experts; n_group <= 1 means no grouping;
+ *   - routed_scaling_factor multiplies the router-weighted sum of the expert
+ *     outputs, not the shared output;
+ *   - apply_router_weight_on_input: the router weight multiplies the
+ *     expert's input row instead of its output.
+ *
  * Every sum is a serial fp64 loop in index order, so the result does not
  * depend on the thread count.
  */
@@ -55,6 +67,9 @@ typedef struct oracle_cfg {
     int32_t normalize;
     int32_t has_fc3;
     double alpha, beta, limit;
+    int32_t n_group, topk_group;         /* grouped top-k; n_group <= 1: none */
+    int32_t apply_router_weight_on_input;
+    double routed_scaling_factor;
 } oracle_cfg;
 
 int oracle_num_threads(void) {
@@ -96,16 +111,37 @@ void oracle_dequant(const uint8_t* packed, const double* scales, int64_t N, int6
 /* Routing ("MoE" page summary; QMoE page attributes k and
  * normalize_routing_weights). */
 void oracle_route(const double* logits, int64_t T, int64_t E, int64_t k, int32_t normalize,
-                  int32_t* idx, double* w) {
+                  int32_t n_group, int32_t topk_group, int32_t* idx, double* w) {
     char* taken = (char*)malloc((size_t)E);
+    char* allowed = (char*)malloc((size_t)E);
     double* p = (double*)malloc(sizeof(double) * (size_t)E);
+    const int64_t G = n_group > 1 ? n_group : 1, gsize = E / G;
+    char* kept = (char*)malloc((size_t)G);
     for (int64_t t = 0; t < T; ++t) {
         const double* l = logits + t * E;
+        /* groups: keep the topk_group groups of largest member logit */
+        memset(kept, G == 1, (size_t)G);
+        for (int64_t r = 0; G > 1 && r < topk_group; ++r) {
+            int64_t bestg = -1;
+            double bests = 0.0;
+            for (int64_t g = 0; g < G; ++g) {
+                if (kept[g]) continue;
+                double sg = l[g * gsize];
+                for (int64_t e = g * gsize + 1; e < (g + 1) * gsize; ++e)
+                    if (l[e] > sg) sg = l[e];
+                if (bestg < 0 || sg > bests) {
+                    bestg = g;
+                    bests = sg;
+                }
+            }
+            kept[bestg] = 1;
+        }
+        for (int64_t e = 0; e < E; ++e) allowed[e] = kept[e / gsize];
         memset(taken, 0, (size_t)E);
         for (int64_t j = 0; j < k; ++j) {
             int64_t best = -1;
             for (int64_t e = 0; e < E; ++e)
-                if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+                if (allowed[e] && !taken[e] && (best < 0 || l[e] > l[best])) best = e;
             taken[best] = 1;
             idx[t * k + j] = (int32_t)best;
         }
@@ -121,6 +157,8 @@ void oracle_route(const double* logits, int64_t T, int64_t E, int64_t k, int32_t
             w[t * k + j] = normalize ? p[idx[t * k + j]] / sel : p[idx[t * k + j]];
     }
     free(taken);
+    free(allowed);
+    free(kept);
     free(p);
 }
 
@@ -190,7 +228,8 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
     const int64_t pk1 = H * bits / 8, pk2 = I * bits / 8;
     const int64_t sc1 = bs > 0 ? H / bs : 1, sc2 = bs > 0 ? I / bs : 1;
 
-    oracle_route(logits, T, E, k, c->normalize, topk_idx, topk_w);
+    oracle_route(logits, T, E, k, c->normalize, c->n_group, c->topk_group, topk_idx, topk_w);
+    const double rsf = c->routed_scaling_factor;
 
     double* a1 = (double*)calloc((size_t)(R * N1), sizeof(double)); /* fc1 pre-activation */
     double* a3 = c->has_fc3 ? (double*)calloc((size_t)(R * I), sizeof(double)) : NULL;
@@ -216,8 +255,10 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
                 dequant_row(w1, s1, H, bits, bs, n, wrow);
                 for (int64_t i = 0; i < m; ++i) {
                     const int64_t r = rows[i], t = r / k;
+                    /* the expert's input row: x[t], or w[r] * x[t] */
+                    const double win = c->apply_router_weight_on_input ? topk_w[r] : 1.0;
                     double acc = 0.0;
-                    for (int64_t kk = 0; kk < H; ++kk) acc += x[t * H + kk] * wrow[kk];
+                    for (int64_t kk = 0; kk < H; ++kk) acc += (win * x[t * H + kk]) * wrow[kk];
                     if (fc1_b) acc += fc1_b[e * N1 + n];
                     a1[r * N1 + n] = acc;
                 }
@@ -230,8 +271,9 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
                     dequant_row(w3, s3, H, bits, bs, n, wrow);
                     for (int64_t i = 0; i < m; ++i) {
                         const int64_t r = rows[i], t = r / k;
+                        const double win = c->apply_router_weight_on_input ? topk_w[r] : 1.0;
                         double acc = 0.0;
-                        for (int64_t kk = 0; kk < H; ++kk) acc += x[t * H + kk] * wrow[kk];
+                        for (int64_t kk = 0; kk < H; ++kk) acc += (win * x[t * H + kk]) * wrow[kk];
                         if (fc3_b) acc += fc3_b[e * I + n];
                         a3[r * I + n] = acc;
                     }
@@ -286,11 +328,16 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
         }
     }
 
-    /* combine: y[t] = sum_j w[t, j] * o[t*k + j] + shared[t], j in list order */
+    /* combine: y[t] = rsf * sum_j w[t, j] * o[t*k + j] + shared[t], j in list
+     * order; the weight is 1 here when it already scaled the expert's input */
     for (int64_t t = 0; t < T; ++t)
         for (int64_t n = 0; n < H; ++n) {
             double acc = 0.0;
-            for (int64_t j = 0; j < k; ++j) acc += topk_w[t * k + j] * o[(t * k + j) * H + n];
+            for (int64_t j = 0; j < k; ++j) {
+                const double wj = c->apply_router_weight_on_input ? 1.0 : topk_w[t * k + j];
+                acc += wj * o[(t * k + j) * H + n];
+            }
+            acc *= rsf;
             if (shared) acc += shared[t * H + n];
             y[t * H + n] = acc;
         }

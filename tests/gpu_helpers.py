@@ -79,7 +79,7 @@ def run_gpu(inp: gen.MoEInputs, device="cuda:0", repeat: int = 1, path=None) -> 
 
 def check_routing(inp: gen.MoEInputs, g: GpuRun):
     c = inp.cfg
-    idx, w = oracle.route(inp.logits, c.k, c.normalize)
+    idx, w = oracle.route(inp.logits, c.k, c.normalize, c.n_group, c.topk_group)
     np.testing.assert_array_equal(g.topk_idx, idx)
     np.testing.assert_allclose(g.topk_w, w, rtol=TOL_ROUTE_W, atol=1e-30)
     off, perm, inv = oracle.permute(idx, c.E)

@@ -39,10 +39,12 @@ def test_library_exports_every_declared_symbol(q):
 
 
 def test_config_struct_layout(q):
-    assert ctypes.sizeof(q.qmoe_config) == 96
+    assert ctypes.sizeof(q.qmoe_config) == 112
     assert q.qmoe_config.expert_weight_bits.offset == 32
     assert q.qmoe_config.activation_alpha.offset == 48
     assert q.qmoe_config.reserved.offset == 92
+    assert q.qmoe_config.n_group.offset == 96
+    assert q.qmoe_config.apply_router_weight_on_input.offset == 108
 
 
 def _cfg(q, **kw):
@@ -66,6 +68,11 @@ BAD = [
     (dict(use_sparse_mixer=1), 3),                              # valid per the page, not built
     (dict(num_experts=512, k=2), 3),
     (dict(hidden_size=96, block_size=32), 3),                   # not a multiple of 64
+    (dict(n_group=3), 1),                                       # E = 8 not divisible by 3
+    (dict(n_group=4, topk_group=0), 1), (dict(n_group=4, topk_group=5), 1),
+    (dict(n_group=4, topk_group=1, k=3), 1),                    # k > topk_group * E / n_group
+    (dict(num_experts=128, n_group=64, topk_group=1, k=1), 3),  # more than 32 groups: not built
+    (dict(apply_router_weight_on_input=2), 1), (dict(routed_scaling_factor=-1.0), 1),
 ]
 
 

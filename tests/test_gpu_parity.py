@@ -76,6 +76,16 @@ CASES = {
                                      beta=1.0, limit=7.0, has_fc1_bias=True, has_fc2_bias=True),
     "wide_tile_int8_percol_fc3_shared": dict(T=520, E=4, k=2, H=256, I=384, bits=8, block_size=0, fusion=0,
                                              has_fc3=True, act=gen.ACT_SILU, normalize=False, has_shared=True),
+    # routing options of the MoE page
+    "grouped_topk": dict(T=40, E=16, k=4, n_group=4, topk_group=2),
+    "grouped_topk_one_group_int8": dict(T=33, E=32, k=3, n_group=8, topk_group=1, bits=8, block_size=64),
+    "routed_scale_shared": dict(routed_scaling_factor=2.5, has_shared=True, has_fc2_bias=True),
+    "weight_on_input_int8_bias": dict(apply_router_weight_on_input=True, bits=8, block_size=32,
+                                      has_fc1_bias=True, normalize=False),
+    "wide_tile_weight_on_input": dict(T=300, E=2, k=1, H=256, I=384, apply_router_weight_on_input=True,
+                                      normalize=False, routed_scaling_factor=0.5),
+    "fp32_weight_on_input_scaled": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, apply_router_weight_on_input=True,
+                                        routed_scaling_factor=0.75, normalize=False, block_size=32),
     "fp32_acts_int8": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, bits=8, block_size=32,
                            has_fc1_bias=True, has_fc2_bias=True, has_shared=True),
     "fp32_acts_percol_fc3": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_BF16, block_size=0,
@@ -114,8 +124,9 @@ def test_all_tokens_to_one_expert_and_empty_experts(cuda_device):
     check_full(inp, g)
 
 
-def test_logit_ties_break_to_lowest_id(cuda_device):
-    cfg = _cfg(T=64, E=16, k=3)
+@pytest.mark.parametrize("groups", [(0, 0), (4, 2), (8, 3)], ids=["plain", "4g2", "8g3"])
+def test_logit_ties_break_to_lowest_id(cuda_device, groups):
+    cfg = _cfg(T=64, E=16, k=3, n_group=groups[0], topk_group=groups[1])
     inp = gen.make_inputs(cfg, seed=6)
     rng = np.random.default_rng(6)
     lg = rng.integers(-2, 3, size=(cfg.T, cfg.E)).astype(np.float32) * 0.25  # many exact ties

@@ -134,6 +134,92 @@ def test_unnormalised_weights_are_softmax_probabilities():
     np.testing.assert_allclose(w2.sum(axis=1), 1.0, rtol=1e-15)
 
 
+# -------------------------------------------------------- routing options (MoE page)
+
+def test_golden_grouped_routing_examples():
+    for case in _golden("routing_grouped.json")["cases"]:
+        lg = np.array([case["logits"]], dtype=np.float64)  # the decimal values exactly
+        idx, w = oracle.route(lg, case["k"], case["normalize"], case["n_group"], case["topk_group"])
+        assert idx[0].tolist() == case["sel"], case
+        np.testing.assert_allclose(w[0], [_eval(s) for s in case["weights"]], rtol=1e-14)
+
+
+@pytest.mark.parametrize("E,G,TG,k", [(8, 4, 2, 3), (16, 4, 1, 4), (32, 8, 3, 6), (64, 8, 4, 6), (12, 3, 2, 5)])
+def test_grouped_routing_against_numpy_sorts(E, G, TG, k):
+    # an independent statement with numpy primitives: group maxima by a
+    # reshape, kept groups and the final choice by lexicographic sorts
+    rng = np.random.default_rng(E + G + TG + k)
+    lg = (rng.integers(-3, 4, size=(300, E)) * 0.5).astype(np.float32)  # many ties
+    idx, _ = oracle.route(lg, k, True, G, TG)
+    for t in range(lg.shape[0]):
+        row = lg[t].astype(np.float64)
+        gmax = row.reshape(G, E // G).max(axis=1)
+        kept = np.lexsort((np.arange(G), -gmax))[:TG]
+        allowed = np.isin(np.arange(E) // (E // G), kept)
+        cand = np.nonzero(allowed)[0]
+        order = cand[np.lexsort((cand, -row[cand]))]
+        np.testing.assert_array_equal(idx[t], order[:k])
+
+
+def test_all_groups_kept_is_plain_top_k():
+    rng = np.random.default_rng(7)
+    lg = rng.standard_normal((100, 16)).astype(np.float32)
+    for normalize in (True, False):
+        i0, w0 = oracle.route(lg, 4, normalize)
+        i1, w1 = oracle.route(lg, 4, normalize, 4, 4)
+        np.testing.assert_array_equal(i0, i1)
+        np.testing.assert_array_equal(w0, w1)
+
+
+def _small(**kw):
+    base = dict(T=6, H=64, I=64, E=4, k=2, bits=4, block_size=32, act=gen.ACT_SWIGLU, fusion=1,
+                normalize=True, act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, has_shared=True)
+    base.update(kw)
+    return gen.MoEConfig(**base)
+
+
+def test_routed_scaling_factor_scales_only_the_routed_sum():
+    # without a shared output, scaling by a power of two is exact
+    cfg = _small(has_shared=False)
+    inp = gen.make_inputs(cfg, 31)
+    y1 = oracle.forward(inp)["y"]
+    inp.cfg = dataclasses.replace(cfg, routed_scaling_factor=2.0)
+    np.testing.assert_array_equal(oracle.forward(inp)["y"], 2.0 * y1)
+    # the shared output is added after the scaling, unscaled
+    cfg = _small()
+    inp = gen.make_inputs(cfg, 31)
+    y1 = oracle.forward(inp)["y"]
+    inp.cfg = dataclasses.replace(cfg, routed_scaling_factor=0.25)
+    sh = oracle.to_f64(inp.shared)
+    np.testing.assert_allclose(oracle.forward(inp)["y"], 0.25 * (y1 - sh) + sh, rtol=0,
+                               atol=1e-14 * np.abs(y1).max())
+
+
+def test_router_weight_on_input_with_one_expert_and_renormalised_weight_changes_nothing():
+    # k = 1 with renormalisation: the weight is exactly 1 wherever it is applied
+    cfg = _small(k=1, has_fc1_bias=True, has_fc2_bias=True)
+    inp = gen.make_inputs(cfg, 32)
+    y0 = oracle.forward(inp)["y"]
+    inp.cfg = dataclasses.replace(cfg, apply_router_weight_on_input=True)
+    np.testing.assert_array_equal(oracle.forward(inp)["y"], y0)
+
+
+def test_router_weight_on_input_of_a_linear_ffn_equals_weight_on_output():
+    # identity activation, no biases: the FFN is linear, so w * FFN(x) = FFN(w * x)
+    cfg = _small(act=gen.ACT_IDENTITY, fusion=0, k=2, normalize=False)
+    inp = gen.make_inputs(cfg, 33)
+    y0 = oracle.forward(inp)["y"]
+    inp.cfg = dataclasses.replace(cfg, apply_router_weight_on_input=True)
+    y1 = oracle.forward(inp)["y"]
+    np.testing.assert_allclose(y1, y0, rtol=0, atol=1e-12 * np.abs(y0).max())
+    # with a non-linear activation the two placements differ
+    cfg = _small(k=2, normalize=False)
+    inp = gen.make_inputs(cfg, 33)
+    y0 = oracle.forward(inp)["y"]
+    inp.cfg = dataclasses.replace(cfg, apply_router_weight_on_input=True)
+    assert np.abs(oracle.forward(inp)["y"] - y0).max() > 1e-6 * np.abs(y0).max()
+
+
 # ------------------------------------------------------------------- permutation
 
 @pytest.mark.parametrize("T,E,k", [(1, 4, 2), (37, 8, 2), (64, 64, 6), (100, 5, 5)])

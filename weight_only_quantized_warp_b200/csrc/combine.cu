@@ -1,7 +1,8 @@
 // combine.cu -- router-weighted combine of the expert outputs.
 //
-// y[t] = sum_j w[t, j] * (o[inv[t, j]] + b2[e_j]) + shared[t], j in list
-// order, fp32, rounded once to the output dtype. The "MoE" page
+// y[t] = rsf * sum_j w[t, j] * (o[inv[t, j]] + b2[e_j]) + shared[t], j in
+// list order, fp32, rounded once to the output dtype (rsf: the
+// routed_scaling_factor; w = 1 when the weights scaled the expert inputs). The "MoE" page
 // (clika_runtime.nn) combines the expert outputs under the router weights;
 // "ClikaRT::nn::QMoEWoQ" forward() folds the optional shared_output into this
 // routed combine (no separate add pass). Reading: the fc2 bias belongs to the
@@ -30,7 +31,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int j = 0; j < a.k; ++j) {
             const int64_t pos = a.inv[t * a.k + j];
-            const float w = a.topk_w[t * a.k + j];
+            const float w = a.weights_on_input ? 1.0f : a.topk_w[t * a.k + j];
             float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             for (int s = 0; s < a.splits; ++s) {
                 const float4 p = __ldcs(reinterpret_cast<const float4*>(o + ((int64_t)s * a.R + pos) * a.H + m));
@@ -50,6 +51,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[q] = fmaf(w, v[q], acc[q]);
         }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] *= a.rsf;
         if (a.act_bf16) {
             if (a.shared) {
                 const uint2 sv = *reinterpret_cast<const uint2*>((const __nv_bfloat16*)a.shared + t * a.H + m);

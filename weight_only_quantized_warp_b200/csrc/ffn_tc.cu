@@ -381,7 +381,54 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* _
 }
 
 
+// Row p of the gathered activations is x[perm[p]] times the router weight
+// of the (token, slot) pair at position p (found through inv), rounded once to
+// the activation dtype. One thread per 16 bytes of output.
+__global__ void gather_rows_weighted_kernel(const void* __restrict__ x, const int32_t* __restrict__ perm,
+                                            const int32_t* __restrict__ inv, const float* __restrict__ topk_w,
+                                            int k, void* __restrict__ xp, int64_t R, int64_t H, int act_bf16) {
+    const int64_t per_vec = act_bf16 ? 8 : 4;
+    const int64_t row_vecs = H / per_vec;
+    const int64_t total = R * row_vecs;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t p = i / row_vecs, v = i - p * row_vecs;
+        const int64_t t = perm[p];
+        float w = 0.0f;
+        for (int j = 0; j < k; ++j)
+            if (inv[t * k + j] == p) w = topk_w[t * k + j];
+        const uint4 in = reinterpret_cast<const uint4*>(x)[t * row_vecs + v];
+        uint4 out;
+        if (act_bf16) {
+            const uint32_t u[4] = {in.x, in.y, in.z, in.w};
+            uint32_t r[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(u[q] << 16) * w,
+                                                               __uint_as_float(u[q] & 0xFFFF0000u) * w);
+                r[q] = *reinterpret_cast<const uint32_t*>(&b);
+            }
+            out = make_uint4(r[0], r[1], r[2], r[3]);
+        } else {
+            out = make_uint4(__float_as_uint(__uint_as_float(in.x) * w), __float_as_uint(__uint_as_float(in.y) * w),
+                             __float_as_uint(__uint_as_float(in.z) * w), __float_as_uint(__uint_as_float(in.w) * w));
+        }
+        reinterpret_cast<uint4*>(xp)[i] = out;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows_weighted(const void* x, const int32_t* perm, const int32_t* inv,
+                                        const float* topk_w, int k, void* xp, int64_t R, int64_t H, int act_bf16,
+                                        cudaStream_t st) {
+    if (R == 0) return cudaSuccess;
+    const int64_t vecs = H / (act_bf16 ? 8 : 4);
+    int64_t blocks = (R * vecs + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    gather_rows_weighted_kernel<<<unsigned(blocks), 256, 0, st>>>(x, perm, inv, topk_w, k, xp, R, H, act_bf16);
+    return cudaGetLastError();
+}
 
 cudaError_t prepare_ffn_tc() {
     cudaError_t e = prepare_bits<4, false>();

@@ -83,7 +83,10 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         p.fc2_splits = int(s);
     }
     p.fused_route = T <= kFusedRouteTokens;
-    p.launches = ((p.path == kPathTc || p.path == kPathTcDecode) ? 6 : 5) - (p.fused_route ? 1 : 0);
+    // the row gather runs on the tensor-core paths, and on every path when
+    // the router weights scale the expert inputs
+    p.gather = p.path == kPathTc || p.path == kPathTcDecode || c.apply_router_weight_on_input;
+    p.launches = (p.fused_route ? 1 : 2) + (p.gather ? 1 : 0) + 3;
     const size_t R = size_t(p.R);
     const size_t act = bf16 ? 2 : 4;
     size_t off = 0;
@@ -95,7 +98,7 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     p.off_offsets = off; off = align256(off + size_t(E + 1) * 4);
     p.off_h = off;       off = align256(off + R * size_t(I) * act);
     p.off_xperm = off;
-    off = align256(off + ((p.path == kPathTc || p.path == kPathTcDecode) ? R * size_t(H) * act : 0));
+    off = align256(off + (p.gather ? R * size_t(H) * act : 0));
     p.off_o = off;       off = align256(off + size_t(p.fc2_splits) * R * size_t(H) * 4);
     p.total = off;
     return p;
@@ -165,6 +168,19 @@ qmoe_status validate(const qmoe_config& c, std::string& why) {
     }
     if (c.num_experts * c.k > (int64_t(1) << 20))
         return bad(QMOE_UNSUPPORTED, "num_experts * k too large");
+    if (c.n_group < 0) return bad(QMOE_INVALID_ARGUMENT, "n_group must be >= 0");
+    if (c.n_group > 1) {
+        if (c.num_experts % c.n_group) return bad(QMOE_INVALID_ARGUMENT, "num_experts must divide by n_group");
+        if (c.topk_group < 1 || c.topk_group > c.n_group)
+            return bad(QMOE_INVALID_ARGUMENT, "topk_group must lie in [1, n_group]");
+        if (c.k > int64_t(c.topk_group) * (c.num_experts / c.n_group))
+            return bad(QMOE_INVALID_ARGUMENT, "k exceeds the experts of the kept groups");
+        if (c.n_group > 32) return bad(QMOE_UNSUPPORTED, "more than 32 expert groups is not built");
+    }
+    if (c.apply_router_weight_on_input != 0 && c.apply_router_weight_on_input != 1)
+        return bad(QMOE_INVALID_ARGUMENT, "apply_router_weight_on_input must be 0 or 1");
+    if (!(c.routed_scaling_factor >= 0.0f) || !std::isfinite(c.routed_scaling_factor))
+        return bad(QMOE_INVALID_ARGUMENT, "routed_scaling_factor must be finite and >= 0");
     return QMOE_OK;
 }
 
@@ -406,12 +422,12 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     int32_t* status = (int32_t*)(ws + p.off_status);  // cleared by the first kernel
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
     if (p.fused_route) {
-        if ((err = launch_route_permute(router_logits, bf16, T, E, k, c.normalize_routing_weights, idx, tw,
-                                        offsets, perm, inv, status, st)) != cudaSuccess)
+        if ((err = launch_route_permute(router_logits, bf16, T, E, k, c.normalize_routing_weights, c.n_group,
+                                        c.topk_group, idx, tw, offsets, perm, inv, status, st)) != cudaSuccess)
             return cuda_fail(h, err, "route+permute");
     } else {
-        if ((err = launch_route(router_logits, bf16, T, E, k, c.normalize_routing_weights, idx, tw, status,
-                                st)) != cudaSuccess)
+        if ((err = launch_route(router_logits, bf16, T, E, k, c.normalize_routing_weights, c.n_group, c.topk_group,
+                                idx, tw, status, st)) != cudaSuccess)
             return cuda_fail(h, err, "route");
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
         if ((err = launch_permute(idx, T, E, k, offsets, perm, inv, st)) != cudaSuccess)
@@ -454,12 +470,15 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     f2.gated = 0;
     f2.is_fc1 = 0;
     f2.splits = p.fc2_splits;
-    if (p.path == kPathTc || p.path == kPathTcDecode) {
+    if (p.gather) {
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
         void* xp = ws + p.off_xperm;
-        if ((err = launch_gather_rows(x, perm, xp, p.R, c.hidden_size * 2, st)) != cudaSuccess)
-            return cuda_fail(h, err, "gather");
+        err = c.apply_router_weight_on_input
+                  ? launch_gather_rows_weighted(x, perm, inv, tw, k, xp, p.R, c.hidden_size, bf16, st)
+                  : launch_gather_rows(x, perm, xp, p.R, c.hidden_size * 2, st);
+        if (err != cudaSuccess) return cuda_fail(h, err, "gather");
         f1.act = xp;
+        f1.rowmap = nullptr;  // rows already in segment order
     }
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
     err = p.path == kPathSimt        ? launch_ffn_simt(f1, st)
@@ -486,6 +505,8 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     ca.R = p.R;
     ca.k = k;
     ca.splits = p.fc2_splits;
+    ca.rsf = c.routed_scaling_factor > 0.0f ? c.routed_scaling_factor : 1.0f;
+    ca.weights_on_input = c.apply_router_weight_on_input;
     ca.act_bf16 = bf16;
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
     if ((err = launch_combine(ca, st)) != cudaSuccess) return cuda_fail(h, err, "combine");

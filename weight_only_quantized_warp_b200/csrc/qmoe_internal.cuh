@@ -59,6 +59,7 @@ struct Plan {
     bool ok = true;      // a kernel configuration exists for this shape
     int bn = 0;          // token tile of the tensor-core path
     bool fused_route = false;  // routing and permutation in one launch (few tokens)
+    bool gather = false;       // routed rows of x gathered (and weighted) into the workspace
     size_t off_idx = 0, off_w = 0, off_inv = 0, off_perm = 0, off_offsets = 0, off_status = 0,
            off_h = 0, off_o = 0, off_xperm = 0, total = 0;
 };
@@ -110,13 +111,13 @@ struct PackArgs {
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t st);
 
 // Top-k softmax routing: warp per token.
-cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
-                         int32_t* topk_idx, float* topk_w, int32_t* status, cudaStream_t st);
+cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int n_group,
+                         int topk_group, int32_t* topk_idx, float* topk_w, int32_t* status, cudaStream_t st);
 // Routing and permutation of at most kFusedRouteTokens tokens in one launch.
 constexpr int64_t kFusedRouteTokens = 64;
 cudaError_t launch_route_permute(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
-                                 int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm_tok,
-                                 int32_t* inv, int32_t* status, cudaStream_t st);
+                                 int n_group, int topk_group, int32_t* topk_idx, float* topk_w, int32_t* offsets,
+                                 int32_t* perm_tok, int32_t* inv, int32_t* status, cudaStream_t st);
 
 // Histogram, scan and stable scatter into per-expert segments (one CTA).
 // prepare_route_permute() raises the permute kernel's shared-memory limit on
@@ -170,6 +171,11 @@ bool tc_decode_fits(int64_t K, int splits, int bn, int block_size);
 cudaError_t launch_ffn_tc_decode(const FfnArgs& a, int bn, int32_t* status, cudaStream_t st);
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm, void* xp, int64_t R, int64_t row_bytes,
                                cudaStream_t st);
+// The same gather with each routed row scaled by its router weight
+// (apply_router_weight_on_input), rounded to the activation dtype.
+cudaError_t launch_gather_rows_weighted(const void* x, const int32_t* perm, const int32_t* inv,
+                                        const float* topk_w, int k, void* xp, int64_t R, int64_t H, int act_bf16,
+                                        cudaStream_t st);
 
 // Router-weighted combine with fc2 bias and shared output; sums the FC2
 // split partials in fixed order.
@@ -183,6 +189,8 @@ struct CombineArgs {
     void* y;                 // [T, H]
     int64_t T, H, R;
     int k, splits, act_bf16;
+    float rsf;               // routed_scaling_factor (1 when unset)
+    int weights_on_input;    // the router weights already scaled FC1's input rows
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 

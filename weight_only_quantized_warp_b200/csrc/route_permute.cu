@@ -25,10 +25,13 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
     return v > bv || (v == bv && e < be);
 }
 
-// Route token t with one warp (lane = this thread's lane).
+// Route token t with one warp (lane = this thread's lane). With n_group > 1
+// the experts form n_group consecutive groups; only the topk_group groups of
+// largest member logit (ties to the lower group id) may be selected.
 __device__ __forceinline__ void route_token(const void* logits, int act_bf16, int64_t t, int E, int k,
-                                            int normalize, int32_t* __restrict__ topk_idx,
-                                            float* __restrict__ topk_w, int lane) {
+                                            int normalize, int n_group, int topk_group,
+                                            int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                            int lane) {
     float v[kMaxPerLane];
     const int per = (E + 31) >> 5;
 #pragma unroll
@@ -55,6 +58,45 @@ __device__ __forceinline__ void route_token(const void* logits, int act_bf16, in
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
 
+    // allowed slots (bit i: expert lane + 32 i may be selected)
+    uint32_t allow = 0xffffffffu;
+    if (n_group > 1) {
+        const int gsize = E / n_group;
+        float gmax = -INFINITY;  // lane g: largest logit of group g
+        for (int g = 0; g < n_group; ++g) {
+            float m = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kMaxPerLane; ++i) {
+                const int e = lane + 32 * i;
+                if (i < per && e < E && e / gsize == g) m = fmaxf(m, v[i]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == g) gmax = m;
+        }
+        uint32_t kept = 0;
+        for (int r = 0; r < topk_group; ++r) {
+            float bv = (lane < n_group && !((kept >> lane) & 1u)) ? gmax : -INFINITY;
+            int bg = (lane < n_group && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int og = __shfl_xor_sync(0xffffffffu, bg, o);
+                if (better(ov, og, bv, bg)) {
+                    bv = ov;
+                    bg = og;
+                }
+            }
+            kept |= 1u << bg;
+        }
+        allow = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxPerLane; ++i) {
+            const int e = lane + 32 * i;
+            if (i < per && e < E && ((kept >> (e / gsize)) & 1u)) allow |= 1u << i;
+        }
+    }
+
     uint32_t taken = 0;
     float p_keep[kMaxPerLane];  // p_j kept by lane j%32 in slot j/32
     float sel = 0.0f;
@@ -64,7 +106,7 @@ __device__ __forceinline__ void route_token(const void* logits, int act_bf16, in
 #pragma unroll
         for (int i = 0; i < kMaxPerLane; ++i) {
             const int e = lane + 32 * i;
-            if (i < per && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, be)) {
+            if (i < per && e < E && ((allow & ~taken) >> i & 1u) && better(v[i], e, bv, be)) {
                 bv = v[i];
                 be = e;
             }
@@ -95,12 +137,13 @@ __device__ __forceinline__ void route_token(const void* logits, int act_bf16, in
 // One warp per token. Thread 0 also clears the workspace status word, which
 // no kernel of the forward has written yet.
 __global__ void route_kernel(const void* logits, int act_bf16, int64_t T, int E, int k,
-                             int normalize, int32_t* __restrict__ topk_idx,
+                             int normalize, int n_group, int topk_group, int32_t* __restrict__ topk_idx,
                              float* __restrict__ topk_w, int32_t* __restrict__ status) {
     if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
     const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
-    route_token(logits, act_bf16, t, E, k, normalize, topk_idx, topk_w, threadIdx.x & 31);
+    route_token(logits, act_bf16, t, E, k, normalize, n_group, topk_group, topk_idx, topk_w,
+                threadIdx.x & 31);
 }
 
 // One CTA of 1024 threads. Token chunks of 1024: for each chunk, warp-level
@@ -189,25 +232,26 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
 // that makes the top-k lists visible to the whole block, permutes them; one
 // launch instead of two. Thread 0 clears the workspace status word first.
 __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
-    const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_w, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok,
-    int32_t* __restrict__ inv, int32_t* __restrict__ status) {
+    const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int n_group, int topk_group,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv, int32_t* __restrict__ status) {
     extern __shared__ uint32_t sm[];
     if (threadIdx.x == 0) *status = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int64_t t = warp; t < T; t += kWarps) route_token(logits, act_bf16, t, E, k, normalize, topk_idx, topk_w, lane);
+    for (int64_t t = warp; t < T; t += kWarps)
+        route_token(logits, act_bf16, t, E, k, normalize, n_group, topk_group, topk_idx, topk_w, lane);
     __syncthreads();
     permute_block(topk_idx, T, E, k, offsets, perm_tok, inv, sm);
 }
 
 }  // namespace
 
-cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
-                         int32_t* topk_idx, float* topk_w, int32_t* status, cudaStream_t st) {
+cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int n_group,
+                         int topk_group, int32_t* topk_idx, float* topk_w, int32_t* status, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int threads = 256;
     const int64_t blocks = (T * 32 + threads - 1) / threads;
-    route_kernel<<<unsigned(blocks), threads, 0, st>>>(logits, act_bf16, T, E, k, normalize,
+    route_kernel<<<unsigned(blocks), threads, 0, st>>>(logits, act_bf16, T, E, k, normalize, n_group, topk_group,
                                                        topk_idx, topk_w, status);
     return cudaGetLastError();
 }
@@ -217,10 +261,10 @@ size_t permute_smem_bytes(int E) {
 }
 
 cudaError_t launch_route_permute(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
-                                 int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* perm_tok,
-                                 int32_t* inv, int32_t* status, cudaStream_t st) {
+                                 int n_group, int topk_group, int32_t* topk_idx, float* topk_w, int32_t* offsets,
+                                 int32_t* perm_tok, int32_t* inv, int32_t* status, cudaStream_t st) {
     route_permute_kernel<<<1, kPermThreads, permute_smem_bytes(E), st>>>(
-        logits, act_bf16, T, E, k, normalize, topk_idx, topk_w, offsets, perm_tok, inv, status);
+        logits, act_bf16, T, E, k, normalize, n_group, topk_group, topk_idx, topk_w, offsets, perm_tok, inv, status);
     return cudaGetLastError();
 }
 

@@ -69,6 +69,12 @@ class MoEConfig:
     has_fc3: bool = False
     has_fc3_bias: bool = False
     has_shared: bool = False
+    # routing options of the MoE page: grouped top-k (n_group <= 1: none),
+    # scaling of the routed sum (0 reads as 1), router weight on the input
+    n_group: int = 0
+    topk_group: int = 0
+    routed_scaling_factor: float = 1.0
+    apply_router_weight_on_input: bool = False
 
     @property
     def gated(self) -> bool:

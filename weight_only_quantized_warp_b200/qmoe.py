@@ -50,7 +50,9 @@ class qmoe_config(ctypes.Structure):
                 ("act_dtype", ctypes.c_int32), ("scale_dtype", ctypes.c_int32),
                 ("has_fc1_bias", ctypes.c_int32), ("has_fc2_bias", ctypes.c_int32),
                 ("has_fc3", ctypes.c_int32), ("has_fc3_bias", ctypes.c_int32),
-                ("use_sparse_mixer", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("use_sparse_mixer", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float), ("apply_router_weight_on_input", ctypes.c_int32)]
 
 
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
@@ -136,7 +138,10 @@ def make_config(cfg) -> qmoe_config:
         swiglu_limit=lim, normalize_routing_weights=int(cfg.normalize), act_dtype=cfg.act_dtype,
         scale_dtype=cfg.scale_dtype, has_fc1_bias=int(cfg.has_fc1_bias),
         has_fc2_bias=int(cfg.has_fc2_bias), has_fc3=int(cfg.has_fc3),
-        has_fc3_bias=int(cfg.has_fc3_bias), use_sparse_mixer=0, reserved=0)
+        has_fc3_bias=int(cfg.has_fc3_bias), use_sparse_mixer=0, reserved=0,
+        n_group=int(getattr(cfg, "n_group", 0)), topk_group=int(getattr(cfg, "topk_group", 0)),
+        routed_scaling_factor=float(getattr(cfg, "routed_scaling_factor", 1.0)),
+        apply_router_weight_on_input=int(getattr(cfg, "apply_router_weight_on_input", False)))
 
 
 def qmoe_create(cfg: qmoe_config) -> int:
