@@ -69,7 +69,19 @@ enum {
     QMOE_ACT_IDENTITY = 4
 };
 
-enum { QMOE_DTYPE_F32 = 0, QMOE_DTYPE_BF16 = 1 };
+/* dtypes; E8M0 (a power-of-two exponent byte, value 2^(x - 127)) is a
+ * scale dtype of MXFP4 weights only. */
+enum { QMOE_DTYPE_F32 = 0, QMOE_DTYPE_BF16 = 1, QMOE_DTYPE_E8M0 = 2 };
+
+/* weight_format. INT: unsigned integer codes with the implicit zero point
+ * 2^(bits-1). MXFP4 (the block format of the QMoEWoQ page's gpt-oss
+ * checkpoint, read as the OCP microscaling FP4 format): each 4-bit code is
+ * e2m1 -- sign, two exponent bits, one mantissa bit, magnitudes 0, 0.5, 1,
+ * 1.5, 2, 3, 4, 6 -- packed two per byte like int4 (even k in the low
+ * nibble), with one E8M0 scale per 32 codes along K; requires
+ * expert_weight_bits 4, block_size 32 and scale_dtype E8M0. The activations
+ * stay floating point either way. */
+enum { QMOE_WEIGHTS_INT = 0, QMOE_WEIGHTS_MXFP4 = 1 };
 
 /*
  * Operator attributes ("QMoE" page attribute list; "ClikaRT::nn::QMoEWoQ",
@@ -126,6 +138,8 @@ typedef struct qmoe_config {
     int32_t topk_group;
     float routed_scaling_factor;
     int32_t apply_router_weight_on_input;
+    int32_t weight_format;        /* QMOE_WEIGHTS_* */
+    int32_t reserved2;            /* must be 0 */
 } qmoe_config;
 
 typedef struct qmoe_handle qmoe_handle;

@@ -30,7 +30,8 @@ class _Cfg(ctypes.Structure):
                 ("beta", ctypes.c_double), ("limit", ctypes.c_double),
                 ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
                 ("apply_router_weight_on_input", ctypes.c_int32),
-                ("routed_scaling_factor", ctypes.c_double)]
+                ("routed_scaling_factor", ctypes.c_double),
+                ("mxfp4", ctypes.c_int32)]
 
 
 def _load():
@@ -44,6 +45,8 @@ def _load():
         lib.oracle_plain_act.restype = ctypes.c_double
         lib.oracle_plain_act.argtypes = [ctypes.c_int32, ctypes.c_double]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_e2m1.restype = ctypes.c_double
+        lib.oracle_e2m1.argtypes = [ctypes.c_int32]
         _lib = lib
     return _lib
 
@@ -53,12 +56,16 @@ def num_threads() -> int:
 
 
 def to_f64(a: Optional[np.ndarray]) -> Optional[np.ndarray]:
-    """Widen stored values to fp64: uint16 arrays are bf16 bit patterns."""
+    """Widen stored values to fp64: uint16 arrays are bf16 bit patterns,
+    uint8 arrays E8M0 scales (2^(x - 127); x = 255 is NaN)."""
     if a is None:
         return None
     a = np.asarray(a)
     if a.dtype == np.uint16:
         return np.ascontiguousarray((a.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    if a.dtype == np.uint8:
+        v = np.ldexp(1.0, a.astype(np.int64) - 127)
+        return np.ascontiguousarray(np.where(a == 255, np.nan, v))
     return np.ascontiguousarray(a, dtype=np.float64)
 
 
@@ -76,13 +83,14 @@ def unpack(packed: np.ndarray, N: int, K: int, bits: int) -> np.ndarray:
 
 
 def dequant(packed: np.ndarray, scales: np.ndarray, N: int, K: int, bits: int,
-            block_size: int) -> np.ndarray:
+            block_size: int, mxfp4: bool = False) -> np.ndarray:
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
     s = to_f64(scales)
     assert s.size == (N * (K // block_size) if block_size > 0 else N)
     w = np.empty((N, K), dtype=np.float64)
     _load().oracle_dequant(_p(packed, _u8p), _p(s, _f64p), ctypes.c_int64(N), ctypes.c_int64(K),
-                           ctypes.c_int32(bits), ctypes.c_int64(block_size), _p(w, _f64p))
+                           ctypes.c_int32(bits), ctypes.c_int64(block_size), ctypes.c_int32(int(mxfp4)),
+                           _p(w, _f64p))
     return w
 
 
@@ -106,6 +114,11 @@ def permute(idx: np.ndarray, E: int):
     _load().oracle_permute(_p(idx, _i32p), ctypes.c_int64(T), ctypes.c_int64(E), ctypes.c_int64(k),
                            _p(offsets, _i32p), _p(perm, _i32p), _p(inv, _i32p))
     return offsets, perm, inv
+
+
+def e2m1(code: int) -> float:
+    """Value of one MXFP4 (e2m1) code."""
+    return float(_load().oracle_e2m1(code))
 
 
 def gated_act(act: int, g: float, u: float, alpha: float, beta: float, limit: float) -> float:
@@ -140,7 +153,8 @@ def forward(inp, tokens: Optional[Sequence[int]] = None, want_h: bool = False) -
                limit=float(c.limit) if c.limit is not None else math.inf,
                n_group=int(c.n_group), topk_group=int(c.topk_group),
                apply_router_weight_on_input=int(c.apply_router_weight_on_input),
-               routed_scaling_factor=float(c.routed_scaling_factor) if c.routed_scaling_factor else 1.0)
+               routed_scaling_factor=float(c.routed_scaling_factor) if c.routed_scaling_factor else 1.0,
+               mxfp4=int(c.weight_format == 1))
     y = np.empty((T, c.H), dtype=np.float64)
     idx = np.empty((T, c.k), dtype=np.int32)
     w = np.empty((T, c.k), dtype=np.float64)

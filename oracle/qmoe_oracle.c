@@ -44,6 +44,13 @@
  *   - apply_router_weight_on_input: the router weight multiplies the
  *     expert's input row instead of its output.
  *
+ * MXFP4 weights (the block format the QMoEWoQ page names for its gpt-oss
+ * checkpoint), read as OCP microscaling FP4: a 4-bit code is e2m1 -- sign
+ * bit 3, exponent bits 2-1, mantissa bit 0; exponent 0 is subnormal
+ * (m * 0.5), otherwise 2^(e - 1) * (1 + m / 2) -- packed like int4 codes,
+ * with one E8M0 scale 2^(x - 127) per 32 codes along K (the scales arrive
+ * here already as fp64 values).
+ *
  * Every sum is a serial fp64 loop in index order, so the result does not
  * depend on the thread count.
  */
@@ -70,6 +77,7 @@ typedef struct oracle_cfg {
     int32_t n_group, topk_group;         /* grouped top-k; n_group <= 1: none */
     int32_t apply_router_weight_on_input;
     double routed_scaling_factor;
+    int32_t mxfp4;                       /* codes are e2m1, no zero point */
 } oracle_cfg;
 
 int oracle_num_threads(void) {
@@ -92,20 +100,28 @@ void oracle_unpack(const uint8_t* packed, int64_t N, int64_t K, int32_t bits, in
         for (int64_t k = 0; k < K; ++k) q[n * K + k] = code_at(packed, K, bits, n, k);
 }
 
+/* Value of an e2m1 code (MXFP4). */
+double oracle_e2m1(int32_t code) {
+    const int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
 /* One dequantised row: w[k] = (q[n,k] - 2^(bits-1)) * s, s from the block of k
- * (QMoE page, fcX_scales and block_size). */
+ * (QMoE page, fcX_scales and block_size); MXFP4: w[k] = e2m1(q[n,k]) * s. */
 static void dequant_row(const uint8_t* packed, const double* scales, int64_t K, int bits,
-                        int64_t bs, int64_t n, double* w) {
+                        int64_t bs, int32_t mxfp4, int64_t n, double* w) {
     const int32_t z = 1 << (bits - 1);
     for (int64_t k = 0; k < K; ++k) {
         const double s = bs > 0 ? scales[n * (K / bs) + k / bs] : scales[n];
-        w[k] = (double)(code_at(packed, K, bits, n, k) - z) * s;
+        const int32_t q = code_at(packed, K, bits, n, k);
+        w[k] = (mxfp4 ? oracle_e2m1(q) : (double)(q - z)) * s;
     }
 }
 
 void oracle_dequant(const uint8_t* packed, const double* scales, int64_t N, int64_t K,
-                    int32_t bits, int64_t bs, double* w) {
-    for (int64_t n = 0; n < N; ++n) dequant_row(packed, scales, K, bits, bs, n, w + n * K);
+                    int32_t bits, int64_t bs, int32_t mxfp4, double* w) {
+    for (int64_t n = 0; n < N; ++n) dequant_row(packed, scales, K, bits, bs, mxfp4, n, w + n * K);
 }
 
 /* Routing ("MoE" page summary; QMoE page attributes k and
@@ -252,7 +268,7 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
             double* wrow = (double*)malloc(sizeof(double) * (size_t)H);
 #pragma omp for schedule(static)
             for (int64_t n = 0; n < N1; ++n) {
-                dequant_row(w1, s1, H, bits, bs, n, wrow);
+                dequant_row(w1, s1, H, bits, bs, c->mxfp4, n, wrow);
                 for (int64_t i = 0; i < m; ++i) {
                     const int64_t r = rows[i], t = r / k;
                     /* the expert's input row: x[t], or w[r] * x[t] */
@@ -268,7 +284,7 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
                 const double* s3 = fc3_s + e * I * sc1;
 #pragma omp for schedule(static)
                 for (int64_t n = 0; n < I; ++n) {
-                    dequant_row(w3, s3, H, bits, bs, n, wrow);
+                    dequant_row(w3, s3, H, bits, bs, c->mxfp4, n, wrow);
                     for (int64_t i = 0; i < m; ++i) {
                         const int64_t r = rows[i], t = r / k;
                         const double win = c->apply_router_weight_on_input ? topk_w[r] : 1.0;
@@ -315,7 +331,7 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
             double* wrow = (double*)malloc(sizeof(double) * (size_t)I);
 #pragma omp for schedule(static)
             for (int64_t n = 0; n < H; ++n) {
-                dequant_row(w2, s2, I, bits, bs, n, wrow);
+                dequant_row(w2, s2, I, bits, bs, c->mxfp4, n, wrow);
                 for (int64_t i = 0; i < m; ++i) {
                     const int64_t r = rows[i];
                     double acc = 0.0;

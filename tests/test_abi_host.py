@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(q):
 
 
 def test_config_struct_layout(q):
-    assert ctypes.sizeof(q.qmoe_config) == 112
+    assert ctypes.sizeof(q.qmoe_config) == 120
     assert q.qmoe_config.expert_weight_bits.offset == 32
     assert q.qmoe_config.activation_alpha.offset == 48
     assert q.qmoe_config.reserved.offset == 92
@@ -73,6 +73,11 @@ BAD = [
     (dict(n_group=4, topk_group=1, k=3), 1),                    # k > topk_group * E / n_group
     (dict(num_experts=128, n_group=64, topk_group=1, k=1), 3),  # more than 32 groups: not built
     (dict(apply_router_weight_on_input=2), 1), (dict(routed_scaling_factor=-1.0), 1),
+    (dict(weight_format=2), 1), (dict(reserved2=1), 1),
+    (dict(weight_format=1, block_size=32), 1),                  # MXFP4 needs E8M0 scales
+    (dict(weight_format=1, block_size=64, scale_dtype=2), 1),   # ... and block_size 32
+    (dict(weight_format=1, expert_weight_bits=8, block_size=32, scale_dtype=2), 1),
+    (dict(scale_dtype=2), 1),                                   # E8M0 only with MXFP4
 ]
 
 

@@ -86,6 +86,14 @@ CASES = {
                                       normalize=False, routed_scaling_factor=0.5),
     "fp32_weight_on_input_scaled": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, apply_router_weight_on_input=True,
                                         routed_scaling_factor=0.75, normalize=False, block_size=32),
+    # MXFP4 expert weights (e2m1 codes, E8M0 scale per 32)
+    "mxfp4_swiglu_bias": dict(weight_format=gen.WEIGHTS_MXFP4, block_size=32, scale_dtype=gen.DT_E8M0, fusion=1,
+                              alpha=1.702, beta=1.0, limit=7.0, has_fc1_bias=True, has_fc2_bias=True),
+    "mxfp4_k128": dict(weight_format=gen.WEIGHTS_MXFP4, block_size=32, scale_dtype=gen.DT_E8M0, H=256, I=384),
+    "mxfp4_wide_tile": dict(weight_format=gen.WEIGHTS_MXFP4, block_size=32, scale_dtype=gen.DT_E8M0, T=300, E=2,
+                            k=1, H=256, I=384),
+    "mxfp4_fp32_acts": dict(weight_format=gen.WEIGHTS_MXFP4, block_size=32, scale_dtype=gen.DT_E8M0,
+                            act_dtype=gen.DT_F32, has_shared=True),
     "fp32_acts_int8": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, bits=8, block_size=32,
                            has_fc1_bias=True, has_fc2_bias=True, has_shared=True),
     "fp32_acts_percol_fc3": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_BF16, block_size=0,
@@ -184,7 +192,7 @@ def _sample(T, n=8, seed=0):
 
 
 @pytest.mark.parametrize("path", [None, PATH_DECODE, PATH_TC, PATH_TC_DECODE], ids=["auto", "decode", "tc", "tcdecode"])
-@pytest.mark.parametrize("name", ["mixtral_decode", "gpt_oss", "deepseek"])
+@pytest.mark.parametrize("name", ["mixtral_decode", "gpt_oss", "gpt_oss_mxfp4", "deepseek"])
 def test_full_size_configs(cuda_device, name, path):
     cfg, seed, kw = gen.workload(name)
     inp = gen.make_inputs(cfg, seed, **kw)

@@ -88,6 +88,58 @@ def test_dequant_round_trip_exact(bits, bs):
     np.testing.assert_array_equal(got, W)
 
 
+# ------------------------------------------------------------------------ MXFP4
+
+def _mx_table():
+    g = _golden("mxfp4_codes.json")
+    return {c["code"]: _eval(c["value"]) for c in g["codes"]}
+
+
+def test_mxfp4_code_and_scale_values():
+    table = _mx_table()
+    for code, v in table.items():
+        got = oracle.e2m1(code)
+        assert got == v and math.copysign(1.0, got) == math.copysign(1.0, v), code
+    for sc in _golden("mxfp4_codes.json")["scales"]:
+        assert oracle.to_f64(np.array([sc["byte"]], dtype=np.uint8))[0] == _eval(sc["value"])
+    assert np.isnan(oracle.to_f64(np.array([255], dtype=np.uint8))[0])
+
+
+def test_mxfp4_dequant_of_every_code_at_every_position():
+    # codes cycle through all 16 values at every k parity; scales from bytes
+    table = _mx_table()
+    N, K = 16, 64
+    q = (np.arange(N * K).reshape(N, K) * 7 + np.arange(N)[:, None]) % 16
+    xb = (120 + (np.arange(N * (K // 32)) % 9)).astype(np.uint8).reshape(N, K // 32)
+    want = np.vectorize(table.get)(q) * np.ldexp(1.0, xb.astype(np.int64) - 127)[:, np.arange(K) // 32]
+    got = oracle.dequant(_pack_codes(q, 4), xb, N, K, 4, 32, mxfp4=True)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_mxfp4_single_expert_is_the_qlinear_chain():
+    # one expert forced (k = 1, renormalised): y = QLinear(act(QLinear(x))) with
+    # the weights decoded through the format table, by numpy
+    table = _mx_table()
+    cfg = gen.MoEConfig(T=5, H=64, I=32, E=3, k=1, bits=4, block_size=32, act=gen.ACT_SWIGLU, fusion=2,
+                        normalize=True, act_dtype=gen.DT_F32, scale_dtype=gen.DT_E8M0,
+                        has_fc1_bias=True, has_fc2_bias=True, weight_format=gen.WEIGHTS_MXFP4)
+    inp = gen.make_inputs(cfg, 41, bias_std=0.1)
+    lg = np.full((cfg.T, cfg.E), -30.0, dtype=np.float32)
+    lg[:, 1] = 5.0
+    inp.logits = lg
+    def deq(w, sc, N, K):
+        q = oracle.unpack(w, N, K, 4)
+        return np.vectorize(table.get)(q) * np.ldexp(1.0, sc.astype(np.int64) - 127)[:, np.arange(K) // 32]
+    W1 = deq(inp.fc1_w[1], inp.fc1_s[1], 2 * cfg.I, cfg.H)
+    W2 = deq(inp.fc2_w[1], inp.fc2_s[1], cfg.H, cfg.I)
+    x = inp.x.astype(np.float64)
+    a = x @ W1.T + inp.fc1_b[1].astype(np.float64)
+    g, u = a[:, :cfg.I], a[:, cfg.I:]
+    h = g * expit(g) * u
+    y = h @ W2.T + inp.fc2_b[1].astype(np.float64)
+    np.testing.assert_allclose(oracle.forward(inp)["y"], y, rtol=1e-12, atol=1e-12 * np.abs(y).max())
+
+
 # ----------------------------------------------------------------------- routing
 
 def test_golden_routing_examples():

@@ -37,6 +37,7 @@
 #include <algorithm>
 
 #include "qmoe_internal.cuh"
+#include "fp4_decode.cuh"
 
 namespace qmoe {
 namespace {
@@ -426,7 +427,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArg
                                             nibble_centered(wv[j], q + 4) * s);
                         }
                     } else {
-                        decode_int4(wv[j], A);
+                        if (a.fp4)
+                            decode_fp4x8(wv[j], A);  // MXFP4: e2m1 values, no zero point
+                        else
+                            decode_int4(wv[j], A);
                         const __nv_bfloat162 pa = __float2bfloat162_rn(sa);
                         const __nv_bfloat162 pb = __float2bfloat162_rn(sb);
                         const uint32_t ua = *reinterpret_cast<const uint32_t*>(&pa);
@@ -604,7 +608,8 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
                     for (int p = 0; p < 8; ++p)
-                        q[p & 1][4 * j + 2 * ((p >> 1) & 1) + (p >> 2)] = nibble_centered(wv[j], p);
+                        q[p & 1][4 * j + 2 * ((p >> 1) & 1) + (p >> 2)] =
+                            a.fp4 ? fp4_to_float(wv[j] >> (4 * p)) : nibble_centered(wv[j], p);
             } else {
 #pragma unroll
                 for (int j = 0; j < 2; ++j)

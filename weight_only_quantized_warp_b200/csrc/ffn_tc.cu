@@ -43,6 +43,7 @@
 
 #include "qmoe_internal.cuh"
 #include "tc_common.cuh"
+#include "fp4_decode.cuh"
 
 namespace qmoe {
 namespace {
@@ -73,7 +74,7 @@ struct TcCfg {
     static constexpr int kSmem = kSmemUse > 120 * 1024 ? kSmemUse : 120 * 1024;
 };
 
-template <int BITS, bool PERCOL, int BNMAX, int STAGES>
+template <int BITS, bool PERCOL, int BNMAX, int STAGES, bool FP4>
 __global__ void __launch_bounds__(kTcThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap bmap, const TcArgs a) {
     using C = TcCfg<BITS, PERCOL, BNMAX, STAGES>;
@@ -248,7 +249,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j) {
                         uint32_t A[4];  // (r0, k 0-1), (r0+8, k 0-1), (r0, k 2-3), (r0+8, k 2-3)
-                        if (BITS == 4) {
+                        if (BITS == 4 && FP4) {
+                            decode_fp4x8(wv[j], A);  // MXFP4: e2m1 values, no zero point
+                        } else if (BITS == 4) {
                             A[0] = bf2_sub((wv[j] & kMask) | kMagic, kBias4);
                             A[1] = bf2_sub(((wv[j] >> 4) & kMask) | kMagic, kBias4);
                             A[2] = bf2_sub(((wv[j] >> 8) & kMask) | kMagic, kBias4);
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-template <int BITS, bool PERCOL, int BNMAX>
+template <int BITS, bool PERCOL, int BNMAX, bool FP4>
 struct Launch {
     static constexpr int kStage = TcCfg<BITS, PERCOL, BNMAX, 1>::kStage;
     static constexpr int kByTmem = (512 - 2 * BNMAX) / kAStageCols;
@@ -342,31 +345,31 @@ struct Launch {
     static constexpr int kStages = kByTmem < kBySmem ? (kByTmem < 12 ? kByTmem : 12) : (kBySmem < 12 ? kBySmem : 12);
     using C = TcCfg<BITS, PERCOL, BNMAX, kStages>;
     static cudaError_t prepare() {
-        return cudaFuncSetAttribute(ffn_tc_kernel<BITS, PERCOL, BNMAX, kStages>,
+        return cudaFuncSetAttribute(ffn_tc_kernel<BITS, PERCOL, BNMAX, kStages, FP4>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     }
     static cudaError_t run(const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t st) {
-        ffn_tc_kernel<BITS, PERCOL, BNMAX, kStages><<<grid, kTcThreads, C::kSmem, st>>>(map, a);
+        ffn_tc_kernel<BITS, PERCOL, BNMAX, kStages, FP4><<<grid, kTcThreads, C::kSmem, st>>>(map, a);
         return cudaGetLastError();
     }
 };
 
-template <int BITS, bool PERCOL>
+template <int BITS, bool PERCOL, bool FP4>
 cudaError_t dispatch_bn(int bnmax, const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t st) {
     switch (bnmax) {
-        case 16: return Launch<BITS, PERCOL, 16>::run(map, a, grid, st);
-        case 32: return Launch<BITS, PERCOL, 32>::run(map, a, grid, st);
-        case 64: return Launch<BITS, PERCOL, 64>::run(map, a, grid, st);
-        default: return Launch<BITS, PERCOL, 128>::run(map, a, grid, st);
+        case 16: return Launch<BITS, PERCOL, 16, FP4>::run(map, a, grid, st);
+        case 32: return Launch<BITS, PERCOL, 32, FP4>::run(map, a, grid, st);
+        case 64: return Launch<BITS, PERCOL, 64, FP4>::run(map, a, grid, st);
+        default: return Launch<BITS, PERCOL, 128, FP4>::run(map, a, grid, st);
     }
 }
 
-template <int BITS, bool PERCOL>
+template <int BITS, bool PERCOL, bool FP4>
 cudaError_t prepare_bits() {
-    cudaError_t e = Launch<BITS, PERCOL, 16>::prepare();
-    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 32>::prepare();
-    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 64>::prepare();
-    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 128>::prepare();
+    cudaError_t e = Launch<BITS, PERCOL, 16, FP4>::prepare();
+    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 32, FP4>::prepare();
+    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 64, FP4>::prepare();
+    if (e == cudaSuccess) e = Launch<BITS, PERCOL, 128, FP4>::prepare();
     return e;
 }
 
@@ -431,10 +434,11 @@ cudaError_t launch_gather_rows_weighted(const void* x, const int32_t* perm, cons
 }
 
 cudaError_t prepare_ffn_tc() {
-    cudaError_t e = prepare_bits<4, false>();
-    if (e == cudaSuccess) e = prepare_bits<4, true>();
-    if (e == cudaSuccess) e = prepare_bits<8, false>();
-    if (e == cudaSuccess) e = prepare_bits<8, true>();
+    cudaError_t e = prepare_bits<4, false, false>();
+    if (e == cudaSuccess) e = prepare_bits<4, true, false>();
+    if (e == cudaSuccess) e = prepare_bits<8, false, false>();
+    if (e == cudaSuccess) e = prepare_bits<8, true, false>();
+    if (e == cudaSuccess) e = prepare_bits<4, false, true>();  // MXFP4
     if (e == cudaSuccess) e = prepare_ffn_tc_decode();
     if (e == cudaSuccess) e = prepare_ffn_tc_wide();
     return e;
@@ -494,8 +498,11 @@ cudaError_t launch_ffn_tc(const FfnArgs& f, int bn, int32_t* status, cudaStream_
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const bool percol = f.block_size == 0;
     if (f.bits == 4)
-        return percol ? dispatch_bn<4, true>(bnmax, map, a, sms, st) : dispatch_bn<4, false>(bnmax, map, a, sms, st);
-    return percol ? dispatch_bn<8, true>(bnmax, map, a, sms, st) : dispatch_bn<8, false>(bnmax, map, a, sms, st);
+        return f.fp4    ? dispatch_bn<4, false, true>(bnmax, map, a, sms, st)
+               : percol ? dispatch_bn<4, true, false>(bnmax, map, a, sms, st)
+                        : dispatch_bn<4, false, false>(bnmax, map, a, sms, st);
+    return percol ? dispatch_bn<8, true, false>(bnmax, map, a, sms, st)
+                  : dispatch_bn<8, false, false>(bnmax, map, a, sms, st);
 }
 
 }  // namespace qmoe

@@ -37,6 +37,7 @@
 
 #include "qmoe_internal.cuh"
 #include "tc_common.cuh"
+#include "fp4_decode.cuh"
 
 namespace qmoe {
 namespace {
@@ -107,7 +108,7 @@ __device__ __forceinline__ int scale_pos(int row) {
     return (row >> 4) * 16 + (rr & 7) * 2 + (rr >> 3);
 }
 
-template <int BITS, int SMODE, int BN>
+template <int BITS, int SMODE, int BN, bool FP4>
 __global__ void __launch_bounds__(kDThreads, 1)
     ffn_tc_decode_kernel(const __grid_constant__ CUtensorMap bmap, const TcArgs a) {
     using C = TcdCfg<BITS, SMODE, BN>;
@@ -341,7 +342,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j) {
                         uint32_t A[4];  // (r0, k 0-1), (r0+8, k 0-1), (r0, k 2-3), (r0+8, k 2-3)
-                        if (BITS == 4) {
+                        if (BITS == 4 && FP4) {
+                            decode_fp4x8(wv[j], A);  // MXFP4: e2m1 values, no zero point
+                        } else if (BITS == 4) {
                             // nibble q OR bf16 128.0 is 128 + q exactly; minus 136.0 gives q - 8
                             A[0] = bf2_sub((wv[j] & kMask) | kMagic, kBias4);
                             A[1] = bf2_sub(((wv[j] >> 4) & kMask) | kMagic, kBias4);
@@ -494,39 +497,39 @@ __global__ void __launch_bounds__(kDThreads, 1)
     }
 }
 
-template <int BITS, int SMODE, int BN>
+template <int BITS, int SMODE, int BN, bool FP4>
 struct LaunchD {
     static cudaError_t prepare() {
-        return cudaFuncSetAttribute(ffn_tc_decode_kernel<BITS, SMODE, BN>,
+        return cudaFuncSetAttribute(ffn_tc_decode_kernel<BITS, SMODE, BN, FP4>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kDSmemMax);
     }
     static cudaError_t run(const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t st) {
         const int smem = 1024 + kDBMax + kDBarBytes + a.ring * TcdCfg<BITS, SMODE, BN>::kPacked +
                          a.sring * a.stage_bytes;
-        ffn_tc_decode_kernel<BITS, SMODE, BN><<<grid, kDThreads, smem, st>>>(map, a);
+        ffn_tc_decode_kernel<BITS, SMODE, BN, FP4><<<grid, kDThreads, smem, st>>>(map, a);
         return cudaGetLastError();
     }
 };
 
-template <int BITS, int SMODE>
+template <int BITS, int SMODE, bool FP4>
 cudaError_t prepare_mode() {
-    cudaError_t e = LaunchD<BITS, SMODE, 16>::prepare();
-    if (e == cudaSuccess) e = LaunchD<BITS, SMODE, 32>::prepare();
+    cudaError_t e = LaunchD<BITS, SMODE, 16, FP4>::prepare();
+    if (e == cudaSuccess) e = LaunchD<BITS, SMODE, 32, FP4>::prepare();
     return e;
 }
 
-template <int BITS, int SMODE>
+template <int BITS, int SMODE, bool FP4>
 cudaError_t run_mode(int bn, const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t st) {
-    return bn <= 16 ? LaunchD<BITS, SMODE, 16>::run(map, a, grid, st) : LaunchD<BITS, SMODE, 32>::run(map, a, grid, st);
+    return bn <= 16 ? LaunchD<BITS, SMODE, 16, FP4>::run(map, a, grid, st) : LaunchD<BITS, SMODE, 32, FP4>::run(map, a, grid, st);
 }
 
-template <int BITS>
+template <int BITS, bool FP4>
 cudaError_t run_bits(int smode, int bn, const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t st) {
     switch (smode) {
-        case 0: return run_mode<BITS, 0>(bn, map, a, grid, st);
-        case 1: return run_mode<BITS, 1>(bn, map, a, grid, st);
-        case 2: return run_mode<BITS, 2>(bn, map, a, grid, st);
-        default: return run_mode<BITS, 4>(bn, map, a, grid, st);
+        case 0: return run_mode<BITS, 0, FP4>(bn, map, a, grid, st);
+        case 1: return run_mode<BITS, 1, FP4>(bn, map, a, grid, st);
+        case 2: return run_mode<BITS, 2, FP4>(bn, map, a, grid, st);
+        default: return run_mode<BITS, 4, FP4>(bn, map, a, grid, st);
     }
 }
 
@@ -543,14 +546,15 @@ int smode_of(int block_size) {
 
 cudaError_t prepare_ffn_tc_decode() {
     cudaError_t e = cudaSuccess;
-    if (e == cudaSuccess) e = prepare_mode<4, 0>();
-    if (e == cudaSuccess) e = prepare_mode<4, 1>();
-    if (e == cudaSuccess) e = prepare_mode<4, 2>();
-    if (e == cudaSuccess) e = prepare_mode<4, 4>();
-    if (e == cudaSuccess) e = prepare_mode<8, 0>();
-    if (e == cudaSuccess) e = prepare_mode<8, 1>();
-    if (e == cudaSuccess) e = prepare_mode<8, 2>();
-    if (e == cudaSuccess) e = prepare_mode<8, 4>();
+    if (e == cudaSuccess) e = prepare_mode<4, 0, false>();
+    if (e == cudaSuccess) e = prepare_mode<4, 1, false>();
+    if (e == cudaSuccess) e = prepare_mode<4, 2, false>();
+    if (e == cudaSuccess) e = prepare_mode<4, 4, false>();
+    if (e == cudaSuccess) e = prepare_mode<8, 0, false>();
+    if (e == cudaSuccess) e = prepare_mode<8, 1, false>();
+    if (e == cudaSuccess) e = prepare_mode<8, 2, false>();
+    if (e == cudaSuccess) e = prepare_mode<8, 4, false>();
+    if (e == cudaSuccess) e = prepare_mode<4, 4, true>();  // MXFP4 (block 32: four blocks per stage)
     return e;
 }
 
@@ -614,7 +618,8 @@ cudaError_t launch_ffn_tc_decode(const FfnArgs& f, int bn, int32_t* status, cuda
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return f.bits == 4 ? run_bits<4>(smode, bn, map, a, sms, st) : run_bits<8>(smode, bn, map, a, sms, st);
+    if (f.fp4) return run_mode<4, 4, true>(bn, map, a, sms, st);  // block 32
+    return f.bits == 4 ? run_bits<4, false>(smode, bn, map, a, sms, st) : run_bits<8, false>(smode, bn, map, a, sms, st);
 }
 
 }  // namespace qmoe

@@ -23,6 +23,7 @@
 // workspace status word; every role leaves its loop and the CTA frees TMEM).
 #include "qmoe_internal.cuh"
 #include "tc_common.cuh"
+#include "fp4_decode.cuh"
 
 namespace qmoe {
 namespace {
@@ -56,7 +57,7 @@ struct WideCfg {
     static_assert(kStages >= 3 && kSmem <= 227 * 1024, "shared-memory budget");
 };
 
-template <int BITS, bool PERCOL>
+template <int BITS, bool PERCOL, bool FP4>
 __global__ void __launch_bounds__(kWThreads, 1)
     ffn_tc_wide_kernel(const __grid_constant__ CUtensorMap bmap, const TcArgs a) {
     using C = WideCfg<BITS>;
@@ -227,7 +228,9 @@ __global__ void __launch_bounds__(kWThreads, 1)
 #pragma unroll
                     for (int j = 0; j < KSTEPS; ++j) {
                         uint32_t A[4];  // (r0, k 0-1), (r0+8, k 0-1), (r0, k 2-3), (r0+8, k 2-3)
-                        if (BITS == 4) {
+                        if (BITS == 4 && FP4) {
+                            decode_fp4x8(wv[j], A);  // MXFP4: e2m1 values, no zero point
+                        } else if (BITS == 4) {
                             A[0] = bf2_sub((wv[j] & kMask) | kMagic, kBias4);
                             A[1] = bf2_sub(((wv[j] >> 4) & kMask) | kMagic, kBias4);
                             A[2] = bf2_sub(((wv[j] >> 8) & kMask) | kMagic, kBias4);
@@ -306,19 +309,20 @@ __global__ void __launch_bounds__(kWThreads, 1)
     }
 }
 
-template <int BITS, bool PERCOL>
+template <int BITS, bool PERCOL, bool FP4>
 cudaError_t prepare_one() {
-    return cudaFuncSetAttribute(ffn_tc_wide_kernel<BITS, PERCOL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(ffn_tc_wide_kernel<BITS, PERCOL, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 WideCfg<BITS>::kSmem);
 }
 
 }  // namespace
 
 cudaError_t prepare_ffn_tc_wide() {
-    cudaError_t e = prepare_one<4, false>();
-    if (e == cudaSuccess) e = prepare_one<4, true>();
-    if (e == cudaSuccess) e = prepare_one<8, false>();
-    if (e == cudaSuccess) e = prepare_one<8, true>();
+    cudaError_t e = prepare_one<4, false, false>();
+    if (e == cudaSuccess) e = prepare_one<4, true, false>();
+    if (e == cudaSuccess) e = prepare_one<8, false, false>();
+    if (e == cudaSuccess) e = prepare_one<8, true, false>();
+    if (e == cudaSuccess) e = prepare_one<4, false, true>();  // MXFP4
     return e;
 }
 
@@ -361,8 +365,10 @@ cudaError_t launch_ffn_tc_wide(const FfnArgs& f, int bn, int32_t* status, cudaSt
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const bool percol = f.block_size == 0;
     void (*kern)(const CUtensorMap, const TcArgs) =
-        f.bits == 4 ? (percol ? ffn_tc_wide_kernel<4, true> : ffn_tc_wide_kernel<4, false>)
-                    : (percol ? ffn_tc_wide_kernel<8, true> : ffn_tc_wide_kernel<8, false>);
+        f.bits == 4 ? (f.fp4    ? ffn_tc_wide_kernel<4, false, true>
+                       : percol ? ffn_tc_wide_kernel<4, true, false>
+                                : ffn_tc_wide_kernel<4, false, false>)
+                    : (percol ? ffn_tc_wide_kernel<8, true, false> : ffn_tc_wide_kernel<8, false, false>);
     const int smem = f.bits == 4 ? WideCfg<4>::kSmem : WideCfg<8>::kSmem;
     kern<<<sms, kWThreads, smem, st>>>(map, a);
     return cudaGetLastError();

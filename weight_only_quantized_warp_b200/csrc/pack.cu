@@ -126,7 +126,12 @@ __global__ void pack_scales_kernel(PackArgs a) {
         }
         const SrcRow s = source_row(a.mode, rt, rr, a.I);
         const int64_t src_idx = (e * src_rows + s.row) * nsb + b;
-        if (a.scale_bf16) {
+        if (a.scale_e8m0) {
+            // E8M0 byte x is 2^(x - 127): the bf16 with exponent field x and an
+            // empty mantissa, bit for bit (x = 0 gives 2^-127 as a subnormal)
+            const uint8_t x = ((const uint8_t*)(s.which ? a.s_src_up : a.s_src))[src_idx];
+            ((uint16_t*)a.s_dst)[id] = x == 0 ? uint16_t(0x0040) : uint16_t(uint16_t(x) << 7);
+        } else if (a.scale_bf16) {
             const uint16_t* src = (const uint16_t*)(s.which ? a.s_src_up : a.s_src);
             ((uint16_t*)a.s_dst)[id] = src[src_idx];
         } else {

@@ -155,10 +155,18 @@ qmoe_status validate(const qmoe_config& c, std::string& why) {
     const bool gated = c.swiglu_fusion != 0 || c.has_fc3;
     if (!gated && c.activation_type == QMOE_ACT_SWIGLU)
         return bad(QMOE_INVALID_ARGUMENT, "swiglu needs a gate and an up projection (fusion 1/2 or fc3)");
-    if ((c.act_dtype != QMOE_DTYPE_F32 && c.act_dtype != QMOE_DTYPE_BF16) ||
-        (c.scale_dtype != QMOE_DTYPE_F32 && c.scale_dtype != QMOE_DTYPE_BF16))
+    if (c.weight_format != QMOE_WEIGHTS_INT && c.weight_format != QMOE_WEIGHTS_MXFP4)
+        return bad(QMOE_INVALID_ARGUMENT, "weight_format must be INT or MXFP4");
+    if (c.weight_format == QMOE_WEIGHTS_MXFP4) {
+        if (c.expert_weight_bits != 4 || c.block_size != 32 || c.scale_dtype != QMOE_DTYPE_E8M0)
+            return bad(QMOE_INVALID_ARGUMENT, "MXFP4 needs 4-bit codes, block_size 32 and E8M0 scales");
+        if (c.act_dtype != QMOE_DTYPE_F32 && c.act_dtype != QMOE_DTYPE_BF16)
+            return bad(QMOE_INVALID_ARGUMENT, "act_dtype must be F32 or BF16");
+    } else if ((c.act_dtype != QMOE_DTYPE_F32 && c.act_dtype != QMOE_DTYPE_BF16) ||
+               (c.scale_dtype != QMOE_DTYPE_F32 && c.scale_dtype != QMOE_DTYPE_BF16)) {
         return bad(QMOE_INVALID_ARGUMENT, "act_dtype and scale_dtype must be F32 or BF16");
-    if (c.reserved != 0) return bad(QMOE_INVALID_ARGUMENT, "reserved must be 0");
+    }
+    if (c.reserved != 0 || c.reserved2 != 0) return bad(QMOE_INVALID_ARGUMENT, "reserved fields must be 0");
     if (c.use_sparse_mixer) return bad(QMOE_UNSUPPORTED, "use_sparse_mixer is not built");
     if (c.num_experts > 256) return bad(QMOE_UNSUPPORTED, "num_experts > 256 is not built");
     if (c.hidden_size % 64 || c.inter_size % 64) {
@@ -271,7 +279,8 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
 
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size, N1 = h->n1;
     const int bits = c.expert_weight_bits, bs = c.block_size;
-    const size_t ssz = c.scale_dtype == QMOE_DTYPE_BF16 ? 2 : 4;
+    // packed scales: bf16 or fp32 as given; E8M0 bytes widen to bf16 (exact)
+    const size_t ssz = c.scale_dtype == QMOE_DTYPE_F32 ? 4 : 2;
     const int64_t nsb1 = bs ? H / bs : 1, nsb2 = bs ? I / bs : 1;
     const bool any_b1 = c.has_fc1_bias || c.has_fc3_bias;
 
@@ -308,7 +317,8 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
     p1.bits = bits;
     p1.block_size = bs;
     p1.mode = c.has_fc3 ? 3 : c.swiglu_fusion;  // 0 identity, 1 interleaved, 2 concatenated
-    p1.scale_bf16 = c.scale_dtype == QMOE_DTYPE_BF16;
+    p1.scale_bf16 = c.scale_dtype != QMOE_DTYPE_F32;
+    p1.scale_e8m0 = c.scale_dtype == QMOE_DTYPE_E8M0;
     p1.act_bf16 = c.act_dtype == QMOE_DTYPE_BF16;
     PackArgs p2 = p1;
     p2.src = (const uint8_t*)fc2_w;
@@ -455,7 +465,8 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     f1.beta = c.activation_beta;
     f1.limit = resolved_limit(c.swiglu_limit);
     f1.splits = 1;
-    f1.scale_bf16 = c.scale_dtype == QMOE_DTYPE_BF16;
+    f1.scale_bf16 = c.scale_dtype != QMOE_DTYPE_F32;
+    f1.fp4 = c.weight_format == QMOE_WEIGHTS_MXFP4;
     f1.act_bf16 = bf16;
     f1.nt = p.nt;
     FfnArgs f2 = f1;

@@ -107,6 +107,7 @@ struct PackArgs {
     int64_t I;               // gated modes: inter size
     int bits, block_size, mode;
     int scale_bf16, act_bf16;
+    int scale_e8m0;          // source scales are E8M0 bytes, packed as bf16
 };
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t st);
 
@@ -142,6 +143,7 @@ struct FfnArgs {
     int splits;
     int scale_bf16, act_bf16;
     int nt;
+    int fp4;                 // codes are MXFP4 e2m1 (no zero point)
 };
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
 // Shared memory of one decode CTA (staged activation rows) and its limit;

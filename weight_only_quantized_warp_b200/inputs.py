@@ -29,7 +29,8 @@ from typing import Optional
 import numpy as np
 
 ACT_RELU, ACT_GELU, ACT_SILU, ACT_SWIGLU, ACT_IDENTITY = 0, 1, 2, 3, 4
-DT_F32, DT_BF16 = 0, 1
+DT_F32, DT_BF16, DT_E8M0 = 0, 1, 2
+WEIGHTS_INT, WEIGHTS_MXFP4 = 0, 1
 ACT_NAMES = {"relu": ACT_RELU, "gelu": ACT_GELU, "silu": ACT_SILU,
              "swiglu": ACT_SWIGLU, "identity": ACT_IDENTITY}
 
@@ -75,6 +76,8 @@ class MoEConfig:
     topk_group: int = 0
     routed_scaling_factor: float = 1.0
     apply_router_weight_on_input: bool = False
+    # WEIGHTS_MXFP4: e2m1 codes with one E8M0 scale byte per 32 codes
+    weight_format: int = WEIGHTS_INT
 
     @property
     def gated(self) -> bool:
@@ -114,6 +117,11 @@ def _weights(rng, E, N, K, bits):
 
 def _scales(rng, cfg: MoEConfig, E, N, K, exact_range: bool):
     shape = (E, N, K // cfg.block_size) if cfg.block_size > 0 else (E, N)
+    if cfg.weight_format == WEIGHTS_MXFP4:
+        # E8M0 exponent bytes around 0.05 * sqrt(64 / K) / 2 (e2m1 magnitudes
+        # average about 2), spread over four powers of two
+        centre = 127 + int(round(math.log2(0.025 * math.sqrt(64.0 / K))))
+        return rng.integers(centre - 2, centre + 2, size=shape, dtype=np.int64).astype(np.uint8)
     s = rng.uniform(0.01, 0.05, size=shape)
     if not exact_range:
         # keep activations O(1): sqrt(64/K) for the reduction length and
@@ -220,6 +228,16 @@ def gpt_oss(T: int = 1024):
     return cfg, 3, dict(logits="normal", logit_std=1.0)
 
 
+def gpt_oss_mxfp4(T: int = 1024):
+    """The gpt-oss-like shape with MXFP4 expert weights (e2m1 codes, one E8M0
+    scale per 32), the checkpoint format the QMoEWoQ page names."""
+    cfg = MoEConfig(T=T, H=2880, I=2880, E=32, k=4, bits=4, block_size=32,
+                    act=ACT_SWIGLU, fusion=1, alpha=1.702, beta=1.0, limit=7.0,
+                    normalize=True, act_dtype=DT_BF16, scale_dtype=DT_E8M0,
+                    has_fc1_bias=True, has_fc2_bias=True, weight_format=WEIGHTS_MXFP4)
+    return cfg, 5, dict(logits="normal", logit_std=1.0)
+
+
 def deepseek(T: int = 4096):
     cfg = MoEConfig(T=T, H=2048, I=1408, E=64, k=6, bits=8, block_size=0,
                     act=ACT_SILU, fusion=0, has_fc3=True, normalize=False,
@@ -243,6 +261,7 @@ WORKLOADS = {
     "tiny": tiny,
     "mixtral_decode": mixtral_decode,
     "gpt_oss": gpt_oss,
+    "gpt_oss_mxfp4": gpt_oss_mxfp4,
     "deepseek": deepseek,
 }
 

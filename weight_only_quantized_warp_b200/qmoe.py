@@ -27,7 +27,8 @@ lib = ctypes.CDLL(LIB_PATH)
 QMOE_OK, QMOE_INVALID_ARGUMENT, QMOE_NOT_BOUND, QMOE_UNSUPPORTED = 0, 1, 2, 3
 QMOE_CUDA_ERROR, QMOE_TIMEOUT, QMOE_OUT_OF_MEMORY = 4, 5, 6
 ACT_RELU, ACT_GELU, ACT_SILU, ACT_SWIGLU, ACT_IDENTITY = 0, 1, 2, 3, 4
-DTYPE_F32, DTYPE_BF16 = 0, 1
+DTYPE_F32, DTYPE_BF16, DTYPE_E8M0 = 0, 1, 2
+WEIGHTS_INT, WEIGHTS_MXFP4 = 0, 1
 PATH_SIMT, PATH_DECODE, PATH_TC, PATH_TC_DECODE = 0, 1, 2, 3
 
 # Every function the header declares (checked against include/qmoe.h by the tests).
@@ -52,7 +53,8 @@ class qmoe_config(ctypes.Structure):
                 ("has_fc3", ctypes.c_int32), ("has_fc3_bias", ctypes.c_int32),
                 ("use_sparse_mixer", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
-                ("routed_scaling_factor", ctypes.c_float), ("apply_router_weight_on_input", ctypes.c_int32)]
+                ("routed_scaling_factor", ctypes.c_float), ("apply_router_weight_on_input", ctypes.c_int32),
+                ("weight_format", ctypes.c_int32), ("reserved2", ctypes.c_int32)]
 
 
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
@@ -141,7 +143,8 @@ def make_config(cfg) -> qmoe_config:
         has_fc3_bias=int(cfg.has_fc3_bias), use_sparse_mixer=0, reserved=0,
         n_group=int(getattr(cfg, "n_group", 0)), topk_group=int(getattr(cfg, "topk_group", 0)),
         routed_scaling_factor=float(getattr(cfg, "routed_scaling_factor", 1.0)),
-        apply_router_weight_on_input=int(getattr(cfg, "apply_router_weight_on_input", False)))
+        apply_router_weight_on_input=int(getattr(cfg, "apply_router_weight_on_input", False)),
+        weight_format=int(getattr(cfg, "weight_format", 0)), reserved2=0)
 
 
 def qmoe_create(cfg: qmoe_config) -> int:
