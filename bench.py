@@ -81,7 +81,7 @@ def algorithmic(cfg, offsets):
     with at least one routed row count once)."""
     counts = np.diff(offsets)
     touched = int((counts > 0).sum())
-    ssz = 2 if cfg.scale_dtype == gen.DT_BF16 else 4
+    ssz = {gen.DT_F32: 4, gen.DT_BF16: 2, gen.DT_E8M0: 1}[cfg.scale_dtype]
     asz = 2 if cfg.act_dtype == gen.DT_BF16 else 4
     n1 = cfg.n1 + (cfg.I if cfg.has_fc3 else 0)
     nsb1 = cfg.H // cfg.block_size if cfg.block_size else 1
