@@ -227,11 +227,11 @@ def run_ours(args):
     from weight_only_quantized_warp_b200 import qmoe, replicas
 
     world, rank, local = dist_env()
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     # every replica: the same weights, its own token batch
     inp = replicas.replica_inputs(args.workload, rank)
@@ -284,7 +284,7 @@ def run_ours(args):
     clocks.start()
     keep_loaded(0.6)
     if world > 1:
-        dist.barrier()
+        dist.barrier(device_ids=[local])
     torch.cuda.synchronize()
     start.record(stream)
     for i in range(K):
@@ -297,7 +297,7 @@ def run_ours(args):
         clk["window"] = "timed region bracketed by 0.6 s / 0.4 s of the same forward"
     ms = replicas.max_over_ranks([start.elapsed_time(stop)], dev)[0]
     if world > 1:
-        dist.barrier()
+        dist.barrier(device_ids=[local])
     per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(launches)]
                            for i in range(K)]).mean(axis=0)
     path = qmoe.qmoe_path_for(h, T)
@@ -326,7 +326,7 @@ def run_ours(args):
         e2e_step()
     torch.cuda.synchronize()
     if world > 1:
-        dist.barrier()
+        dist.barrier(device_ids=[local])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(K):
