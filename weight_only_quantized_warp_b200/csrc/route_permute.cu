@@ -228,9 +228,58 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
     permute_block(topk_idx, T, E, k, offsets, perm_tok, inv, sm);
 }
 
+// The permutation by one warp (few routed pairs): histogram and scan in
+// shared memory, then the pairs in order, 32 at a time; lanes holding the
+// same expert find each other with a match and take consecutive slots after
+// the expert's running base, so a segment keeps token order.
+__device__ __forceinline__ void permute_warp(const int32_t* __restrict__ topk_idx, int64_t T, int E, int k,
+                                             int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok,
+                                             int32_t* __restrict__ inv, int32_t* cnt, int32_t* base, int lane) {
+    const int R = int(T) * k;
+    for (int e = lane; e < E; e += 32) cnt[e] = 0;
+    __syncwarp();
+    for (int r = lane; r < R; r += 32) atomicAdd(&cnt[topk_idx[r]], 1);
+    __syncwarp();
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const int v = e < E ? cnt[e] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        if (e < E) {
+            offsets[e] = carry + incl - v;
+            base[e] = carry + incl - v;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) offsets[E] = carry;
+    __syncwarp();
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int r0 = 0; r0 < R; r0 += 32) {
+        const int r = r0 + lane;
+        const uint32_t act = __ballot_sync(0xffffffffu, r < R);
+        if (r < R) {
+            const int e = topk_idx[r];
+            const uint32_t same = __match_any_sync(act, e);
+            const int rank = __popc(same & lt);
+            const int pos = base[e] + rank;
+            perm_tok[pos] = r / k;
+            inv[r] = pos;
+            __syncwarp(act);  // every lane has read base[e] before it moves on
+            if (rank == 0) base[e] += __popc(same);
+        }
+        __syncwarp();
+    }
+}
+
 // Few tokens: one CTA routes them (a warp per token) and, after a barrier
-// that makes the top-k lists visible to the whole block, permutes them; one
-// launch instead of two. Thread 0 clears the workspace status word first.
+// that makes the top-k lists visible to the whole block, one warp permutes
+// them; one launch instead of two. Thread 0 clears the workspace status word
+// first.
 __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
     const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int n_group, int topk_group,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int32_t* __restrict__ offsets,
@@ -241,7 +290,10 @@ __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
     for (int64_t t = warp; t < T; t += kWarps)
         route_token(logits, act_bf16, t, E, k, normalize, n_group, topk_group, topk_idx, topk_w, lane);
     __syncthreads();
-    permute_block(topk_idx, T, E, k, offsets, perm_tok, inv, sm);
+    if (warp == 0) {
+        int32_t* cnt = reinterpret_cast<int32_t*>(sm);
+        permute_warp(topk_idx, T, E, k, offsets, perm_tok, inv, cnt, cnt + E, lane);
+    }
 }
 
 }  // namespace
