@@ -62,6 +62,8 @@ CASES = {
     "e64_k6": dict(T=40, E=64, k=6, bits=8, block_size=0, fusion=0, has_fc3=True,
                    act=gen.ACT_SILU, normalize=False),
     "k_equals_E": dict(T=9, E=4, k=4),
+    "e256_k8": dict(T=20, E=256, k=8, H=128, I=128, block_size=64),
+    "one_expert": dict(T=7, E=1, k=1, normalize=False),
     "t1": dict(T=1),
     # shapes the streaming tensor-core kernels take (H, I multiples of 128)
     "k128_int4_bs32_bias": dict(H=256, I=384, block_size=32, fusion=1, has_fc1_bias=True, has_fc2_bias=True),
