@@ -8,5 +8,5 @@ shares no code with the CUDA path and imports nothing from it.
 header for the passages it follows). ``literal.py`` restates the whole
 forward a second time in the most literal numpy, for tiny shapes.
 """
-from .binding import (dequant, e2m1, forward, gated_act, num_threads, permute, plain_act,  # noqa: F401
-                      route, to_f64, unpack)
+from .binding import (dequant, e2m1, forward, gated_act, linear_i8, num_threads, permute,  # noqa: F401
+                      plain_act, quantize_i8, round_act, route, to_f64, unpack)

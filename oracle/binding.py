@@ -31,7 +31,8 @@ class _Cfg(ctypes.Structure):
                 ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
                 ("apply_router_weight_on_input", ctypes.c_int32),
                 ("routed_scaling_factor", ctypes.c_double),
-                ("mxfp4", ctypes.c_int32)]
+                ("mxfp4", ctypes.c_int32), ("act_bf16", ctypes.c_int32),
+                ("int8_block", ctypes.c_int32)]
 
 
 def _load():
@@ -47,6 +48,8 @@ def _load():
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_e2m1.restype = ctypes.c_double
         lib.oracle_e2m1.argtypes = [ctypes.c_int32]
+        lib.oracle_round_act.restype = ctypes.c_double
+        lib.oracle_round_act.argtypes = [ctypes.c_double, ctypes.c_int32]
         _lib = lib
     return _lib
 
@@ -121,6 +124,44 @@ def e2m1(code: int) -> float:
     return float(_load().oracle_e2m1(code))
 
 
+def round_act(v: float, bf16: bool) -> float:
+    """Round one value to the activation dtype (nearest, ties to even)."""
+    return float(_load().oracle_round_act(float(v), int(bf16)))
+
+
+def quantize_i8(x: np.ndarray, block_size: int):
+    """Per-block int8 rounding of activation rows (int8 block compute tier).
+
+    ``x`` [rows, K] (fp32 values or bf16 bit patterns). Returns the codes
+    [rows, K] int8 and the scales [rows, K / block_size] float32."""
+    v = to_f64(x)
+    rows, K = v.shape
+    q = np.empty((rows, K), dtype=np.int8)
+    s = np.empty((rows, K // block_size), dtype=np.float32)
+    lib = _load()
+    for r in range(rows):
+        lib.oracle_quantize_i8(_p(np.ascontiguousarray(v[r]), _f64p), ctypes.c_int64(K),
+                               ctypes.c_int64(block_size),
+                               q[r].ctypes.data_as(ctypes.POINTER(ctypes.c_int8)),
+                               s[r].ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return q, s
+
+
+def linear_i8(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, N: int, K: int, bits: int,
+              block_size: int) -> np.ndarray:
+    """The int8-tier dot of activation rows ``x`` [rows, K] (values as stored;
+    they are widened, not rounded) with the packed weight [N, K]: [rows, N] fp64."""
+    v = to_f64(x)
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    s = to_f64(scales)
+    rows = v.shape[0]
+    y = np.empty((rows, N), dtype=np.float64)
+    _load().oracle_linear_i8(_p(v, _f64p), ctypes.c_int64(rows), _p(packed, _u8p), _p(s, _f64p),
+                             ctypes.c_int64(N), ctypes.c_int64(K), ctypes.c_int32(bits),
+                             ctypes.c_int64(block_size), _p(y, _f64p))
+    return y
+
+
 def gated_act(act: int, g: float, u: float, alpha: float, beta: float, limit: float) -> float:
     return float(_load().oracle_gated_act(act, g, u, alpha, beta, limit))
 
@@ -154,7 +195,9 @@ def forward(inp, tokens: Optional[Sequence[int]] = None, want_h: bool = False) -
                n_group=int(c.n_group), topk_group=int(c.topk_group),
                apply_router_weight_on_input=int(c.apply_router_weight_on_input),
                routed_scaling_factor=float(c.routed_scaling_factor) if c.routed_scaling_factor else 1.0,
-               mxfp4=int(c.weight_format == 1))
+               mxfp4=int(c.weight_format == 1),
+               act_bf16=int(np.asarray(inp.x).dtype == np.uint16),
+               int8_block=int(getattr(c, "compute_mode", 0) == 1))
     y = np.empty((T, c.H), dtype=np.float64)
     idx = np.empty((T, c.k), dtype=np.int32)
     w = np.empty((T, c.k), dtype=np.float64)

@@ -51,6 +51,17 @@
  * with one E8M0 scale 2^(x - 127) per 32 codes along K (the scales arrive
  * here already as fp64 values).
  *
+ * Int8 block compute tier ("ClikaRT::nn::QMoEWoQ" page, class description:
+ * a packed block weight on the int8 tier rounds the activation to per-block
+ * int8 before the dot). The pages give no rounding rule; read as symmetric
+ * absmax rounding over the weight's own K blocks, decided in fp32:
+ *   s = absmax(block) / 127, q = clamp(rint(v / s), -127, 127), ties to even
+ *   (s = 0 and q = 0 for an all-zero block);
+ *   dot = sum_b s_w[n, b] * s[b] * sum_{k in b} (q_w[n, k] - 2^(bits-1)) * q[k].
+ * The expert's input row is the activation as stored (the router-weighted row
+ * rounded to the activation dtype when the weight scales the input), and
+ * FC2's input is h rounded to the activation dtype.
+ *
  * Every sum is a serial fp64 loop in index order, so the result does not
  * depend on the thread count.
  */
@@ -78,6 +89,8 @@ typedef struct oracle_cfg {
     int32_t apply_router_weight_on_input;
     double routed_scaling_factor;
     int32_t mxfp4;                       /* codes are e2m1, no zero point */
+    int32_t act_bf16;                    /* activation dtype: 1 bf16, 0 fp32 */
+    int32_t int8_block;                  /* int8 block compute tier */
 } oracle_cfg;
 
 int oracle_num_threads(void) {
@@ -223,6 +236,69 @@ double oracle_gated_act(int32_t act, double g, double u, double alpha, double be
 
 double oracle_plain_act(int32_t act, double a) { return plain_act(act, a); }
 
+/* Round to the activation dtype, to nearest with ties to even: fp32 by the
+ * C conversion; bf16 (8 significant bits, fp32's exponent range) by scaling
+ * the value so that its last kept bit is the unit and rounding to an integer
+ * (exact in fp64). */
+double oracle_round_act(double v, int32_t bf16) {
+    if (!bf16) return (double)(float)v;
+    if (v == 0.0 || !isfinite(v)) return v;
+    int ex;
+    frexp(v, &ex);                     /* |v| in [2^(ex-1), 2^ex) */
+    int lsb = ex - 8;                  /* exponent of the last kept bit */
+    if (lsb < -133) lsb = -133;        /* subnormal spacing of bf16 */
+    return ldexp(nearbyint(ldexp(v, -lsb)), lsb);
+}
+
+/* Per-block int8 rounding of one activation row of K values (int8 tier, see
+ * the header): q[K] codes, s[K / bs] scales. All decisions in fp32. */
+void oracle_quantize_i8(const double* v, int64_t K, int64_t bs, int8_t* q, float* s) {
+    for (int64_t b = 0; b < K / bs; ++b) {
+        float amax = 0.0f;
+        for (int64_t k = b * bs; k < (b + 1) * bs; ++k) {
+            const float a = fabsf((float)v[k]);
+            if (a > amax) amax = a;
+        }
+        const float sc = amax / 127.0f;
+        s[b] = sc;
+        for (int64_t k = b * bs; k < (b + 1) * bs; ++k) {
+            float r = sc > 0.0f ? rintf((float)v[k] / sc) : 0.0f;
+            if (r > 127.0f) r = 127.0f;
+            if (r < -127.0f) r = -127.0f;
+            q[k] = (int8_t)r;
+        }
+    }
+}
+
+/* One output of the int8 tier: sum over the K blocks of
+ * s_w * s_x * (exact integer dot of centred weight codes and activation codes). */
+static double dot_i8(const uint8_t* packed, const double* scales, int64_t K, int bits, int64_t bs,
+                     int64_t n, const int8_t* q, const float* s) {
+    const int32_t z = 1 << (bits - 1);
+    double acc = 0.0;
+    for (int64_t b = 0; b < K / bs; ++b) {
+        int64_t d = 0;
+        for (int64_t k = b * bs; k < (b + 1) * bs; ++k)
+            d += (int64_t)(code_at(packed, K, bits, n, k) - z) * (int64_t)q[k];
+        acc += scales[n * (K / bs) + b] * (double)s[b] * (double)d;
+    }
+    return acc;
+}
+
+/* y[r, n] = the int8-tier dot of activation row r with weight row n, for
+ * rows x[rows, K] (no bias). */
+void oracle_linear_i8(const double* x, int64_t rows, const uint8_t* packed, const double* scales,
+                      int64_t N, int64_t K, int32_t bits, int64_t bs, double* y) {
+    int8_t* q = (int8_t*)malloc((size_t)K);
+    float* s = (float*)malloc(sizeof(float) * (size_t)(K / bs));
+    for (int64_t r = 0; r < rows; ++r) {
+        oracle_quantize_i8(x + r * K, K, bs, q, s);
+        for (int64_t n = 0; n < N; ++n) y[r * N + n] = dot_i8(packed, scales, K, bits, bs, n, q, s);
+    }
+    free(q);
+    free(s);
+}
+
 /*
  * The whole forward. Float inputs arrive as fp64 arrays holding the stored
  * values exactly. Outputs: y[T,H] (fp64, unrounded), topk_idx[T,k],
@@ -263,6 +339,22 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
         /* FC1 (and FC3): a[r, n] = sum_k x[t, k] * W[n, k] + b[n] */
         const uint8_t* w1 = fc1_w + e * N1 * pk1;
         const double* s1 = fc1_s + e * N1 * sc1;
+        /* int8 tier: the expert's input rows rounded per block to int8 */
+        int8_t* q1 = NULL;
+        float* qs1 = NULL;
+        if (c->int8_block) {
+            q1 = (int8_t*)malloc((size_t)(m * H));
+            qs1 = (float*)malloc(sizeof(float) * (size_t)(m * sc1));
+            double* v = (double*)malloc(sizeof(double) * (size_t)H);
+            if (!q1 || !qs1 || !v) return -1;
+            for (int64_t i = 0; i < m; ++i) {
+                const int64_t r = rows[i], t = r / k;
+                const double win = c->apply_router_weight_on_input ? topk_w[r] : 1.0;
+                for (int64_t kk = 0; kk < H; ++kk) v[kk] = oracle_round_act(win * x[t * H + kk], c->act_bf16);
+                oracle_quantize_i8(v, H, bs, q1 + i * H, qs1 + i * sc1);
+            }
+            free(v);
+        }
 #pragma omp parallel
         {
             double* wrow = (double*)malloc(sizeof(double) * (size_t)H);
@@ -274,7 +366,10 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
                     /* the expert's input row: x[t], or w[r] * x[t] */
                     const double win = c->apply_router_weight_on_input ? topk_w[r] : 1.0;
                     double acc = 0.0;
-                    for (int64_t kk = 0; kk < H; ++kk) acc += (win * x[t * H + kk]) * wrow[kk];
+                    if (c->int8_block)
+                        acc = dot_i8(w1, s1, H, bits, bs, n, q1 + i * H, qs1 + i * sc1);
+                    else
+                        for (int64_t kk = 0; kk < H; ++kk) acc += (win * x[t * H + kk]) * wrow[kk];
                     if (fc1_b) acc += fc1_b[e * N1 + n];
                     a1[r * N1 + n] = acc;
                 }
@@ -289,7 +384,10 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
                         const int64_t r = rows[i], t = r / k;
                         const double win = c->apply_router_weight_on_input ? topk_w[r] : 1.0;
                         double acc = 0.0;
-                        for (int64_t kk = 0; kk < H; ++kk) acc += (win * x[t * H + kk]) * wrow[kk];
+                        if (c->int8_block)
+                            acc = dot_i8(w3, s3, H, bits, bs, n, q1 + i * H, qs1 + i * sc1);
+                        else
+                            for (int64_t kk = 0; kk < H; ++kk) acc += (win * x[t * H + kk]) * wrow[kk];
                         if (fc3_b) acc += fc3_b[e * I + n];
                         a3[r * I + n] = acc;
                     }
@@ -323,9 +421,26 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
             }
         }
 
+        free(q1);
+        free(qs1);
+
         /* FC2: o[r, m] = sum_i h[r, i] * W2[m, i] + b2[m] */
         const uint8_t* w2 = fc2_w + e * H * pk2;
         const double* s2 = fc2_s + e * H * sc2;
+        /* int8 tier: h rounded to the activation dtype, then per block to int8 */
+        int8_t* q2 = NULL;
+        float* qs2 = NULL;
+        if (c->int8_block) {
+            q2 = (int8_t*)malloc((size_t)(m * I));
+            qs2 = (float*)malloc(sizeof(float) * (size_t)(m * sc2));
+            double* v = (double*)malloc(sizeof(double) * (size_t)I);
+            if (!q2 || !qs2 || !v) return -1;
+            for (int64_t i = 0; i < m; ++i) {
+                for (int64_t kk = 0; kk < I; ++kk) v[kk] = oracle_round_act(h[rows[i] * I + kk], c->act_bf16);
+                oracle_quantize_i8(v, I, bs, q2 + i * I, qs2 + i * sc2);
+            }
+            free(v);
+        }
 #pragma omp parallel
         {
             double* wrow = (double*)malloc(sizeof(double) * (size_t)I);
@@ -335,13 +450,18 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
                 for (int64_t i = 0; i < m; ++i) {
                     const int64_t r = rows[i];
                     double acc = 0.0;
-                    for (int64_t kk = 0; kk < I; ++kk) acc += h[r * I + kk] * wrow[kk];
+                    if (c->int8_block)
+                        acc = dot_i8(w2, s2, I, bits, bs, n, q2 + i * I, qs2 + i * sc2);
+                    else
+                        for (int64_t kk = 0; kk < I; ++kk) acc += h[r * I + kk] * wrow[kk];
                     if (fc2_b) acc += fc2_b[e * H + n];
                     o[r * H + n] = acc;
                 }
             }
             free(wrow);
         }
+        free(q2);
+        free(qs2);
     }
 
     /* combine: y[t] = rsf * sum_j w[t, j] * o[t*k + j] + shared[t], j in list

@@ -31,6 +31,7 @@ import numpy as np
 ACT_RELU, ACT_GELU, ACT_SILU, ACT_SWIGLU, ACT_IDENTITY = 0, 1, 2, 3, 4
 DT_F32, DT_BF16, DT_E8M0 = 0, 1, 2
 WEIGHTS_INT, WEIGHTS_MXFP4 = 0, 1
+COMPUTE_FLOAT, COMPUTE_INT8_BLOCK = 0, 1
 ACT_NAMES = {"relu": ACT_RELU, "gelu": ACT_GELU, "silu": ACT_SILU,
              "swiglu": ACT_SWIGLU, "identity": ACT_IDENTITY}
 
@@ -78,6 +79,8 @@ class MoEConfig:
     apply_router_weight_on_input: bool = False
     # WEIGHTS_MXFP4: e2m1 codes with one E8M0 scale byte per 32 codes
     weight_format: int = WEIGHTS_INT
+    # COMPUTE_INT8_BLOCK: the activations are rounded per K block to int8
+    compute_mode: int = COMPUTE_FLOAT
 
     @property
     def gated(self) -> bool:
@@ -238,6 +241,13 @@ def gpt_oss_mxfp4(T: int = 1024):
     return cfg, 5, dict(logits="normal", logit_std=1.0)
 
 
+def mixtral_decode_i8(T: int = 8):
+    """The decode shape of mixtral_decode on the int8 block compute tier."""
+    cfg, seed, kw = mixtral_decode(T)
+    cfg.compute_mode = COMPUTE_INT8_BLOCK
+    return cfg, seed, kw
+
+
 def deepseek(T: int = 4096):
     cfg = MoEConfig(T=T, H=2048, I=1408, E=64, k=6, bits=8, block_size=0,
                     act=ACT_SILU, fusion=0, has_fc3=True, normalize=False,
@@ -260,6 +270,7 @@ def sweep(bits: int, T: int):
 WORKLOADS = {
     "tiny": tiny,
     "mixtral_decode": mixtral_decode,
+    "mixtral_decode_i8": mixtral_decode_i8,
     "gpt_oss": gpt_oss,
     "gpt_oss_mxfp4": gpt_oss_mxfp4,
     "deepseek": deepseek,
