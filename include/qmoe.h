@@ -83,6 +83,19 @@ enum { QMOE_DTYPE_F32 = 0, QMOE_DTYPE_BF16 = 1, QMOE_DTYPE_E8M0 = 2 };
  * stay floating point either way. */
 enum { QMOE_WEIGHTS_INT = 0, QMOE_WEIGHTS_MXFP4 = 1 };
 
+/* compute_mode ("ClikaRT::nn::QMoEWoQ" page, class description: a packed
+ * block weight on the int8 block tier rounds the activation to per-block int8
+ * before the dot; the pages give no rounding rule). FLOAT: the activations
+ * stay floating point. INT8_BLOCK: every expert input row -- x (or the
+ * router-weighted row, rounded to act_dtype) for FC1, h rounded to act_dtype
+ * for FC2 -- is cut into the weight's K blocks and rounded per block with
+ * s = absmax / 127 and q = clamp(rint(v / s), -127, 127), ties to even,
+ * decided in fp32 (s = 0, q = 0 for an all-zero block); each weight row then
+ * sums s_w * s * (integer dot of (code - zero point) and q) over its blocks.
+ * Requires weight_format INT and block_size >= 64 (4-bit codes) or >= 32
+ * (8-bit codes); runs on path 4 for every T and both act dtypes. */
+enum { QMOE_COMPUTE_FLOAT = 0, QMOE_COMPUTE_INT8_BLOCK = 1 };
+
 /*
  * Operator attributes ("QMoE" page attribute list; "ClikaRT::nn::QMoEWoQ",
  * make(): the four counts and the bias flags).
@@ -139,7 +152,7 @@ typedef struct qmoe_config {
     float routed_scaling_factor;
     int32_t apply_router_weight_on_input;
     int32_t weight_format;        /* QMOE_WEIGHTS_* */
-    int32_t reserved2;            /* must be 0 */
+    int32_t compute_mode;         /* QMOE_COMPUTE_* */
 } qmoe_config;
 
 typedef struct qmoe_handle qmoe_handle;
@@ -283,13 +296,27 @@ QMOE_API const char* qmoe_status_string(qmoe_status s);
  * the handle. */
 QMOE_API const char* qmoe_last_error(const qmoe_handle* h);
 
+/*
+ * qmoe_quantize_act_i8 -- the int8 block tier's activation rounding as a
+ * standalone operation (see compute_mode): rows x [rows, K] of dtype
+ * (QMOE_DTYPE_F32 or QMOE_DTYPE_BF16) to codes q [rows, K] int8 in k order
+ * and scales [rows, K / block_size] fp32, on `stream` (asynchronous). All
+ * pointers are DEVICE pointers owned by the caller; x 16-byte aligned, q and
+ * scales 4-byte aligned. block_size is a power of two >= 16 dividing K.
+ * rows == 0 is a no-op. QMOE_INVALID_ARGUMENT for a bad size, dtype or
+ * alignment; QMOE_CUDA_ERROR if the launch fails.
+ */
+QMOE_API qmoe_status qmoe_quantize_act_i8(const void* x, int32_t dtype, int64_t rows, int64_t K,
+                                          int32_t block_size, int8_t* q, float* scales, void* stream);
+
 /* Tunable options (qmoe_set_option). QMOE_OPT_PATH selects the expert-FFN
  * kernels for bf16 activations: -1 (default) chooses by shape, 1 forces the
  * weight-streaming mma.sync kernels, 2 the tcgen05 grouped GEMM, 3 the
  * tcgen05 streaming decode kernels (falls back to 1 for shapes they do not
  * cover: more than 32 rows per expert, K not a multiple of 128, or a K range
  * whose resident activations exceed 128 KB). fp32 activations always take
- * the fp32 path (0). */
+ * the fp32 path (0); compute_mode INT8_BLOCK always takes path 4 and ignores
+ * this option. */
 enum { QMOE_OPT_PATH = 1 };
 
 /* qmoe_set_option -- set a tunable option on the handle. QMOE_INVALID_ARGUMENT
@@ -299,12 +326,14 @@ QMOE_API qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t val
 
 /* The forward path qmoe_forward takes for T tokens: 0 = fp32 SIMT path,
  * 1 = weight-streaming decode path (mma.sync), 2 = tcgen05 grouped GEMM,
- * 3 = tcgen05 streaming decode. -1 for a NULL handle. */
+ * 3 = tcgen05 streaming decode, 4 = int8 block tier (weight-streaming
+ * integer mma.sync). -1 for a NULL handle. */
 QMOE_API int32_t qmoe_path_for(const qmoe_handle* h, int64_t T);
 
 /* Number of kernel launches qmoe_forward enqueues for T tokens: routing and
  * permutation (one launch for T <= 64, two above), the row gather (tensor-core
- * paths), FC1, FC2 and the combine. 0 for T = 0. */
+ * paths, and apply_router_weight_on_input), the int8 rounding of FC1's and
+ * FC2's input rows (int8 block tier), FC1, FC2 and the combine. 0 for T = 0. */
 QMOE_API int32_t qmoe_launches_for(const qmoe_handle* h, int64_t T);
 
 /* Token-tile width (the MMA N dimension, rows of one expert per work item)

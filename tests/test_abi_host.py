@@ -45,6 +45,7 @@ def test_config_struct_layout(q):
     assert q.qmoe_config.reserved.offset == 92
     assert q.qmoe_config.n_group.offset == 96
     assert q.qmoe_config.apply_router_weight_on_input.offset == 108
+    assert q.qmoe_config.compute_mode.offset == 116
 
 
 def _cfg(q, **kw):
@@ -73,7 +74,11 @@ BAD = [
     (dict(n_group=4, topk_group=1, k=3), 1),                    # k > topk_group * E / n_group
     (dict(num_experts=128, n_group=64, topk_group=1, k=1), 3),  # more than 32 groups: not built
     (dict(apply_router_weight_on_input=2), 1), (dict(routed_scaling_factor=-1.0), 1),
-    (dict(weight_format=2), 1), (dict(reserved2=1), 1),
+    (dict(weight_format=2), 1), (dict(compute_mode=2), 1), (dict(compute_mode=-1), 1),
+    (dict(compute_mode=1, block_size=0), 1),                    # the int8 tier needs block scales
+    (dict(compute_mode=1, weight_format=1, block_size=32, scale_dtype=2), 1),  # ... and integer codes
+    (dict(compute_mode=1, block_size=32), 3),                   # 4-bit codes: blocks below 64 not built
+    (dict(compute_mode=1, expert_weight_bits=8, block_size=16), 3),
     (dict(weight_format=1, block_size=32), 1),                  # MXFP4 needs E8M0 scales
     (dict(weight_format=1, block_size=64, scale_dtype=2), 1),   # ... and block_size 32
     (dict(weight_format=1, expert_weight_bits=8, block_size=32, scale_dtype=2), 1),
@@ -154,3 +159,52 @@ def test_status_strings(q):
                     (3, b"QMOE_UNSUPPORTED"), (4, b"QMOE_CUDA_ERROR"), (5, b"QMOE_TIMEOUT"),
                     (6, b"QMOE_OUT_OF_MEMORY")]:
         assert q.lib.qmoe_status_string(s) == name
+
+
+def test_int8_tier_plan(q):
+    # compute_mode INT8_BLOCK: path 4 for every T, the two rounding launches
+    # added, and the code buffers in the workspace
+    h = q.qmoe_create(_cfg(q, compute_mode=q.COMPUTE_INT8_BLOCK))
+    hf = q.qmoe_create(_cfg(q))
+    ha = q.qmoe_create(_cfg(q, compute_mode=q.COMPUTE_INT8_BLOCK, apply_router_weight_on_input=1))
+    try:
+        for T in (1, 8, 64, 65, 4096):
+            assert q.qmoe_path_for(h, T) == q.PATH_INT8
+            assert q.qmoe_token_tile_for(h, T) == 0
+        assert q.qmoe_launches_for(h, 8) == 6     # route+permute, quantize x, FC1, quantize h, FC2, combine
+        assert q.qmoe_launches_for(h, 65) == 7    # routing and permutation apart
+        assert q.qmoe_launches_for(ha, 8) == 7    # plus the weighted row gather
+        # codes and scales of x [T, H] and h [T*k, I] on top of the float plan
+        T, H, I, k, bs = 8, 256, 512, 2, 64
+        extra = T * H + T * (H // bs) * 4 + T * k * I + T * k * (I // bs) * 4
+        assert q.qmoe_workspace_size(h, T) >= q.qmoe_workspace_size(hf, T) + extra
+        q.qmoe_set_option(h, q.QMOE_OPT_PATH, 2)  # ignored on the int8 tier
+        assert q.qmoe_path_for(h, 8) == q.PATH_INT8
+    finally:
+        q.qmoe_destroy(h)
+        q.qmoe_destroy(hf)
+        q.qmoe_destroy(ha)
+    hs = q.qmoe_create(_cfg(q, compute_mode=q.COMPUTE_INT8_BLOCK, act_dtype=q.DTYPE_F32,
+                            scale_dtype=q.DTYPE_F32))
+    assert q.qmoe_path_for(hs, 8) == q.PATH_INT8  # fp32 activations take the tier too
+    q.qmoe_destroy(hs)
+
+
+@pytest.mark.parametrize("args", [
+    (1, 64, 8),        # block_size below 16
+    (1, 96, 64),       # K not a multiple of block_size
+    (1, 64, 48),       # block_size not a power of two
+    (-1, 64, 16),      # negative rows
+    (1, 0, 16),        # empty rows
+])
+def test_quantize_entry_rejects_bad_sizes_without_device_work(q, args):
+    rows, K, bs = args
+    assert q.lib.qmoe_quantize_act_i8(256, q.DTYPE_BF16, rows, K, bs, 256, 256, None) == q.QMOE_INVALID_ARGUMENT
+
+
+def test_quantize_entry_rejects_bad_dtype_alignment_and_null(q):
+    assert q.lib.qmoe_quantize_act_i8(256, q.DTYPE_E8M0, 1, 64, 16, 256, 256, None) == q.QMOE_INVALID_ARGUMENT
+    assert q.lib.qmoe_quantize_act_i8(264, q.DTYPE_BF16, 1, 64, 16, 256, 256, None) == q.QMOE_INVALID_ARGUMENT
+    assert q.lib.qmoe_quantize_act_i8(256, q.DTYPE_BF16, 1, 64, 16, 258, 256, None) == q.QMOE_INVALID_ARGUMENT
+    assert q.lib.qmoe_quantize_act_i8(None, q.DTYPE_BF16, 1, 64, 16, 256, 256, None) == q.QMOE_INVALID_ARGUMENT
+    assert q.lib.qmoe_quantize_act_i8(None, q.DTYPE_BF16, 0, 64, 16, None, None, None) == q.QMOE_OK  # no rows

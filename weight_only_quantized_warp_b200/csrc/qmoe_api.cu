@@ -40,7 +40,9 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
                                touched * (padded_rows(H) / kBlockRows) * tcd_s2 < 4 * kSms))
         ++tcd_s2;
     const bool tcd_ok = per_expert <= 32 && tc_decode_fits(H, 1, tcd_bn, bs) && tc_decode_fits(I, tcd_s2, tcd_bn, bs);
-    if (!bf16)
+    if (c.compute_mode == QMOE_COMPUTE_INT8_BLOCK)
+        p.path = kPathI8;
+    else if (!bf16)
         p.path = kPathSimt;
     else if (h.path_override == kPathDecode || h.path_override == kPathTc)
         p.path = h.path_override;
@@ -52,10 +54,15 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         p.bn = tcd_bn;
         p.fc2_splits = tcd_s2;
     }
-    if (p.path == kPathDecode) {
+    if (p.path == kPathDecode || p.path == kPathI8) {
+        // shared memory of one CTA: staged bf16 rows, or int8 code rows
+        auto smem = [&](int64_t K, int splits, int nt) {
+            return p.path == kPathI8 ? i8_smem_bytes(K, bits, bs, splits, nt)
+                                     : decode_smem_bytes(K, bits, bs, splits, nt);
+        };
         p.nt = per_expert <= 8 ? 1 : (per_expert <= 16 ? 2 : 4);
         // FC1 runs unsplit; keep its staged rows small enough for two CTAs per SM
-        while (p.nt > 1 && decode_smem_bytes(H, bits, bs, 1, p.nt) > kDecodeSmemTarget) p.nt /= 2;
+        while (p.nt > 1 && smem(H, 1, p.nt) > kDecodeSmemTarget) p.nt /= 2;
         // enough FC2 warps (one per 16-row tile per touched expert per split)
         // to give every SM several resident warps
         const int64_t warps = touched * (H / kTileRows);
@@ -63,11 +70,11 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         const int64_t ngr = I / kgroup_of(bits);
         int64_t s = ceil_div(want, warps);
         s = std::min<int64_t>(s, 8);
-        while (s < ngr && decode_smem_bytes(I, bits, bs, int(s), p.nt) > kDecodeSmemTarget) ++s;
+        while (s < ngr && smem(I, int(s), p.nt) > kDecodeSmemTarget) ++s;
         s = std::min<int64_t>(s, ngr);
         p.fc2_splits = int(std::max<int64_t>(s, 1));
-        p.ok = decode_smem_bytes(H, bits, bs, 1, p.nt) <= int64_t(kDecodeSmemLimit) &&
-               decode_smem_bytes(I, bits, bs, p.fc2_splits, p.nt) <= int64_t(kDecodeSmemLimit);
+        p.ok = smem(H, 1, p.nt) <= int64_t(kDecodeSmemLimit) &&
+               smem(I, p.fc2_splits, p.nt) <= int64_t(kDecodeSmemLimit);
     } else if (p.path == kPathTc) {
         // token tile: the power of two covering the average segment with a
         // third to spare, so that most experts take one tile (the weights of
@@ -86,7 +93,8 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     // the row gather runs on the tensor-core paths, and on every path when
     // the router weights scale the expert inputs
     p.gather = p.path == kPathTc || p.path == kPathTcDecode || c.apply_router_weight_on_input;
-    p.launches = (p.fused_route ? 1 : 2) + (p.gather ? 1 : 0) + 3;
+    // the int8 tier adds the rounding of FC1's input rows and of h
+    p.launches = (p.fused_route ? 1 : 2) + (p.gather ? 1 : 0) + 3 + (p.path == kPathI8 ? 2 : 0);
     const size_t R = size_t(p.R);
     const size_t act = bf16 ? 2 : 4;
     size_t off = 0;
@@ -100,6 +108,15 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     p.off_xperm = off;
     off = align256(off + (p.gather ? R * size_t(H) * act : 0));
     p.off_o = off;       off = align256(off + size_t(p.fc2_splits) * R * size_t(H) * 4);
+    if (p.path == kPathI8) {
+        const size_t nsb1 = size_t(H / bs), nsb2 = size_t(I / bs);
+        p.xq_rows = p.gather ? p.R : T;
+        const size_t xr = size_t(p.xq_rows);
+        p.off_xq = off; off = align256(off + xr * size_t(H));
+        p.off_xs = off; off = align256(off + xr * nsb1 * 4);
+        p.off_hq = off; off = align256(off + R * size_t(I));
+        p.off_hs = off; off = align256(off + R * nsb2 * 4);
+    }
     p.total = off;
     return p;
 }
@@ -166,7 +183,16 @@ qmoe_status validate(const qmoe_config& c, std::string& why) {
                (c.scale_dtype != QMOE_DTYPE_F32 && c.scale_dtype != QMOE_DTYPE_BF16)) {
         return bad(QMOE_INVALID_ARGUMENT, "act_dtype and scale_dtype must be F32 or BF16");
     }
-    if (c.reserved != 0 || c.reserved2 != 0) return bad(QMOE_INVALID_ARGUMENT, "reserved fields must be 0");
+    if (c.reserved != 0) return bad(QMOE_INVALID_ARGUMENT, "reserved fields must be 0");
+    if (c.compute_mode != QMOE_COMPUTE_FLOAT && c.compute_mode != QMOE_COMPUTE_INT8_BLOCK)
+        return bad(QMOE_INVALID_ARGUMENT, "compute_mode must be FLOAT or INT8_BLOCK");
+    if (c.compute_mode == QMOE_COMPUTE_INT8_BLOCK) {
+        if (c.weight_format != QMOE_WEIGHTS_INT || c.block_size == 0)
+            return bad(QMOE_INVALID_ARGUMENT, "the int8 block tier needs integer codes with block scales");
+        if (c.block_size < kgroup_of(c.expert_weight_bits))
+            return bad(QMOE_UNSUPPORTED,
+                       "int8 block tier: block_size below 64 (4-bit codes) or 32 (8-bit codes) is not built");
+    }
     if (c.use_sparse_mixer) return bad(QMOE_UNSUPPORTED, "use_sparse_mixer is not built");
     if (c.num_experts > 256) return bad(QMOE_UNSUPPORTED, "num_experts > 256 is not built");
     if (c.hidden_size % 64 || c.inter_size % 64) {
@@ -275,6 +301,7 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
     err = prepare_route_permute();
     if (err == cudaSuccess) err = prepare_ffn_decode();
     if (err == cudaSuccess) err = prepare_ffn_tc();
+    if (err == cudaSuccess) err = prepare_ffn_i8();
     if (err != cudaSuccess) return cuda_fail(h, err, "prepare kernels");
 
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size, N1 = h->n1;
@@ -491,18 +518,42 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
         f1.act = xp;
         f1.rowmap = nullptr;  // rows already in segment order
     }
-    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-    err = p.path == kPathSimt        ? launch_ffn_simt(f1, st)
-          : p.path == kPathTc        ? launch_ffn_tc(f1, p.bn, status, st)
-          : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f1, p.bn, status, st)
-                                     : launch_ffn_decode(f1, st);
-    if (err != cudaSuccess) return cuda_fail(h, err, "fc1");
-    if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-    err = p.path == kPathSimt        ? launch_ffn_simt(f2, st)
-          : p.path == kPathTc        ? launch_ffn_tc(f2, p.bn, status, st)
-          : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f2, p.bn, status, st)
-                                     : launch_ffn_decode(f2, st);
-    if (err != cudaSuccess) return cuda_fail(h, err, "fc2");
+    if (p.path == kPathI8) {
+        // FC1's input rows (x by token, or the gathered rows) to int8 codes
+        const int perm = c.expert_weight_bits == 4;
+        int8_t* xq = (int8_t*)(ws + p.off_xq);
+        float* xs = (float*)(ws + p.off_xs);
+        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+        if ((err = launch_quantize_i8(f1.act, bf16, p.xq_rows, c.hidden_size, c.block_size, perm, xq, xs, st)) !=
+            cudaSuccess)
+            return cuda_fail(h, err, "quantize x");
+        f1.aq = xq;
+        f1.as = xs;
+        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+        if ((err = launch_ffn_i8(f1, st)) != cudaSuccess) return cuda_fail(h, err, "fc1");
+        int8_t* hq = (int8_t*)(ws + p.off_hq);
+        float* hs = (float*)(ws + p.off_hs);
+        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+        if ((err = launch_quantize_i8(hid, bf16, p.R, c.inter_size, c.block_size, perm, hq, hs, st)) != cudaSuccess)
+            return cuda_fail(h, err, "quantize h");
+        f2.aq = hq;
+        f2.as = hs;
+        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+        if ((err = launch_ffn_i8(f2, st)) != cudaSuccess) return cuda_fail(h, err, "fc2");
+    } else {
+        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+        err = p.path == kPathSimt        ? launch_ffn_simt(f1, st)
+              : p.path == kPathTc        ? launch_ffn_tc(f1, p.bn, status, st)
+              : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f1, p.bn, status, st)
+                                         : launch_ffn_decode(f1, st);
+        if (err != cudaSuccess) return cuda_fail(h, err, "fc1");
+        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
+        err = p.path == kPathSimt        ? launch_ffn_simt(f2, st)
+              : p.path == kPathTc        ? launch_ffn_tc(f2, p.bn, status, st)
+              : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f2, p.bn, status, st)
+                                         : launch_ffn_decode(f2, st);
+        if (err != cudaSuccess) return cuda_fail(h, err, "fc2");
+    }
     CombineArgs ca{};
     ca.o = o;
     ca.topk_idx = idx;
@@ -574,6 +625,20 @@ qmoe_status qmoe_debug_hidden(const qmoe_handle* h, int64_t T, const void* works
     cudaError_t err = cudaMemcpyAsync(hidden, (const char*)workspace + p.off_h, n,
                                       cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
     return err == cudaSuccess ? QMOE_OK : cuda_fail(h, err, "debug_hidden");
+}
+
+qmoe_status qmoe_quantize_act_i8(const void* x, int32_t dtype, int64_t rows, int64_t K, int32_t block_size,
+                                 int8_t* q, float* scales, void* stream) {
+    if (rows < 0 || K < 1 || !pow2(block_size) || block_size < 16 || K % block_size)
+        return QMOE_INVALID_ARGUMENT;
+    if (dtype != QMOE_DTYPE_F32 && dtype != QMOE_DTYPE_BF16) return QMOE_INVALID_ARGUMENT;
+    if (rows == 0) return QMOE_OK;
+    if (!x || !q || !scales || (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(q) & 3) ||
+        (reinterpret_cast<uintptr_t>(scales) & 3))
+        return QMOE_INVALID_ARGUMENT;
+    const cudaError_t err = launch_quantize_i8(x, dtype == QMOE_DTYPE_BF16, rows, K, block_size, 0, q, scales,
+                                               (cudaStream_t)stream);
+    return err == cudaSuccess ? QMOE_OK : QMOE_CUDA_ERROR;
 }
 
 qmoe_status qmoe_read_device_status(const qmoe_handle* h, const void* workspace, void* stream) {

@@ -48,7 +48,7 @@ __host__ __device__ constexpr int64_t padded_rows(int64_t n) {
 }
 
 // Hot-path selection.
-enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2, kPathTcDecode = 3 };
+enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2, kPathTcDecode = 3, kPathI8 = 4 };
 
 struct Plan {
     int path = kPathDecode;
@@ -62,6 +62,10 @@ struct Plan {
     bool gather = false;       // routed rows of x gathered (and weighted) into the workspace
     size_t off_idx = 0, off_w = 0, off_inv = 0, off_perm = 0, off_offsets = 0, off_status = 0,
            off_h = 0, off_o = 0, off_xperm = 0, total = 0;
+    // int8 block tier: codes and block scales of FC1's input rows (x, or the
+    // gathered rows) and of h
+    int64_t xq_rows = 0;
+    size_t off_xq = 0, off_xs = 0, off_hq = 0, off_hs = 0;
 };
 
 }  // namespace qmoe
@@ -144,6 +148,11 @@ struct FfnArgs {
     int scale_bf16, act_bf16;
     int nt;
     int fp4;                 // codes are MXFP4 e2m1 (no zero point)
+    // int8 block tier: the activation rows as codes [rows, K] (for 4-bit
+    // weights every run of 4 codes in the order k+0, k+2, k+1, k+3) and
+    // per-block scales [rows, K / block_size]; rows indexed like `act`
+    const int8_t* aq;
+    const float* as;
 };
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
 // Shared memory of one decode CTA (staged activation rows) and its limit;
@@ -179,6 +188,13 @@ cudaError_t launch_gather_rows_weighted(const void* x, const int32_t* perm, cons
                                         const float* topk_w, int k, void* xp, int64_t R, int64_t H, int act_bf16,
                                         cudaStream_t st);
 
+// Int8 block compute tier: per-block int8 rounding of activation rows (perm:
+// the 4-code order of 4-bit weights), and the expert FFN layer on the codes.
+cudaError_t launch_quantize_i8(const void* x, int act_bf16, int64_t rows, int64_t K, int bs, int perm, int8_t* q,
+                               float* s, cudaStream_t st);
+int64_t i8_smem_bytes(int64_t K, int bits, int block_size, int splits, int nt);
+cudaError_t prepare_ffn_i8();
+cudaError_t launch_ffn_i8(const FfnArgs& a, cudaStream_t st);
 // Router-weighted combine with fc2 bias and shared output; sums the FC2
 // split partials in fixed order.
 struct CombineArgs {

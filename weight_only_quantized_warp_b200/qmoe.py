@@ -29,7 +29,8 @@ QMOE_CUDA_ERROR, QMOE_TIMEOUT, QMOE_OUT_OF_MEMORY = 4, 5, 6
 ACT_RELU, ACT_GELU, ACT_SILU, ACT_SWIGLU, ACT_IDENTITY = 0, 1, 2, 3, 4
 DTYPE_F32, DTYPE_BF16, DTYPE_E8M0 = 0, 1, 2
 WEIGHTS_INT, WEIGHTS_MXFP4 = 0, 1
-PATH_SIMT, PATH_DECODE, PATH_TC, PATH_TC_DECODE = 0, 1, 2, 3
+COMPUTE_FLOAT, COMPUTE_INT8_BLOCK = 0, 1
+PATH_SIMT, PATH_DECODE, PATH_TC, PATH_TC_DECODE, PATH_INT8 = 0, 1, 2, 3, 4
 
 # Every function the header declares (checked against include/qmoe.h by the tests).
 EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forward",
@@ -37,7 +38,8 @@ EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forwa
            "qmoe_debug_routing", "qmoe_debug_hidden", "qmoe_read_device_status", "qmoe_destroy",
            "qmoe_status_string", "qmoe_last_error", "qmoe_path_for", "qmoe_launches_for",
            "qmoe_token_tile_for",
-           "qmoe_set_option", "qmoe_forward_noalloc", "qmoe_noalloc_scratch_bytes")
+           "qmoe_set_option", "qmoe_forward_noalloc", "qmoe_noalloc_scratch_bytes",
+           "qmoe_quantize_act_i8")
 QMOE_OPT_PATH = 1
 
 
@@ -54,7 +56,7 @@ class qmoe_config(ctypes.Structure):
                 ("use_sparse_mixer", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
                 ("routed_scaling_factor", ctypes.c_float), ("apply_router_weight_on_input", ctypes.c_int32),
-                ("weight_format", ctypes.c_int32), ("reserved2", ctypes.c_int32)]
+                ("weight_format", ctypes.c_int32), ("compute_mode", ctypes.c_int32)]
 
 
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
@@ -93,6 +95,8 @@ lib.qmoe_launches_for.restype = ctypes.c_int32
 lib.qmoe_launches_for.argtypes = [_vp, _i64]
 lib.qmoe_token_tile_for.restype = ctypes.c_int32
 lib.qmoe_token_tile_for.argtypes = [_vp, _i64]
+lib.qmoe_quantize_act_i8.restype = ctypes.c_int
+lib.qmoe_quantize_act_i8.argtypes = [_vp, ctypes.c_int32, _i64, _i64, ctypes.c_int32, _vp, _vp, _vp]
 
 
 class QMoEError(RuntimeError):
@@ -144,7 +148,8 @@ def make_config(cfg) -> qmoe_config:
         n_group=int(getattr(cfg, "n_group", 0)), topk_group=int(getattr(cfg, "topk_group", 0)),
         routed_scaling_factor=float(getattr(cfg, "routed_scaling_factor", 1.0)),
         apply_router_weight_on_input=int(getattr(cfg, "apply_router_weight_on_input", False)),
-        weight_format=int(getattr(cfg, "weight_format", 0)), reserved2=0)
+        weight_format=int(getattr(cfg, "weight_format", 0)),
+        compute_mode=int(getattr(cfg, "compute_mode", 0)))
 
 
 def qmoe_create(cfg: qmoe_config) -> int:
@@ -221,6 +226,13 @@ def qmoe_launches_for(h, T: int) -> int:
 
 def qmoe_token_tile_for(h, T: int) -> int:
     return int(lib.qmoe_token_tile_for(h, T))
+
+
+def qmoe_quantize_act_i8(x, dtype: int, rows: int, K: int, block_size: int, q, scales, stream=None):
+    """Int8 block tier rounding of activation rows x [rows, K] into codes q
+    [rows, K] int8 and scales [rows, K / block_size] fp32 (device buffers)."""
+    _check(lib.qmoe_quantize_act_i8(_ptr(x), dtype, rows, K, block_size, _ptr(q), _ptr(scales),
+                                    _stream(stream)))
 
 
 # ------------------------------------------------------------- torch plumbing
