@@ -133,7 +133,7 @@ constexpr int kRing = 8;               // weight loads in flight per lane
 // part (loads always in range, no guards), one guarded drain round and a
 // tail; all shared-memory, weight and scale addresses advance by constants.
 template <int BITS, int SMODE, bool SF32, int NT, int P>
-__global__ void __launch_bounds__(kWarps * 32, 2) ffn_decode_kernel(const FfnArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 3) ffn_decode_kernel(const FfnArgs a) {
     constexpr int KG = kgroup_of(BITS);
     constexpr int D = kRing;
     static_assert(D % P == 0, "scale chunk must divide the ring");

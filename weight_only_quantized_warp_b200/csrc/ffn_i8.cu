@@ -46,7 +46,8 @@ namespace qmoe {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kRing = 8;  // weight loads in flight per lane
+constexpr int kRing = 8;       // weight loads in flight per lane
+constexpr int kMaxChunk = 8;   // k-groups per scale chunk at most (the kernels built)
 
 // D (int32) = A (u8) x B (s8) [+ D]
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(const void* x, in
 // 32-bit reads of rows r0 = 0..7 at offsets 4c land in 32 distinct banks.
 __host__ __device__ constexpr int64_t staged_row_bytes_i8(int64_t kr) { return kr + 16; }
 
-// P: k-groups per scale chunk (min(groups per block, kRing)); the chunk's
+// P: k-groups per scale chunk (min(groups per block, kMaxChunk)); the chunk's
 // int32 partial is scaled and added to the fp32 accumulator at its end.
 //
 // One CTA = 8 warps = the 8 row tiles of one 128-row block of one expert, for
@@ -149,7 +150,7 @@ __host__ __device__ constexpr int64_t staged_row_bytes_i8(int64_t kr) { return k
 // has a steady part (loads always in range), one guarded drain round and a
 // tail, as in the bf16 decode kernels.
 template <int BITS, bool SF32, int NT, int P>
-__global__ void __launch_bounds__(kWarps * 32, 2) ffn_i8_kernel(const FfnArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 3) ffn_i8_kernel(const FfnArgs a) {
     constexpr int KG = kgroup_of(BITS);
     constexpr int D = kRing;
     static_assert(D % P == 0, "scale chunk must divide the ring");
@@ -390,7 +391,7 @@ cudaError_t raise_sf() {
 
 int chunk_groups(int bits, int block_size) {
     const int gpb = block_size / kgroup_of(bits);
-    return gpb >= kRing ? kRing : gpb;
+    return gpb >= kMaxChunk ? kMaxChunk : gpb;
 }
 
 }  // namespace

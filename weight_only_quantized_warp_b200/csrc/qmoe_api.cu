@@ -61,7 +61,7 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
                                      : decode_smem_bytes(K, bits, bs, splits, nt);
         };
         p.nt = per_expert <= 8 ? 1 : (per_expert <= 16 ? 2 : 4);
-        // FC1 runs unsplit; keep its staged rows small enough for two CTAs per SM
+        // FC1 runs unsplit; keep its staged rows small enough for at least two CTAs per SM
         while (p.nt > 1 && smem(H, 1, p.nt) > kDecodeSmemTarget) p.nt /= 2;
         // enough FC2 warps (one per 16-row tile per touched expert per split)
         // to give every SM several resident warps

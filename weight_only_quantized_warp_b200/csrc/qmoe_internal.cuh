@@ -158,7 +158,7 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
 // Shared memory of one decode CTA (staged activation rows) and its limit;
 // prepare_ffn_decode() raises the kernels' limit on the current device.
 constexpr size_t kDecodeSmemLimit = 200 * 1024;
-constexpr int64_t kDecodeSmemTarget = 112 * 1024;  // two CTAs per SM
+constexpr int64_t kDecodeSmemTarget = 112 * 1024;  // at least two CTAs per SM (three fit below 75 KB)
 // Rows per expert up to which the weight-streaming kernels are chosen.
 constexpr int64_t kDecodeRowsPerExpert = 16;
 int64_t decode_smem_bytes(int64_t K, int bits, int block_size, int splits, int nt);
