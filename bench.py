@@ -3,7 +3,10 @@
 Default workload: Mixtral-like decode (T=8, H=4096, I=14336, E=8, k=2, int4
 block_size 128, bf16 activations and scales, swiglu fused not interleaved,
 renormalised routing), seeded synthetic inputs. One step = one whole forward
-(routing, permutation, FC1 + SwiGLU, FC2, combine) over the batch.
+(routing, permutation, FC1 + SwiGLU, FC2, combine) over the batch, launched
+as one CUDA graph replay; the JSON line also gives the step time with direct
+launches, the per-kernel times of a separate event-bracketed pass, and the
+end-to-end rate through the public call with host buffers.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle, timed on host cores
@@ -72,6 +75,7 @@ def config_of(cfg, name, world):
     return {"workload": name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
             "bits": cfg.bits, "block_size": cfg.block_size, "swiglu_fusion": cfg.fusion,
             "act_dtype": "bf16" if cfg.act_dtype == gen.DT_BF16 else "f32",
+            "compute": "int8 block tier" if cfg.compute_mode == gen.COMPUTE_INT8_BLOCK else "float",
             "tokens_per_step": cfg.T * world, "parallelism": f"replicas x{world}",
             "l2": "no flush: the expert weights a step streams exceed the 126 MB L2"}
 
@@ -258,6 +262,15 @@ def run_ours(args):
         fwd()
     torch.cuda.synchronize()
 
+    # one step = one forward, replayed from a CUDA graph (the forward enqueues
+    # only stream-ordered device work, so it captures as is)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):  # captures on a side stream; replays on `stream`
+        qmoe.qmoe_forward(h, T, x, lg, sh, y, ws, nws, torch.cuda.current_stream())
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+
     # routing of this batch (for the algorithmic byte count)
     off = torch.empty(cfg.E + 1, dtype=torch.int32, device=dev)
     qmoe.qmoe_debug_routing(h, T, ws, offsets=off)
@@ -278,7 +291,7 @@ def run_ours(args):
         t_end = time.perf_counter() + seconds
         while time.perf_counter() < t_end:
             for _ in range(20):
-                fwd()
+                graph.replay()
             torch.cuda.synchronize()
 
     clocks.start()
@@ -288,7 +301,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     start.record(stream)
     for i in range(K):
-        qmoe.qmoe_forward_profiled(h, T, x, lg, sh, y, ws, nws, evs[i], stream)
+        graph.replay()
     stop.record(stream)
     torch.cuda.synchronize()
     keep_loaded(0.4)
@@ -298,13 +311,31 @@ def run_ours(args):
     ms = replicas.max_over_ranks([start.elapsed_time(stop)], dev)[0]
     if world > 1:
         dist.barrier(device_ids=[local])
+
+    # after the timed region: the same K steps as direct launches, and once
+    # more with an event between kernels for the per-kernel times (the events
+    # themselves add a few microseconds per launch)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for i in range(K):
+        fwd()
+    s1.record(stream)
+    for i in range(K):
+        qmoe.qmoe_forward_profiled(h, T, x, lg, sh, y, ws, nws, evs[i], stream)
+    torch.cuda.synchronize()
+    stream_ms = replicas.max_over_ranks([s0.elapsed_time(s1)], dev)[0]
+    del graph
+    if world > 1:
+        dist.barrier(device_ids=[local])
     per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(launches)]
                            for i in range(K)]).mean(axis=0)
     path = qmoe.qmoe_path_for(h, T)
     gather = path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE) or bool(cfg.apply_router_weight_on_input)
-    fused = launches - int(gather) - 3 == 1  # routing and permutation in one launch
+    i8 = path == qmoe.PATH_INT8
+    ffn = ["quantize_x", "fc1", "quantize_h", "fc2"] if i8 else ["fc1", "fc2"]
+    fused = launches - int(gather) - len(ffn) - 1 == 1  # routing and permutation in one launch
     names = ((["route_permute"] if fused else ["route", "permute"]) + (["gather"] if gather else [])
-             + ["fc1", "fc2", "combine"])
+             + ffn + ["combine"])
 
     # ---- end to end through the public call, host buffers, copies inside
     x_h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu())
@@ -367,7 +398,8 @@ def run_ours(args):
     t_tc = fc1_flops / (tc_peak * 1e12)
     tile = qmoe.qmoe_token_tile_for(h, T)
     kbase = ("ffn_tc_wide_kernel" if tile > 128 else "ffn_tc_kernel") if path == qmoe.PATH_TC else \
-        {qmoe.PATH_TC_DECODE: "ffn_tc_decode_kernel", qmoe.PATH_SIMT: "ffn_simt_kernel"}.get(path, "ffn_decode_kernel")
+        {qmoe.PATH_TC_DECODE: "ffn_tc_decode_kernel", qmoe.PATH_SIMT: "ffn_simt_kernel",
+         qmoe.PATH_INT8: "ffn_i8_kernel"}.get(path, "ffn_decode_kernel")
     kname = kbase + " (FC1 + activation)"
     tr = traffic_record("fc1_" + kbase + "_" + args.workload)
     if t_hbm >= t_tc:
@@ -385,14 +417,18 @@ def run_ours(args):
     whole = alg["total_bytes"] / (step_ms / 1e3) / 1e9
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.act_dtype else "f32",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "s8" if i8 else ("bf16" if cfg.act_dtype else "f32"),
             "data": "synthetic (seeded, shapes of the workload; no trained weights)",
             "config": config_of(cfg, args.workload, world),
             "roofline": roofline,
             "step": {"hbm_gbs": whole, "tflops": alg["flops"] / (step_ms / 1e3) / 1e12,
                      "hbm_frac": whole / hbm_peak, "experts_touched": alg["touched"],
                      "algorithmic_bytes": alg["total_bytes"],
-                     "kernel_ms": kms, "path": path, "token_tile": tile},
+                     "kernel_ms": kms, "path": path, "token_tile": tile,
+                     "launch": "CUDA graph of one forward per step",
+                     "ms_per_step_direct_launches": stream_ms / K,
+                     "kernel_ms_note": "from a separate pass with an event between kernels"},
             "cpu_baseline": cpu,
             "e2e": {"value": replicas.job_tokens_per_s(T, world, K, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
