@@ -12,8 +12,8 @@ The forward is compared like the float tier: routing bit for bit, h within
 sides, so h differs only by fp32 accumulation -- and y within 1e-2 for both
 activation dtypes. The looser y bound for fp32 comes from the arithmetic: FC2
 rounds h to int8, and where the kernel's fp32 h and the oracle's exact h fall
-on the two sides of a rounding boundary (a few per thousand codes when h
-differs by ~1e-6 relative) the code moves by one step, which moves an output
+on the two sides of a rounding boundary (a few per ten thousand codes when
+h differs by ~1e-6 relative) the code moves by one step, which moves an output
 by up to s_h * |s_w| * 2^(bits-1), about 1e-3 of it.
 """
 from __future__ import annotations
