@@ -9,7 +9,11 @@ Definitions followed are the same passages as the C oracle: the "QMoE"
 operator page (layouts, pack_size, block_size, swiglu_fusion, activation
 attributes, k, normalize_routing_weights), the "MoE" page summary (top-k,
 gated FFN, weighted combine), the "QLinearWoQ" summary (x @ dequant(W).T + b)
-and "ClikaRT::nn::QMoEWoQ" forward() (shared_output folds into the combine).
+and "ClikaRT::nn::QMoEWoQ" forward() (shared_output folds into the combine),
+plus its class description's int8 block tier (compute_mode 1: per-block
+int8 rounding of each expert input row, decided with numpy float32 scalars,
+and integer dots per block). Grouped routing, the router weight on the
+input, routed scaling and MXFP4 are left to the C oracle.
 """
 from __future__ import annotations
 
@@ -65,6 +69,46 @@ def route_weights(logits_row, sel, normalize):
     return w
 
 
+def round_act(v, bf16):
+    """v rounded to the activation dtype: fp32 by numpy's conversion; bf16 by
+    keeping 8 significant bits (round half to even, Python's round on an
+    exactly scaled float)."""
+    if not bf16:
+        return float(np.float32(v))
+    if v == 0.0 or not math.isfinite(v):
+        return v
+    ex = math.frexp(v)[1]
+    lsb = max(ex - 8, -133)
+    return math.ldexp(round(math.ldexp(v, -lsb)), lsb)
+
+
+def quantize_row(v, bs):
+    """Int8 block tier ("ClikaRT::nn::QMoEWoQ" class description, read as
+    symmetric absmax rounding decided in fp32): per block of bs values,
+    s = absmax / 127 and q = rint(v / s) clamped to +-127, with numpy float32
+    scalars for every decision."""
+    codes, scales = [], []
+    for b in range(len(v) // bs):
+        blk = [np.float32(a) for a in v[b * bs:(b + 1) * bs]]
+        amax = max(abs(a) for a in blk)
+        s = np.float32(amax) / np.float32(127.0)
+        scales.append(float(s))
+        for a in blk:
+            q = 0 if s == 0 else int(np.rint(a / s))
+            codes.append(max(-127, min(127, q)))
+    return codes, scales
+
+
+def dot_i8(packed_row, scales_row, K, bits, bs, codes, xs):
+    """sum over blocks of s_w * s_x * (integer dot of centred codes)."""
+    z = 2 ** (bits - 1)
+    tot = 0.0
+    for b in range(K // bs):
+        d = sum((_code(packed_row, k, bits) - z) * codes[k] for k in range(b * bs, (b + 1) * bs))
+        tot += float(scales_row[b]) * xs[b] * d
+    return tot
+
+
 def activation(act, g, u, alpha, beta, limit, gated):
     sig = lambda v: 1.0 / (1.0 + math.exp(-v))  # noqa: E731
     if not gated:
@@ -104,6 +148,11 @@ def forward(inp):
     W3 = ([dense_weight(inp.fc3_w[e], scl(inp.fc3_s)[e], c.I, c.H, c.bits, c.block_size)
            for e in range(c.E)] if c.has_fc3 else None)
 
+    i8 = getattr(c, "compute_mode", 0) == 1
+    bf16 = np.asarray(inp.x).dtype == np.uint16
+    S1, S2 = scl(inp.fc1_s), scl(inp.fc2_s)
+    S3 = scl(inp.fc3_s) if c.has_fc3 else None
+
     y = np.zeros((c.T, c.H))
     sels, wts = [], []
     for t in range(c.T):
@@ -115,7 +164,12 @@ def forward(inp):
         xt = x[t].tolist()
         for j, e in enumerate(sel):
             b1, b2, b3 = bias(inp.fc1_b, e), bias(inp.fc2_b, e), bias(inp.fc3_b, e)
-            a = [sum(xt[kk] * W1[e][n][kk] for kk in range(c.H)) + b1[n] for n in range(N1)]
+            if i8:
+                qx, sx = quantize_row(xt, c.block_size)
+                a = [dot_i8(inp.fc1_w[e][n], S1[e][n], c.H, c.bits, c.block_size, qx, sx) + b1[n]
+                     for n in range(N1)]
+            else:
+                a = [sum(xt[kk] * W1[e][n][kk] for kk in range(c.H)) + b1[n] for n in range(N1)]
             h = []
             for i in range(c.I):
                 if not gated:
@@ -127,10 +181,18 @@ def forward(inp):
                     g, u = a[i], a[c.I + i]
                 else:
                     g = a[i]
-                    u = sum(xt[kk] * W3[e][i][kk] for kk in range(c.H)) + b3[i]
+                    if i8:
+                        u = dot_i8(inp.fc3_w[e][i], S3[e][i], c.H, c.bits, c.block_size, qx, sx) + b3[i]
+                    else:
+                        u = sum(xt[kk] * W3[e][i][kk] for kk in range(c.H)) + b3[i]
                 h.append(activation(c.act, g, u, c.alpha, c.beta, c.limit, True))
+            if i8:
+                qh, sh_ = quantize_row([round_act(v, bf16) for v in h], c.block_size)
             for m in range(c.H):
-                o = sum(h[i] * W2[e][m][i] for i in range(c.I)) + b2[m]
+                if i8:
+                    o = dot_i8(inp.fc2_w[e][m], S2[e][m], c.I, c.bits, c.block_size, qh, sh_) + b2[m]
+                else:
+                    o = sum(h[i] * W2[e][m][i] for i in range(c.I)) + b2[m]
                 y[t, m] += w[j] * o
         if sh is not None:
             y[t] += sh[t]

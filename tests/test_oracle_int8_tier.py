@@ -21,6 +21,7 @@ import numpy as np
 import pytest
 
 import oracle
+from oracle import literal
 from weight_only_quantized_warp_b200 import inputs as gen
 
 
@@ -178,3 +179,35 @@ def test_int8_tier_stays_close_to_the_float_tier():
     yf = oracle.forward(dataclasses.replace(inp, cfg=dataclasses.replace(cfg, compute_mode=0)))["y"]
     rel = np.abs(y8 - yf).max() / np.abs(yf).max()
     assert 0 < rel < 0.03
+
+
+LITERAL_TIER_CASES = [
+    dict(),
+    dict(bits=8, block_size=16, fusion=2, has_fc1_bias=True, has_fc2_bias=True),
+    dict(fusion=0, has_fc3=True, act=gen.ACT_SILU, has_fc3_bias=True, has_shared=True),
+    dict(act_dtype=gen.DT_BF16, scale_dtype=gen.DT_BF16, k=3, E=5),
+    dict(act_dtype=gen.DT_BF16, scale_dtype=gen.DT_BF16, fusion=0, act=gen.ACT_GELU, bits=8),
+]
+
+
+@pytest.mark.parametrize("kw", LITERAL_TIER_CASES, ids=[str(i) for i in range(len(LITERAL_TIER_CASES))])
+def test_forward_matches_the_literal_restatement(kw):
+    # the Python-float restatement (numpy float32 rounding decisions, integer
+    # dots, bf16 rounding by exact scaling) against the C oracle
+    cfg = _tier_cfg(**{"T": 4, "H": 32, "I": 16, "block_size": 16, **kw})
+    inp = gen.make_inputs(cfg, seed=34, bias_std=0.1)
+    a = oracle.forward(inp)
+    b = literal.forward(inp)
+    np.testing.assert_array_equal(a["topk_idx"], b["topk_idx"])
+    np.testing.assert_allclose(a["y"], b["y"], rtol=1e-12, atol=1e-12 * np.abs(b["y"]).max())
+
+
+def test_literal_rounding_equals_the_oracle_rounding():
+    rng = np.random.default_rng(35)
+    x = (rng.standard_normal((6, 64)) * np.exp(rng.uniform(-8, 8, size=(6, 1)))).astype(np.float32)
+    x[2, :16] = 0.0
+    q, s = oracle.quantize_i8(x, 16)
+    for r in range(6):
+        lq, ls = literal.quantize_row(x[r].astype(np.float64).tolist(), 16)
+        np.testing.assert_array_equal(q[r], lq)
+        np.testing.assert_array_equal(s[r], np.array(ls, dtype=np.float32))
