@@ -80,6 +80,21 @@ def config_of(cfg, name, world):
             "l2": "no flush: the expert weights a step streams exceed the 126 MB L2"}
 
 
+def launch_names(path, launches, weights_on_input):
+    """Names of the forward's launches in order, for a path and the launch
+    count the library reports: routing and permutation (one launch or two),
+    the row gather (tensor-core paths, or router weights on the input), the
+    int8 tier's two rounding launches, FC1, FC2 and the combine."""
+    from weight_only_quantized_warp_b200 import qmoe
+    gather = path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE) or weights_on_input
+    ffn = ["quantize_x", "fc1", "quantize_h", "fc2"] if path == qmoe.PATH_INT8 else ["fc1", "fc2"]
+    routing = launches - int(gather) - len(ffn) - 1
+    if routing not in (1, 2):
+        raise ValueError(f"{launches} launches do not fit path {path}")
+    return ((["route_permute"] if routing == 1 else ["route", "permute"]) + (["gather"] if gather else [])
+            + ffn + ["combine"])
+
+
 def algorithmic(cfg, offsets):
     """Algorithmic bytes / FLOPs of one forward, from the routing (experts
     with at least one routed row count once)."""
@@ -330,12 +345,8 @@ def run_ours(args):
     per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(launches)]
                            for i in range(K)]).mean(axis=0)
     path = qmoe.qmoe_path_for(h, T)
-    gather = path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE) or bool(cfg.apply_router_weight_on_input)
     i8 = path == qmoe.PATH_INT8
-    ffn = ["quantize_x", "fc1", "quantize_h", "fc2"] if i8 else ["fc1", "fc2"]
-    fused = launches - int(gather) - len(ffn) - 1 == 1  # routing and permutation in one launch
-    names = ((["route_permute"] if fused else ["route", "permute"]) + (["gather"] if gather else [])
-             + ffn + ["combine"])
+    names = launch_names(path, launches, bool(cfg.apply_router_weight_on_input))
 
     # ---- end to end through the public call, host buffers, copies inside
     x_h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu())

@@ -208,3 +208,30 @@ def test_quantize_entry_rejects_bad_dtype_alignment_and_null(q):
     assert q.lib.qmoe_quantize_act_i8(256, q.DTYPE_BF16, 1, 64, 16, 258, 256, None) == q.QMOE_INVALID_ARGUMENT
     assert q.lib.qmoe_quantize_act_i8(None, q.DTYPE_BF16, 1, 64, 16, 256, 256, None) == q.QMOE_INVALID_ARGUMENT
     assert q.lib.qmoe_quantize_act_i8(None, q.DTYPE_BF16, 0, 64, 16, None, None, None) == q.QMOE_OK  # no rows
+
+
+@pytest.mark.parametrize("kw,T,path", [
+    (dict(), 8, 1), (dict(), 65, 2), (dict(), 4096, 2),
+    (dict(compute_mode=1), 8, 4), (dict(compute_mode=1), 300, 4),
+    (dict(compute_mode=1, apply_router_weight_on_input=1), 8, 4),
+    (dict(apply_router_weight_on_input=1), 8, 1),
+    (dict(act_dtype=0, scale_dtype=0), 8, 0), (dict(act_dtype=0, scale_dtype=0), 100, 0),
+])
+def test_bench_launch_names_match_the_plan(q, kw, T, path):
+    # the benchmark's per-kernel labels follow the library's own launch count
+    import bench
+    h = q.qmoe_create(_cfg(q, **kw))
+    try:
+        assert q.qmoe_path_for(h, T) == path
+        n = q.qmoe_launches_for(h, T)
+        names = bench.launch_names(path, n, bool(kw.get("apply_router_weight_on_input")))
+        assert len(names) == n
+        assert names[-1] == "combine" and names.index("fc1") < names.index("fc2")
+        assert ("route_permute" in names) == (T <= 64)
+        assert ("quantize_x" in names) == (path == q.PATH_INT8)
+        assert ("gather" in names) == (path in (q.PATH_TC, q.PATH_TC_DECODE) or
+                                       bool(kw.get("apply_router_weight_on_input")))
+    finally:
+        q.qmoe_destroy(h)
+    with pytest.raises(ValueError):
+        bench.launch_names(path, 99, False)
