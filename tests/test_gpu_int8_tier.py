@@ -226,3 +226,17 @@ def test_int8_tier_full_size_decode(cuda_device, T):
     tokens = np.arange(T) if T <= 8 else np.sort(np.random.default_rng(T).choice(T, 8, replace=False))
     err = check_sampled(inp, g, tokens)
     assert err <= TOL_Y
+
+
+@pytest.mark.parametrize("bits,T", [(8, 16), (4, 128)])
+def test_int8_tier_full_size_sweep_shapes(cuda_device, bits, T):
+    # the sweep's H=4096, I=14336 shapes on the int8 tier: int8 codes with
+    # 128-code blocks, and int4 with 64-code blocks at 32 rows per expert
+    # (two passes of the two-tile kernel)
+    cfg, seed, kw = gen.sweep(bits, T)
+    cfg.compute_mode = gen.COMPUTE_INT8_BLOCK
+    inp = gen.make_inputs(cfg, seed, **kw)
+    g = run_gpu(inp)
+    assert g.path == PATH_INT8
+    tokens = np.sort(np.random.default_rng(seed).choice(T, 4, replace=False))
+    assert check_sampled(inp, g, tokens) <= TOL_Y
