@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -126,7 +127,9 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        # raw samples: QMOE_CLOCKS_DIR if set, else the system temp directory
+        folder = os.environ.get("QMOE_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(folder, f"clocks_bench_{os.getpid()}.csv")
 
     def start(self):
         try:
