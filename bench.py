@@ -283,7 +283,10 @@ def run_ours(args):
     # one step = one forward, replayed from a CUDA graph (the forward enqueues
     # only stream-ordered device work, so it captures as is)
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):  # captures on a side stream; replays on `stream`
+    # captures on a side stream and replays on `stream`; thread-local capture
+    # so that other threads' CUDA calls (a process group's watchdog) are not
+    # treated as part of the capture
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
         qmoe.qmoe_forward(h, T, x, lg, sh, y, ws, nws, torch.cuda.current_stream())
     for _ in range(3):
         graph.replay()
