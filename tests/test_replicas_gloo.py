@@ -67,7 +67,7 @@ def _rank_main(rank, world, port, workload, out_dir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("workload", ["tiny"])
+@pytest.mark.parametrize("workload", ["tiny", "tiny_i8"])
 def test_two_gloo_replicas_equal_one_batch(tmp_path, workload):
     import oracle
     from weight_only_quantized_warp_b200 import inputs as gen

@@ -216,6 +216,14 @@ def tiny():
     return cfg, 1, dict(logits="normal", logit_std=1.0, tiny_scales=True)
 
 
+def tiny_i8():
+    """The tiny shape on the int8 block compute tier (64-code blocks)."""
+    cfg = MoEConfig(T=16, H=128, I=128, E=4, k=2, bits=4, block_size=64,
+                    act=ACT_SWIGLU, fusion=1, limit=math.inf, normalize=True,
+                    act_dtype=DT_F32, scale_dtype=DT_F32, compute_mode=COMPUTE_INT8_BLOCK)
+    return cfg, 6, dict(logits="normal", logit_std=1.0, tiny_scales=True)
+
+
 def mixtral_decode(T: int = 8):
     cfg = MoEConfig(T=T, H=4096, I=14336, E=8, k=2, bits=4, block_size=128,
                     act=ACT_SWIGLU, fusion=2, normalize=True,
@@ -269,6 +277,7 @@ def sweep(bits: int, T: int):
 
 WORKLOADS = {
     "tiny": tiny,
+    "tiny_i8": tiny_i8,
     "mixtral_decode": mixtral_decode,
     "mixtral_decode_i8": mixtral_decode_i8,
     "gpt_oss": gpt_oss,
