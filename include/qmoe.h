@@ -199,12 +199,18 @@ QMOE_API size_t qmoe_workspace_size(const qmoe_handle* h, int64_t T);
 /*
  * qmoe_forward -- "ClikaRT::nn::QMoEWoQ", forward(): one MoE step.
  *
- *   x              [T, H] act_dtype
- *   router_logits  [T, E] act_dtype (logits; softmax is applied inside)
- *   shared_output  [T, H] act_dtype or NULL (folded into the combine)
- *   y              [T, H] act_dtype (written)
+ *   x              [T, H] act_dtype, 16-byte aligned
+ *   router_logits  [T, E] act_dtype (logits; softmax is applied inside),
+ *                  aligned to its element size
+ *   shared_output  [T, H] act_dtype or NULL (folded into the combine),
+ *                  16-byte aligned
+ *   y              [T, H] act_dtype (written), 16-byte aligned
  *   workspace      >= qmoe_workspace_size(h, T) bytes, 256-byte aligned,
  *                  owned by the caller; contents on entry are ignored
+ *
+ * For T > 0 a NULL required pointer or a misaligned one is
+ * QMOE_INVALID_ARGUMENT, checked before the handle's binding
+ * (QMOE_NOT_BOUND).
  *
  * Enqueues all work on `stream` and returns without waiting; it never
  * synchronises the host. The handle is only read, so concurrent calls on

@@ -235,3 +235,21 @@ def test_bench_launch_names_match_the_plan(q, kw, T, path):
         q.qmoe_destroy(h)
     with pytest.raises(ValueError):
         bench.launch_names(path, 99, False)
+
+
+@pytest.mark.parametrize("x,lg,sh,y,ws,status", [
+    (16, 16, None, 16, 256, 2),       # well-formed: the binding is checked next
+    (24, 16, None, 16, 256, 1),       # x not 16-byte aligned
+    (16, 16, 40, 16, 256, 1),         # shared_output not 16-byte aligned
+    (16, 16, None, 8, 256, 1),        # y not 16-byte aligned
+    (16, 17, None, 16, 256, 1),       # bf16 logits on an odd address
+    (16, 16, None, 16, 128, 1),       # workspace not 256-byte aligned
+    (None, 16, None, 16, 256, 1),     # x missing
+])
+def test_forward_argument_checks_precede_the_binding(q, x, lg, sh, y, ws, status):
+    h = q.qmoe_create(_cfg(q))
+    try:
+        assert q.lib.qmoe_forward(h, 4, x, lg, sh, y, ws, 1 << 20, None) == status
+        assert q.lib.qmoe_forward(h, -1, x, lg, sh, y, ws, 1 << 20, None) == q.QMOE_INVALID_ARGUMENT
+    finally:
+        q.qmoe_destroy(h)

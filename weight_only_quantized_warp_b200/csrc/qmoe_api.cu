@@ -417,15 +417,24 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
                                 void* workspace, size_t workspace_bytes, void* stream,
                                 void* const* events, int32_t n_events) {
     if (!h) return QMOE_INVALID_ARGUMENT;
-    if (!h->bound) return fail(h, QMOE_NOT_BOUND, "forward before set_weights bound the weights");
     if (T < 0) return fail(h, QMOE_INVALID_ARGUMENT, "T must be >= 0");
+    if (T > 0) {
+        // the kernels read x and shared_output and write y in 8- and 16-byte
+        // vectors, and the logits element by element
+        auto addr = [](const void* p) { return reinterpret_cast<uintptr_t>(p); };
+        const uintptr_t act_bytes = h->cfg.act_dtype == QMOE_DTYPE_BF16 ? 2 : 4;
+        if (!x || !router_logits || !y || !workspace)
+            return fail(h, QMOE_INVALID_ARGUMENT, "x, router_logits, y and workspace are required");
+        if ((addr(x) | addr(y) | addr(shared_output)) & 15)
+            return fail(h, QMOE_INVALID_ARGUMENT, "x, shared_output and y must be 16-byte aligned");
+        if (addr(router_logits) & (act_bytes - 1))
+            return fail(h, QMOE_INVALID_ARGUMENT, "router_logits must be aligned to its element size");
+        if (addr(workspace) & 255) return fail(h, QMOE_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
+    }
+    if (!h->bound) return fail(h, QMOE_NOT_BOUND, "forward before set_weights bound the weights");
     if (T == 0) return QMOE_OK;
-    if (!x || !router_logits || !y || !workspace)
-        return fail(h, QMOE_INVALID_ARGUMENT, "x, router_logits, y and workspace are required");
     if (T * h->cfg.k >= (int64_t(1) << 31))
         return fail(h, QMOE_UNSUPPORTED, "T * k must stay below 2^31");
-    if (reinterpret_cast<uintptr_t>(workspace) & 255)
-        return fail(h, QMOE_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
     const Plan p = make_plan(*h, T);
     if (!p.ok)
         return fail(h, QMOE_UNSUPPORTED, "no kernel configuration fits this shape (hidden_size too large)");
