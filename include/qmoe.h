@@ -177,7 +177,9 @@ QMOE_API qmoe_status qmoe_create(const qmoe_config* cfg, qmoe_handle** out);
  *   fc3_w  [E, I, H*bits/8], fc3_s like fc1_s with I rows; required iff has_fc3
  *   fc3_b  [E, I]; required iff has_fc3_bias
  *
- * All pointers are device pointers. The call re-lays the packed bytes into the
+ * All pointers are device pointers; scales and biases aligned to their
+ * element size (QMOE_INVALID_ARGUMENT otherwise), codes at any address. The
+ * call re-lays the packed bytes into the
  * kernels' tile order in handle-owned device memory of the same size (the
  * weights stay quantized; this copy is the one resident copy), waits for that
  * work on `stream`, and returns; the caller may then free its buffers. A

@@ -149,6 +149,11 @@ def test_set_weights_argument_errors_precede_device_work(q):
         assert q.lib.qmoe_set_weights(h, a, a, a, a, a, a, None, None, None, None) == 1
         # fc3 given without has_fc3
         assert q.lib.qmoe_set_weights(h, a, a, a, a, a, None, a, a, None, None) == 1
+        # bf16 scales or bias on an odd address; codes may sit anywhere
+        assert q.lib.qmoe_set_weights(h, a, a + 1, a, a, a, None, None, None, None, None) == 1
+        assert b"scales" in q.lib.qmoe_last_error(h)
+        assert q.lib.qmoe_set_weights(h, a, a, a + 1, a, a, None, None, None, None, None) == 1
+        assert b"biases" in q.lib.qmoe_last_error(h)
         assert b"bias" in q.lib.qmoe_last_error(h) or b"fc3" in q.lib.qmoe_last_error(h)
     finally:
         q.qmoe_destroy(h)

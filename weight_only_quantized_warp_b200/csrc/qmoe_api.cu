@@ -293,6 +293,16 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
         return fail(h, QMOE_INVALID_ARGUMENT, "fc3 weights and scales must be given iff has_fc3");
     if (bool(fc3_b) != bool(c.has_fc3_bias))
         return fail(h, QMOE_INVALID_ARGUMENT, "fc3 bias must be given iff has_fc3_bias");
+    {
+        // the pack reads codes byte by byte, scales and biases element by element
+        const uintptr_t s_align = c.scale_dtype == QMOE_DTYPE_F32 ? 4 : (c.scale_dtype == QMOE_DTYPE_BF16 ? 2 : 1);
+        const uintptr_t b_align = c.act_dtype == QMOE_DTYPE_F32 ? 4 : 2;
+        auto addr = [](const void* p) { return reinterpret_cast<uintptr_t>(p); };
+        if ((addr(fc1_s) | addr(fc2_s) | addr(fc3_s)) & (s_align - 1))
+            return fail(h, QMOE_INVALID_ARGUMENT, "scales must be aligned to their element size");
+        if ((addr(fc1_b) | addr(fc2_b) | addr(fc3_b)) & (b_align - 1))
+            return fail(h, QMOE_INVALID_ARGUMENT, "biases must be aligned to their element size");
+    }
 
     cudaStream_t st = (cudaStream_t)stream;
     int dev = 0;
