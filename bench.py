@@ -1,26 +1,34 @@
 """Benchmark of the QMoE forward on B200 (one JSON line on rank 0).
 
-Default workload: Mixtral-like decode (T=8, H=4096, I=14336, E=8, k=2, int4
-block_size 128, bf16 activations and scales, swiglu fused not interleaved,
-renormalised routing), seeded synthetic inputs. One step = one whole forward
-(routing, permutation, FC1 + SwiGLU, FC2, combine) over the batch, launched
-as one CUDA graph replay; the JSON line also gives the step time with direct
-launches, the per-kernel times of a separate event-bracketed pass, and the
-end-to-end rate through the public call with host buffers.
+Headline workload: the prefill sweep's largest shape (T=8192, H=4096,
+I=14336, E=8, k=2, int4 block_size 64, bf16 activations and scales, swiglu
+fused not interleaved, renormalised uniform-random routing), the largest
+single-GPU configuration, bound by the tensor cores. The same line carries
+the decode half of the metric as a nested record (Mixtral-like decode: T=8,
+int4 block_size 128, bound by HBM bandwidth) with its own roofline, per-kernel
+times and clocks, and the decode-to-compute crossover measured over T on the
+headline's weights. Inputs are seeded synthetic draws of the shapes; no
+trained weights.
+
+One step = one whole forward (routing, permutation, row gather, FC1 + SwiGLU,
+FC2, combine) over the batch, launched as one CUDA graph replay. The line
+also gives the step time with direct launches, the per-kernel times of a
+separate event-bracketed pass, and the end-to-end rate through the public
+call with host buffers copied in and out inside the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle, timed on host cores
 
-With N > 1 (torchrun) every rank runs an independent replica on its own
-token batch (tokens are independent; no collective on the data path) and the
-job throughput is all ranks' tokens over the slowest rank's time.
+With N > 1 (torchrun) every rank runs an independent replica of the headline
+workload on its own token batch (tokens are independent; no collective on the
+data path) and the job throughput is all ranks' tokens over the slowest
+rank's time; the nested decode record and the crossover run at N = 1 only.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -36,6 +44,9 @@ sys.path.insert(0, ROOT)
 from weight_only_quantized_warp_b200 import inputs as gen  # noqa: E402
 
 METRIC = "QMoE fwd tokens/s; HBM GB/s (decode) / TFLOP/s (prefill) vs roofline"
+HEADLINE = "sweep_int4_T8192"
+DECODE = "mixtral_decode"
+CROSSOVER_T = (1, 16, 64, 128, 256, 512, 1024, 2048, 4096, 8192)
 L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -45,14 +56,17 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mixtral_decode")
+    ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", type=int, default=None,
                     help="force the expert-FFN kernels: 1 mma.sync streaming, 2 tcgen05 GEMM, "
                          "3 tcgen05 streaming (default: by shape)")
+    ap.add_argument("--decode-workload", default=DECODE,
+                    help="workload of the nested decode record ('none' to skip)")
+    ap.add_argument("--no-crossover", action="store_true", help="skip the crossover sweep over T")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0,
-                    help="tokens in the CPU-baseline sample (0: whole batch, capped by time)")
+                    help="tokens per oracle call in the CPU-baseline sample (0: 32, capped by the batch)")
     return ap.parse_args()
 
 
@@ -65,6 +79,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -72,13 +97,21 @@ def dist_env():
     return ws, rank, local
 
 
-def config_of(cfg, name, world):
-    return {"workload": name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
-            "bits": cfg.bits, "block_size": cfg.block_size, "swiglu_fusion": cfg.fusion,
-            "act_dtype": "bf16" if cfg.act_dtype == gen.DT_BF16 else "f32",
-            "compute": "int8 block tier" if cfg.compute_mode == gen.COMPUTE_INT8_BLOCK else "float",
-            "tokens_per_step": cfg.T * world, "parallelism": f"replicas x{world}",
-            "l2": "no flush: the expert weights a step streams exceed the 126 MB L2"}
+def l2_note(alg):
+    if alg["weight_bytes"] > L2_BYTES:
+        return "no flush: the expert weights a step streams exceed the 126 MB L2"
+    return "weights fit L2 (not flushed between steps)"
+
+
+def config_of(cfg, name, world, alg=None):
+    d = {"workload": name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+         "bits": cfg.bits, "block_size": cfg.block_size, "swiglu_fusion": cfg.fusion,
+         "act_dtype": "bf16" if cfg.act_dtype == gen.DT_BF16 else "f32",
+         "compute": "int8 block tier" if cfg.compute_mode == gen.COMPUTE_INT8_BLOCK else "float",
+         "tokens_per_step": cfg.T * world, "parallelism": f"replicas x{world}"}
+    if alg is not None:
+        d["l2"] = l2_note(alg)
+    return d
 
 
 def launch_names(path, launches, weights_on_input):
@@ -111,10 +144,32 @@ def algorithmic(cfg, offsets):
     R = cfg.T * cfg.k
     act_fc1 = cfg.T * cfg.H * asz + R * cfg.I * asz                # x in, h out
     io = cfg.T * cfg.H * asz * (2 + int(cfg.has_shared)) + cfg.T * cfg.E * asz
-    flops = 2 * R * 3 * cfg.H * cfg.I if (cfg.fusion or cfg.has_fc3) else 2 * R * 2 * cfg.H * cfg.I
+    gated = cfg.fusion or cfg.has_fc3
+    flops = 2 * R * 3 * cfg.H * cfg.I if gated else 2 * R * 2 * cfg.H * cfg.I
+    fc1_flops = 2.0 * R * n1 * cfg.H
     return dict(touched=touched, fc1_bytes=touched * fc1 + act_fc1, fc2_bytes=touched * fc2,
-                total_bytes=touched * (fc1 + fc2) + io, flops=flops,
-                fc1_per_expert=fc1, fc2_per_expert=fc2)
+                total_bytes=touched * (fc1 + fc2) + io, weight_bytes=touched * (fc1 + fc2), flops=flops,
+                fc1_flops=fc1_flops, fc1_per_expert=fc1, fc2_per_expert=fc2)
+
+
+def roofline_of(cfg, alg, fc1_ms, peaks, peaks_kind, kname, traffic):
+    """Roofline record of the FC1 launch: the slower of its algorithmic bytes
+    at the measured HBM bandwidth and its FLOPs at the burst bf16 peak binds."""
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"])
+    t_hbm = alg["fc1_bytes"] / (hbm_peak * 1e9)
+    t_tc = alg["fc1_flops"] / (tc_peak * 1e12)
+    if t_hbm >= t_tc:
+        achieved = alg["fc1_bytes"] / (fc1_ms / 1e3) / 1e9
+        r = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+             "frac": achieved / hbm_peak, "algorithmic_bytes": alg["fc1_bytes"]}
+    else:
+        achieved = alg["fc1_flops"] / (fc1_ms / 1e3) / 1e12
+        r = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+             "frac": achieved / tc_peak, "algorithmic_flops": alg["fc1_flops"]}
+    r.update({"kernel": kname, "peak_kind": peaks_kind + (" (burst bf16)" if r["bound"] == "tensor" else ""),
+              "traffic": traffic["bytes_per_launch"] if traffic else None, "avg_launch_ms": fc1_ms})
+    return r
 
 
 class ClockSampler:
@@ -124,12 +179,12 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
+    def __init__(self, index, tag="bench"):
         self.index = index
         self.proc = None
         # raw samples: QMOE_CLOCKS_DIR if set, else the system temp directory
         folder = os.environ.get("QMOE_CLOCKS_DIR") or tempfile.gettempdir()
-        self.path = os.path.join(folder, f"clocks_bench_{os.getpid()}.csv")
+        self.path = os.path.join(folder, f"clocks_{tag}_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -160,11 +215,13 @@ class ClockSampler:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "power_w_median": statistics.median(pw) if pw else None}
 
 
 def traffic_record(kernel_key):
@@ -187,6 +244,13 @@ def source_digest(sources):
         with open(os.path.join(ROOT, "weight_only_quantized_warp_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def fc1_kernel_name(qmoe, path, tile):
+    if path == qmoe.PATH_TC:
+        return "ffn_tc_wide_kernel" if tile > 128 else "ffn_tc_kernel"
+    return {qmoe.PATH_TC_DECODE: "ffn_tc_decode_kernel", qmoe.PATH_SIMT: "ffn_simt_kernel",
+            qmoe.PATH_INT8: "ffn_i8_kernel"}.get(path, "ffn_decode_kernel")
 
 
 # ---------------------------------------------------------------- reference arm
@@ -225,7 +289,7 @@ def run_reference(args):
         oracle.forward(inp, tokens=s)
         times.append(time.perf_counter() - t0)
     total = sum(times)
-    tok = ntok * args.steps
+    tok = len(samples[0]) * args.steps
     value = tok / total
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -233,8 +297,8 @@ def run_reference(args):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "config": config_of(cfg, args.workload, 1),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
-                             "kind": "oracle",
-                             "sample": f"{ntok} token(s) of the {cfg.T}-token batch per step"},
+                             "cpu_model": cpu_model(), "kind": "oracle",
+                             "sample": f"{len(samples[0])} token(s) of the {cfg.T}-token batch per step"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -242,6 +306,174 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------- our arm
+
+class Bound:
+    """One operator instance with its device inputs, workspace and a graph of
+    one forward."""
+
+    def __init__(self, inp, dev, path=None, m=None):
+        import torch
+        from weight_only_quantized_warp_b200 import qmoe
+        self.qmoe, self.torch = qmoe, torch
+        self.inp, self.cfg, self.dev = inp, inp.cfg, dev
+        if m is None:
+            m = qmoe.QMoE(inp.cfg, dev, path=path)
+            m.set_weights_from(inp)
+        self.m = m
+        self.h = m.handle
+        self.x = qmoe.to_device(inp.x, dev)
+        self.lg = qmoe.to_device(inp.logits, dev)
+        self.sh = qmoe.to_device(inp.shared, dev)
+        self.y = torch.empty_like(self.x)
+        self.T = inp.cfg.T
+        self.ws = m.workspace(self.T)
+        self.nws = self.ws.numel()
+        self.launches = qmoe.qmoe_launches_for(self.h, self.T)
+        self.path = qmoe.qmoe_path_for(self.h, self.T)
+        self.tile = qmoe.qmoe_token_tile_for(self.h, self.T)
+        self.graph = None
+
+    def fwd(self, stream):
+        self.qmoe.qmoe_forward(self.h, self.T, self.x, self.lg, self.sh, self.y, self.ws, self.nws, stream)
+
+    def capture(self):
+        torch = self.torch
+        self.graph = torch.cuda.CUDAGraph()
+        # captures on a side stream and replays on the current one;
+        # thread-local capture so that other threads' CUDA calls (a process
+        # group's watchdog) are not treated as part of the capture
+        with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
+            self.fwd(torch.cuda.current_stream())
+
+    def release(self):
+        self.graph = None
+
+    def offsets(self):
+        torch = self.torch
+        off = torch.empty(self.cfg.E + 1, dtype=torch.int32, device=self.dev)
+        self.qmoe.qmoe_debug_routing(self.h, self.T, self.ws, offsets=off)
+        return off.cpu().numpy()
+
+    def per_kernel_ms(self, stream, n):
+        torch = self.torch
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(self.launches + 1)] for _ in range(n)]
+        for row in evs:
+            for e in row:
+                e.record(stream)  # materialise the event handles
+        torch.cuda.synchronize()
+        for i in range(n):
+            self.qmoe.qmoe_forward_profiled(self.h, self.T, self.x, self.lg, self.sh, self.y, self.ws, self.nws,
+                                            evs[i], stream)
+        torch.cuda.synchronize()
+        per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(self.launches)]
+                        for i in range(n)]).mean(axis=0)
+        names = launch_names(self.path, self.launches, bool(self.cfg.apply_router_weight_on_input))
+        return dict(zip(names, [float(v) for v in per]))
+
+
+def timed_replays(b, stream, K, local, world, clocks_tag=None, dist=None):
+    """K graph replays bracketed by events (and a barrier with N > 1); the
+    clock sampler brackets the region with the same forward under load."""
+    import torch
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local, clocks_tag) if clocks_tag else None
+
+    def keep_loaded(seconds):
+        t_end = time.perf_counter() + seconds
+        while time.perf_counter() < t_end:
+            for _ in range(5):
+                b.graph.replay()
+            torch.cuda.synchronize()
+
+    if clocks:
+        clocks.start()
+        keep_loaded(0.6)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(K):
+        b.graph.replay()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    clk = None
+    if clocks:
+        keep_loaded(0.4)
+        clk = clocks.stop()
+        if clk is not None:
+            clk["window"] = "timed region bracketed by 0.6 s / 0.4 s of the same forward"
+    return start.elapsed_time(stop), clk
+
+
+def measure_record(b, stream, K, warmup, local, peaks, peaks_kind, workload, clocks_tag):
+    """Graph-timed step, per-kernel times and the FC1 roofline of one bound
+    workload at N = 1 (the nested decode record and the crossover points)."""
+    import torch
+    for _ in range(max(warmup, 3)):
+        b.fwd(stream)
+    torch.cuda.synchronize()
+    b.capture()
+    for _ in range(3):
+        b.graph.replay()
+    torch.cuda.synchronize()
+    alg = algorithmic(b.cfg, b.offsets())
+    ms, clk = timed_replays(b, stream, K, local, 1, clocks_tag)
+    kms = b.per_kernel_ms(stream, min(K, 10))
+    b.release()
+    step_ms = ms / K
+    kbase = fc1_kernel_name(b.qmoe, b.path, b.tile)
+    rl = roofline_of(b.cfg, alg, kms["fc1"], peaks, peaks_kind, kbase + " (FC1 + activation)",
+                     traffic_record("fc1_" + kbase + "_" + workload))
+    hbm_peak, tc_peak = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    t_roof = max(alg["total_bytes"] / (hbm_peak * 1e9), alg["flops"] / (tc_peak * 1e12))
+    return {"workload": workload, "T": b.T, "value": b.T / (step_ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": step_ms, "steps": K, "roofline": rl,
+            "step": {"hbm_gbs": alg["total_bytes"] / (step_ms / 1e3) / 1e9,
+                     "tflops": alg["flops"] / (step_ms / 1e3) / 1e12,
+                     "roofline_frac_of_step": t_roof / (step_ms / 1e3),
+                     "experts_touched": alg["touched"], "algorithmic_bytes": alg["total_bytes"],
+                     "kernel_ms": kms, "path": b.path, "token_tile": b.tile,
+                     "launch": "CUDA graph of one forward per step"},
+            "gpu_launches": b.launches * K, "clocks": clk, "l2": l2_note(alg)}
+
+
+def crossover(head_inp, m, dev, stream, peaks, peaks_kind, ts=CROSSOVER_T):
+    """Step time over T on the headline's weights (token batches of each T
+    from their own seeds): the flat part is bound by streaming the touched
+    experts' weights, the rising part by the tensor cores. The measured
+    crossover is where the compute line through the two largest T meets the
+    streaming floor (the mean step time of the T <= 128 points)."""
+    import torch
+    cfg0 = head_inp.cfg
+    pts = []
+    for T in ts:
+        cfg = gen.MoEConfig(**{**cfg0.__dict__, "T": T})
+        x, lg, sh = gen.make_token_batch(cfg, 5000 + T, logits="uniform")
+        inp = gen.MoEInputs(cfg, x, lg, head_inp.fc1_w, head_inp.fc1_s, head_inp.fc2_w, head_inp.fc2_s,
+                            shared=sh)
+        b = Bound(inp, dev, m=m)
+        K = 20 if T <= 1024 else 8
+        r = measure_record(b, stream, K, 3, 0, peaks, peaks_kind, f"crossover_T{T}", None)
+        pts.append({"T": T, "ms_per_step": r["ms_per_step"], "tokens_per_s": r["value"],
+                    "fc1_kernel": r["roofline"]["kernel"].split(" ")[0], "fc1_bound": r["roofline"]["bound"],
+                    "fc1_frac": r["roofline"]["frac"], "path": r["step"]["path"], "token_tile": r["step"]["token_tile"],
+                    "step_roofline_frac": r["step"]["roofline_frac_of_step"]})
+        del b
+        torch.cuda.synchronize()
+    floor = float(np.mean([p["ms_per_step"] for p in pts if p["T"] <= 128]))
+    big = sorted(pts, key=lambda p: p["T"])[-2:]
+    slope = (big[1]["ms_per_step"] - big[0]["ms_per_step"]) / (big[1]["T"] - big[0]["T"])
+    icept = big[1]["ms_per_step"] - slope * big[1]["T"]
+    measured = (floor - icept) / slope if slope > 0 else None
+    alg = algorithmic(gen.MoEConfig(**{**cfg0.__dict__, "T": 1}), np.arange(cfg0.E + 1))
+    wbytes = cfg0.E * (alg["fc1_per_expert"] + alg["fc2_per_expert"])
+    per_tok_flops = 2 * cfg0.k * 3 * cfg0.H * cfg0.I
+    model = wbytes * float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9 * per_tok_flops)
+    return {"weights": HEADLINE + " (all T share them)", "points": pts,
+            "streaming_floor_ms": floor, "compute_ms_per_token": slope,
+            "measured_crossover_T": measured, "model_crossover_T": model,
+            "model": "all experts' weight bytes at the HBM peak = T tokens' FLOPs at the bf16 peak"}
+
 
 def run_ours(args):
     import torch
@@ -254,121 +486,61 @@ def run_ours(args):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    peaks, peaks_kind = load_peaks()
 
     # every replica: the same weights, its own token batch
     inp = replicas.replica_inputs(args.workload, rank)
     cfg = inp.cfg
-
-    m = qmoe.QMoE(cfg, dev, path=args.path)
-    m.set_weights_from(inp)
-    x = qmoe.to_device(inp.x, dev)
-    lg = qmoe.to_device(inp.logits, dev)
-    sh = qmoe.to_device(inp.shared, dev)
-    y = torch.empty_like(x)
-    T = cfg.T
-    ws = m.workspace(T)
-    nws = ws.numel()
-    h = m.handle
-    launches = qmoe.qmoe_launches_for(h, T)
+    b = Bound(inp, dev, path=args.path)
+    T, h = b.T, b.h
     stream = torch.cuda.current_stream()
-
-    def fwd():
-        qmoe.qmoe_forward(h, T, x, lg, sh, y, ws, nws, stream)
-
-    # warm-up
-    for _ in range(max(args.warmup, 3)):
-        fwd()
-    torch.cuda.synchronize()
-
-    # one step = one forward, replayed from a CUDA graph (the forward enqueues
-    # only stream-ordered device work, so it captures as is)
-    graph = torch.cuda.CUDAGraph()
-    # captures on a side stream and replays on `stream`; thread-local capture
-    # so that other threads' CUDA calls (a process group's watchdog) are not
-    # treated as part of the capture
-    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
-        qmoe.qmoe_forward(h, T, x, lg, sh, y, ws, nws, torch.cuda.current_stream())
-    for _ in range(3):
-        graph.replay()
-    torch.cuda.synchronize()
-
-    # routing of this batch (for the algorithmic byte count)
-    off = torch.empty(cfg.E + 1, dtype=torch.int32, device=dev)
-    qmoe.qmoe_debug_routing(h, T, ws, offsets=off)
-    alg = algorithmic(cfg, off.cpu().numpy())
-
-    # ---- timed region: K whole forwards, events per kernel on this stream
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(launches + 1)] for _ in range(K)]
-    for row in evs:
-        for e in row:
-            e.record(stream)  # materialise the event handles
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
 
-    def keep_loaded(seconds):
-        # the same forward, back to back, so clock samples bracket the timed
-        # region under its own load (a short region ends between samples)
-        t_end = time.perf_counter() + seconds
-        while time.perf_counter() < t_end:
-            for _ in range(20):
-                graph.replay()
-            torch.cuda.synchronize()
+    for _ in range(max(args.warmup, 3)):
+        b.fwd(stream)
+    torch.cuda.synchronize()
+    b.capture()
+    for _ in range(3):
+        b.graph.replay()
+    torch.cuda.synchronize()
+    alg = algorithmic(cfg, b.offsets())
 
-    clocks.start()
-    keep_loaded(0.6)
-    if world > 1:
-        dist.barrier(device_ids=[local])
-    torch.cuda.synchronize()
-    start.record(stream)
-    for i in range(K):
-        graph.replay()
-    stop.record(stream)
-    torch.cuda.synchronize()
-    keep_loaded(0.4)
-    clk = clocks.stop()
-    if clk is not None:
-        clk["window"] = "timed region bracketed by 0.6 s / 0.4 s of the same forward"
-    ms = replicas.max_over_ranks([start.elapsed_time(stop)], dev)[0]
+    # ---- timed region: K graph replays of the whole forward
+    ms, clk = timed_replays(b, stream, K, local, world, "headline", dist)
+    ms = replicas.max_over_ranks([ms], dev)[0]
     if world > 1:
         dist.barrier(device_ids=[local])
 
-    # after the timed region: the same K steps as direct launches, and once
-    # more with an event between kernels for the per-kernel times (the events
+    # after the timed region: the same K steps as direct launches, and a
+    # pass with an event between kernels for the per-kernel times (the events
     # themselves add a few microseconds per launch)
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s0.record(stream)
-    for i in range(K):
-        fwd()
+    for _ in range(K):
+        b.fwd(stream)
     s1.record(stream)
-    for i in range(K):
-        qmoe.qmoe_forward_profiled(h, T, x, lg, sh, y, ws, nws, evs[i], stream)
     torch.cuda.synchronize()
     stream_ms = replicas.max_over_ranks([s0.elapsed_time(s1)], dev)[0]
-    del graph
+    kms = b.per_kernel_ms(stream, min(K, 10))
+    b.release()
     if world > 1:
         dist.barrier(device_ids=[local])
-    per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(launches)]
-                           for i in range(K)]).mean(axis=0)
-    path = qmoe.qmoe_path_for(h, T)
-    i8 = path == qmoe.PATH_INT8
-    names = launch_names(path, launches, bool(cfg.apply_router_weight_on_input))
 
     # ---- end to end through the public call, host buffers, copies inside
-    x_h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu())
-    lg_h = torch.empty(lg.shape, dtype=lg.dtype, pin_memory=True).copy_(lg.cpu())
-    sh_h = None if sh is None else torch.empty(sh.shape, dtype=sh.dtype, pin_memory=True).copy_(sh.cpu())
-    y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-    x_d, lg_d = torch.empty_like(x), torch.empty_like(lg)
-    sh_d = None if sh is None else torch.empty_like(sh)
+    x_h = torch.empty(b.x.shape, dtype=b.x.dtype, pin_memory=True).copy_(b.x.cpu())
+    lg_h = torch.empty(b.lg.shape, dtype=b.lg.dtype, pin_memory=True).copy_(b.lg.cpu())
+    sh_h = None if b.sh is None else torch.empty(b.sh.shape, dtype=b.sh.dtype, pin_memory=True).copy_(b.sh.cpu())
+    y_h = torch.empty(b.y.shape, dtype=b.y.dtype, pin_memory=True)
+    x_d, lg_d = torch.empty_like(b.x), torch.empty_like(b.lg)
+    sh_d = None if b.sh is None else torch.empty_like(b.sh)
 
     def e2e_step():
         x_d.copy_(x_h, non_blocking=True)
         lg_d.copy_(lg_h, non_blocking=True)
         if sh_d is not None:
             sh_d.copy_(sh_h, non_blocking=True)
-        qmoe.qmoe_forward(h, T, x_d, lg_d, sh_d, y, ws, nws, stream)
-        y_h.copy_(y, non_blocking=True)
+        qmoe.qmoe_forward(h, T, x_d, lg_d, sh_d, b.y, b.ws, b.nws, stream)
+        y_h.copy_(b.y, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
@@ -386,70 +558,65 @@ def run_ours(args):
         0 if sh_h is None else sh_h.numel() * sh_h.element_size())
     d2h = y_h.numel() * y_h.element_size()
 
-    # ---- CPU baseline (rank 0, N = 1 only)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ntok = args.cpu_sample_tokens or min(T, 8)
-        rng = np.random.default_rng(1)
-        toks = sorted(rng.choice(T, size=ntok, replace=False).tolist())
-        v, el, done, cores = cpu_oracle_timing(inp, toks)
-        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{done} tokens ({ntok} per call) of the {T}-token batch, {el:.1f} s"}
-
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    peaks, peaks_kind = load_peaks()
-    kms = dict(zip(names, [float(v) for v in per_kernel]))
-    fc1_ms = kms["fc1"]
+    # ---- N = 1 only: the nested decode record and the crossover over T
+    decode = None
+    if world == 1 and args.decode_workload != "none":
+        dinp = replicas.replica_inputs(args.decode_workload, 0)
+        db = Bound(dinp, dev)
+        decode = measure_record(db, stream, max(K, 20), args.warmup, local, peaks, peaks_kind,
+                                args.decode_workload, "decode")
+        decode["config"] = config_of(dinp.cfg, args.decode_workload, 1)
+        del db
+        torch.cuda.synchronize()
+    cross = None
+    if world == 1 and not args.no_crossover and args.workload == HEADLINE:
+        cross = crossover(inp, b.m, dev, stream, peaks, peaks_kind)
+
+    # ---- CPU baseline (rank 0, N = 1 only): the oracle on a bounded sample
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        ntok = min(T, args.cpu_sample_tokens or 32)
+        rng = np.random.default_rng(1)
+        toks = sorted(rng.choice(T, size=ntok, replace=False).tolist())
+        v, el, done, cores = cpu_oracle_timing(inp, toks)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+               "sample": f"{done} tokens ({ntok} per call) of the {T}-token batch, {el:.1f} s"}
+
     step_ms = ms / K
     value = replicas.job_tokens_per_s(T, world, K, ms)
-    # dominant kernel by algorithmic work: FC1 (gate + up rows); its bound is
-    # the slower of its bytes at HBM bandwidth and its FLOPs at bf16 peak
-    hbm_peak = float(peaks["hbm_gbs"])
-    tc_peak = float(peaks["bf16_tflops"])
-    fc1_flops = 2.0 * cfg.T * cfg.k * (cfg.n1 + (cfg.I if cfg.has_fc3 else 0)) * cfg.H
-    t_hbm = alg["fc1_bytes"] / (hbm_peak * 1e9)
-    t_tc = fc1_flops / (tc_peak * 1e12)
-    tile = qmoe.qmoe_token_tile_for(h, T)
-    kbase = ("ffn_tc_wide_kernel" if tile > 128 else "ffn_tc_kernel") if path == qmoe.PATH_TC else \
-        {qmoe.PATH_TC_DECODE: "ffn_tc_decode_kernel", qmoe.PATH_SIMT: "ffn_simt_kernel",
-         qmoe.PATH_INT8: "ffn_i8_kernel"}.get(path, "ffn_decode_kernel")
-    kname = kbase + " (FC1 + activation)"
-    tr = traffic_record("fc1_" + kbase + "_" + args.workload)
-    if t_hbm >= t_tc:
-        achieved = alg["fc1_bytes"] / (fc1_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved / hbm_peak, "algorithmic_bytes": alg["fc1_bytes"]}
-    else:
-        achieved = fc1_flops / (fc1_ms / 1e3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                    "frac": achieved / tc_peak, "algorithmic_flops": fc1_flops}
-    roofline.update({"kernel": kname, "peak_kind": peaks_kind + (" (burst bf16)" if roofline["bound"] == "tensor" else ""),
-                     "traffic": tr["bytes_per_launch"] if tr else None, "avg_launch_ms": fc1_ms,
-                     "roofline_frac_of_step": max(alg["total_bytes"] / (hbm_peak * 1e9),
-                                                  alg["flops"] / (tc_peak * 1e12)) / (ms / K / 1e3)})
-    whole = alg["total_bytes"] / (step_ms / 1e3) / 1e9
+    kbase = fc1_kernel_name(qmoe, b.path, b.tile)
+    roofline = roofline_of(cfg, alg, kms["fc1"], peaks, peaks_kind, kbase + " (FC1 + activation)",
+                           traffic_record("fc1_" + kbase + "_" + args.workload))
+    hbm_peak, tc_peak = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    t_roof = max(alg["total_bytes"] / (hbm_peak * 1e9), alg["flops"] / (tc_peak * 1e12))
+    roofline["roofline_frac_of_step"] = t_roof / (step_ms / 1e3)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "s8" if i8 else ("bf16" if cfg.act_dtype else "f32"),
+            "dtype": "s8" if cfg.compute_mode == gen.COMPUTE_INT8_BLOCK else (
+                "bf16" if cfg.act_dtype == gen.DT_BF16 else "f32"),
             "data": "synthetic (seeded, shapes of the workload; no trained weights)",
-            "config": config_of(cfg, args.workload, world),
+            "config": config_of(cfg, args.workload, world, alg),
             "roofline": roofline,
-            "step": {"hbm_gbs": whole, "tflops": alg["flops"] / (step_ms / 1e3) / 1e12,
-                     "hbm_frac": whole / hbm_peak, "experts_touched": alg["touched"],
-                     "algorithmic_bytes": alg["total_bytes"],
-                     "kernel_ms": kms, "path": path, "token_tile": tile,
+            "step": {"hbm_gbs": alg["total_bytes"] / (step_ms / 1e3) / 1e9,
+                     "tflops": alg["flops"] / (step_ms / 1e3) / 1e12,
+                     "experts_touched": alg["touched"], "algorithmic_bytes": alg["total_bytes"],
+                     "algorithmic_flops": alg["flops"],
+                     "kernel_ms": kms, "path": b.path, "token_tile": b.tile,
                      "launch": "CUDA graph of one forward per step",
                      "ms_per_step_direct_launches": stream_ms / K,
                      "kernel_ms_note": "from a separate pass with an event between kernels"},
+            "decode": decode,
+            "crossover": cross,
             "cpu_baseline": cpu,
-            "e2e": {"value": replicas.job_tokens_per_s(T, world, K, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches * K,
+            "e2e": {"value": replicas.job_tokens_per_s(T, world, K, e2e_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": b.launches * K,
             "clocks": clk}
     print(json.dumps(line), flush=True)
     return 0

@@ -282,7 +282,8 @@ QMOE_API qmoe_status qmoe_read_device_status(const qmoe_handle* h, const void* w
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture. All calls share the one array, which keeps the
+ * before any stream capture (a first call on a capturing stream returns
+ * QMOE_INVALID_ARGUMENT). All calls share the one array, which keeps the
  * last call's contents: calls whose GPU work can overlap (other streams,
  * other host threads) race on it and must be serialised by the caller.
  */
@@ -292,6 +293,16 @@ QMOE_API qmoe_status qmoe_forward_noalloc(const qmoe_handle* h, int64_t T, const
 
 /* Size in bytes of the fixed scratch array behind qmoe_forward_noalloc. */
 QMOE_API size_t qmoe_noalloc_scratch_bytes(void);
+
+/*
+ * qmoe_noalloc_read_device_status -- qmoe_read_device_status for the forward
+ * run by qmoe_forward_noalloc on the current device: wait for `stream`, then
+ * read the device status word in the fixed scratch array (QMOE_OK, or
+ * QMOE_TIMEOUT when a bounded device wait of the last no-alloc forward on
+ * this device gave up). QMOE_INVALID_ARGUMENT if no no-alloc forward has run
+ * on the current device. (No counterpart on the pages.)
+ */
+QMOE_API qmoe_status qmoe_noalloc_read_device_status(const qmoe_handle* h, void* stream);
 
 /* qmoe_destroy -- "ClikaRT::nn::QMoEWoQ", ~QMoEWoQ(): release the packed
  * weights and the handle. NULL is a no-op. */
@@ -326,6 +337,19 @@ QMOE_API qmoe_status qmoe_quantize_act_i8(const void* x, int32_t dtype, int64_t 
  * the fp32 path (0); compute_mode INT8_BLOCK always takes path 4 and ignores
  * this option. */
 enum { QMOE_OPT_PATH = 1 };
+
+/* QMOE_OPT_WAIT_LIMIT_NS: the limit, in nanoseconds, of every bounded
+ * device-side wait of the tcgen05 kernels (paths 2 and 3): 1e5 .. 6e10,
+ * default 2e9. A wait that runs out sets QMOE_TIMEOUT in the workspace status
+ * word (qmoe_read_device_status); every role of the kernel then leaves its
+ * loop, the CTA frees its tensor memory, and the call's later kernels still
+ * run (their results are then undefined).
+ * QMOE_OPT_TEST_WITHHOLD (test support for that failure path; 0 or 1): with
+ * 1, the MMA-issuing warp of each path-2 CTA never announces its first work
+ * item's accumulator, so the epilogue's wait runs out after the limit. No
+ * memory is touched out of place and no copy is left in flight; the next
+ * forward with the option back at 0 is a normal one. */
+enum { QMOE_OPT_WAIT_LIMIT_NS = 2, QMOE_OPT_TEST_WITHHOLD = 3 };
 
 /* qmoe_set_option -- set a tunable option on the handle. QMOE_INVALID_ARGUMENT
  * for an unknown option or value. Not thread-safe against concurrent

@@ -45,20 +45,30 @@ def dense_weight(packed, scales, N, K, bits, bs):
     return W
 
 
+def _nan_as_neg_inf(logits_row):
+    return [-math.inf if math.isnan(v) else v for v in logits_row]
+
+
 def select_experts(logits_row, k):
     """Brute force: the k-subset with the largest logit sum; among equal sums
     the lexicographically smallest sorted id tuple. Returned in list order
-    (logit descending, id ascending)."""
-    E = len(logits_row)
-    best, best_sum = None, -math.inf
+    (logit descending, id ascending). A NaN logit reads as -inf; for the
+    subset sums -inf stands as a finite value below every finite logit, so
+    subsets of -inf members still compare."""
+    vals = _nan_as_neg_inf(logits_row)
+    E = len(vals)
+    floor = min([v for v in vals if math.isfinite(v)] + [0.0]) - 1e6
+    key = [v if v != -math.inf else floor for v in vals]
+    best, best_sum = None, None
     for sub in itertools.combinations(range(E), k):
-        s = sum(logits_row[e] for e in sub)
-        if s > best_sum:
+        s = sum(key[e] for e in sub)
+        if best_sum is None or s > best_sum:
             best, best_sum = sub, s
-    return sorted(best, key=lambda e: (-logits_row[e], e))
+    return sorted(best, key=lambda e: (-key[e], e))
 
 
 def route_weights(logits_row, sel, normalize):
+    logits_row = _nan_as_neg_inf(logits_row)
     m = max(logits_row)
     ex = [math.exp(v - m) for v in logits_row]
     p = [v / sum(ex) for v in ex]

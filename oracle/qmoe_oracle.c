@@ -138,16 +138,19 @@ void oracle_dequant(const uint8_t* packed, const double* scales, int64_t N, int6
 }
 
 /* Routing ("MoE" page summary; QMoE page attributes k and
- * normalize_routing_weights). */
+ * normalize_routing_weights). A NaN logit reads as -inf: it loses to every
+ * number, and among equal values the lower id wins, so every selected index
+ * names an expert. */
 void oracle_route(const double* logits, int64_t T, int64_t E, int64_t k, int32_t normalize,
                   int32_t n_group, int32_t topk_group, int32_t* idx, double* w) {
     char* taken = (char*)malloc((size_t)E);
     char* allowed = (char*)malloc((size_t)E);
     double* p = (double*)malloc(sizeof(double) * (size_t)E);
+    double* l = (double*)malloc(sizeof(double) * (size_t)E);
     const int64_t G = n_group > 1 ? n_group : 1, gsize = E / G;
     char* kept = (char*)malloc((size_t)G);
     for (int64_t t = 0; t < T; ++t) {
-        const double* l = logits + t * E;
+        for (int64_t e = 0; e < E; ++e) l[e] = isnan(logits[t * E + e]) ? -INFINITY : logits[t * E + e];
         /* groups: keep the topk_group groups of largest member logit */
         memset(kept, G == 1, (size_t)G);
         for (int64_t r = 0; G > 1 && r < topk_group; ++r) {
@@ -189,6 +192,7 @@ void oracle_route(const double* logits, int64_t T, int64_t E, int64_t k, int32_t
     free(allowed);
     free(kept);
     free(p);
+    free(l);
 }
 
 /* Token -> expert permutation: segments in expert order, tokens ascending

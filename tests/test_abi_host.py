@@ -159,6 +159,29 @@ def test_set_weights_argument_errors_precede_device_work(q):
         q.qmoe_destroy(h)
 
 
+def test_wait_limit_and_withhold_options_are_validated(q):
+    h = q.qmoe_create(_cfg(q))
+    try:
+        for opt, val in [(q.QMOE_OPT_WAIT_LIMIT_NS, 99999), (q.QMOE_OPT_WAIT_LIMIT_NS, 61 * 10**9),
+                         (q.QMOE_OPT_TEST_WITHHOLD, 2), (q.QMOE_OPT_TEST_WITHHOLD, -1), (99, 0)]:
+            assert q.lib.qmoe_set_option(h, opt, val) == q.QMOE_INVALID_ARGUMENT
+        for opt, val in [(q.QMOE_OPT_WAIT_LIMIT_NS, 10**6), (q.QMOE_OPT_WAIT_LIMIT_NS, 2 * 10**9),
+                         (q.QMOE_OPT_TEST_WITHHOLD, 1), (q.QMOE_OPT_TEST_WITHHOLD, 0)]:
+            assert q.lib.qmoe_set_option(h, opt, val) == q.QMOE_OK
+    finally:
+        q.qmoe_destroy(h)
+
+
+def test_noalloc_status_before_any_noalloc_call(q):
+    # no device is current here, or no no-alloc forward has run: never QMOE_OK
+    h = q.qmoe_create(_cfg(q))
+    try:
+        assert q.lib.qmoe_noalloc_read_device_status(h, None) in (q.QMOE_INVALID_ARGUMENT, q.QMOE_CUDA_ERROR)
+        assert q.lib.qmoe_noalloc_read_device_status(None, None) == q.QMOE_INVALID_ARGUMENT
+    finally:
+        q.qmoe_destroy(h)
+
+
 def test_status_strings(q):
     for s, name in [(0, b"QMOE_OK"), (1, b"QMOE_INVALID_ARGUMENT"), (2, b"QMOE_NOT_BOUND"),
                     (3, b"QMOE_UNSUPPORTED"), (4, b"QMOE_CUDA_ERROR"), (5, b"QMOE_TIMEOUT"),

@@ -15,7 +15,7 @@ import pytest
 
 from weight_only_quantized_warp_b200 import inputs as gen
 
-from gpu_helpers import check_full, check_routing, check_sampled, run_gpu
+from gpu_helpers import boundary_tokens, check_full, check_routing, check_sampled, run_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -78,6 +78,12 @@ CASES = {
                                      beta=1.0, limit=7.0, has_fc1_bias=True, has_fc2_bias=True),
     "wide_tile_int8_percol_fc3_shared": dict(T=520, E=4, k=2, H=256, I=384, bits=8, block_size=0, fusion=0,
                                              has_fc3=True, act=gen.ACT_SILU, normalize=False, has_shared=True),
+    "wide_tile_int8_bs128": dict(T=300, E=2, k=1, H=256, I=384, bits=8, block_size=128),
+    "wide_tile_int8_bs32_bias": dict(T=300, E=2, k=1, H=256, I=384, bits=8, block_size=32, fusion=1,
+                                     has_fc1_bias=True, has_fc2_bias=True),
+    "wide_tile_int8_bs16": dict(T=300, E=2, k=1, H=256, I=384, bits=8, block_size=16),
+    "wide_tile_int4_bs16": dict(T=300, E=2, k=1, H=256, I=384, block_size=16),
+    "wide_tile_int4_bs128_f32scales": dict(T=300, E=2, k=1, H=256, I=384, block_size=128, scale_dtype=gen.DT_F32),
     # routing options of the MoE page
     "grouped_topk": dict(T=40, E=16, k=4, n_group=4, topk_group=2),
     "grouped_topk_one_group_int8": dict(T=33, E=32, k=3, n_group=8, topk_group=1, bits=8, block_size=64),
@@ -120,7 +126,34 @@ def test_parity_small(cuda_device, name, path):
         assert g.path in (PATH_TC_DECODE, PATH_DECODE)
     else:
         assert g.path == path
-    check_full(inp, g)
+    check_full(inp, g, name=f"{name}/path{g.path}")
+
+
+# Every tensor-core kernel instantiation against the oracle: code width x
+# scale mode x token tile (16..128 take the kernel with the decoded weights
+# in tensor memory, 256 the one with them in shared memory), plus MXFP4.
+# The average rows per expert (T * k / E, E = 4, k = 2) picks the tile; the
+# segments vary around it, so several tiles and ragged tails occur.
+TILE_T = {16: 20, 32: 40, 64: 80, 128: 160, 256: 300}
+SCALE_MODES = {"bs16": 16, "bs32": 32, "bs64": 64, "bs128": 128, "percol": 0}
+
+
+@pytest.mark.parametrize("tile", list(TILE_T))
+@pytest.mark.parametrize("scales", list(SCALE_MODES) + ["mxfp4"])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_tensor_core_instantiations(cuda_device, bits, scales, tile):
+    if scales == "mxfp4" and bits == 8:
+        pytest.skip("MXFP4 codes are 4-bit")
+    kw = dict(T=TILE_T[tile], E=4, k=2, H=256, I=384, bits=bits, fusion=1, has_fc1_bias=True, has_fc2_bias=True)
+    if scales == "mxfp4":
+        kw.update(weight_format=gen.WEIGHTS_MXFP4, block_size=32, scale_dtype=gen.DT_E8M0)
+    else:
+        kw.update(block_size=SCALE_MODES[scales])
+    cfg = _cfg(**kw)
+    inp = gen.make_inputs(cfg, seed=300 + tile + 7 * bits + len(scales), bias_std=0.1)
+    g = run_gpu(inp, path=PATH_TC)
+    assert g.path == PATH_TC and g.tile == tile
+    check_full(inp, g, name=f"tc_int{bits}_{scales}_tile{tile}")
 
 
 def test_all_tokens_to_one_expert_and_empty_experts(cuda_device):
@@ -143,6 +176,31 @@ def test_logit_ties_break_to_lowest_id(cuda_device, groups):
     inp.logits = gen.f32_to_bf16_bits(lg)
     g = run_gpu(inp)
     check_full(inp, g)
+
+
+@pytest.mark.parametrize("groups", [(0, 0), (4, 2)], ids=["plain", "4g2"])
+def test_nan_logits_select_real_experts(cuda_device, groups):
+    """NaN logits read as -inf (the oracle's reading): indices stay in range
+    and equal the oracle's; rows with a finite logit keep finite outputs."""
+    cfg = _cfg(T=40, E=16, k=3, n_group=groups[0], topk_group=groups[1])
+    inp = gen.make_inputs(cfg, seed=12)
+    rng = np.random.default_rng(12)
+    lg = rng.standard_normal((cfg.T, cfg.E)).astype(np.float32)
+    lg[rng.random(lg.shape) < 0.3] = np.nan
+    lg[0, :] = np.nan             # every logit NaN: weights NaN, indices 0, 1, 2
+    lg[1, :] = np.nan
+    lg[1, 7] = 1.0                # fewer finite logits than k
+    inp.logits = gen.f32_to_bf16_bits(lg)
+    g = run_gpu(inp)
+    assert ((g.topk_idx >= 0) & (g.topk_idx < cfg.E)).all()
+    assert g.topk_idx[0].tolist() == [0, 1, 2]
+    check_routing(inp, g)
+    import oracle
+    from gpu_helpers import TOL_BF16, max_rel
+    ref = oracle.forward(inp)["y"]
+    assert np.isnan(g.y[0]).all() and np.isnan(ref[0]).all()
+    err = max_rel(g.y[1:], ref[1:])
+    assert err <= TOL_BF16, f"y max rel err {err:.3e}"
 
 
 def test_zero_tokens_is_a_noop(cuda_device):
@@ -188,9 +246,15 @@ def test_rebind_replaces_the_pack(cuda_device):
 
 # ------------------------------------------------------------ full-size configs
 
-def _sample(T, n=8, seed=0):
-    rng = np.random.default_rng(seed)
-    return np.sort(rng.choice(T, size=min(n, T), replace=False))
+def _full_size(inp, path, name, per_tile, extra, seed):
+    """One full-size forward, then y and h on tokens at every expert segment's
+    ends and token-tile boundaries (plus a few random ones) against the
+    oracle, token by token."""
+    cfg = inp.cfg
+    g = run_gpu(inp, path=path)
+    tokens = np.arange(cfg.T) if cfg.T <= 8 else boundary_tokens(g, cfg.k, per_tile, extra, seed)
+    g = run_gpu(inp, path=path, hidden_tokens=tokens)
+    check_sampled(inp, g, tokens, name=f"{name}/path{g.path}", hidden=True)
 
 
 @pytest.mark.parametrize("path", [None, PATH_DECODE, PATH_TC, PATH_TC_DECODE], ids=["auto", "decode", "tc", "tcdecode"])
@@ -198,15 +262,18 @@ def _sample(T, n=8, seed=0):
 def test_full_size_configs(cuda_device, name, path):
     cfg, seed, kw = gen.workload(name)
     inp = gen.make_inputs(cfg, seed, **kw)
-    g = run_gpu(inp, path=path)
-    tokens = np.arange(cfg.T) if cfg.T <= 8 else _sample(cfg.T)
-    check_sampled(inp, g, tokens)
+    _full_size(inp, path, name, per_tile=1, extra=4, seed=seed)
 
 
+# The prefill sweep at full size (H=4096, I=14336, E=8, k=2): every T of both
+# code families on the kernels the planner picks, plus the opt-in streaming
+# tensor-core path where it applies.
 @pytest.mark.parametrize("path", [None, PATH_TC_DECODE], ids=["auto", "tcdecode"])
-@pytest.mark.parametrize("bits,T", [(4, 1), (4, 16), (8, 1), (8, 128), (4, 1024)])
+@pytest.mark.parametrize("bits,T", [(4, 1), (4, 16), (4, 128), (4, 1024), (4, 8192),
+                                    (8, 1), (8, 16), (8, 128), (8, 1024), (8, 8192)])
 def test_sweep_configs(cuda_device, bits, T, path):
+    if path == PATH_TC_DECODE and T > 128:
+        pytest.skip("the streaming tensor-core path takes at most 32 rows per expert")
     cfg, seed, kw = gen.sweep(bits, T)
     inp = gen.make_inputs(cfg, seed, **kw)
-    g = run_gpu(inp, path=path)
-    check_sampled(inp, g, _sample(T, 4, seed))
+    _full_size(inp, path, f"sweep_int{bits}_T{T}", per_tile=1, extra=2, seed=seed)

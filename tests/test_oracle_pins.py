@@ -163,6 +163,49 @@ def test_routing_brute_force_with_ties(E, k):
         assert math.isclose(sum(row[e] for e in idx[t]), best, rel_tol=0, abs_tol=0)
 
 
+def test_nan_logits_read_as_negative_infinity():
+    """A NaN logit loses to every number and ties resolve by id, so every
+    selected index names an expert; its softmax term is exp(-inf) = 0."""
+    rng = np.random.default_rng(11)
+    E, k = 6, 3
+    lg = rng.standard_normal((300, E))
+    nan_mask = rng.random((300, E)) < 0.4
+    lg[nan_mask] = np.nan
+    lg[0, :] = np.nan                       # no finite logit at all
+    lg[1, :] = np.nan
+    lg[1, 4] = 0.5                          # one finite logit
+    lg = lg.astype(np.float32)
+    for normalize in (True, False):
+        idx, w = oracle.route(lg, k, normalize)
+        assert ((idx >= 0) & (idx < E)).all()
+        for t in range(lg.shape[0]):
+            row = lg[t].astype(np.float64)
+            assert idx[t].tolist() == literal.select_experts(row.tolist(), k)
+            finite = np.flatnonzero(~np.isnan(row))
+            # finite logits first (value desc, id asc), then NaN ids ascending
+            want = sorted(finite.tolist(), key=lambda e: (-row[e], e))[:k]
+            want += [e for e in range(E) if np.isnan(row[e])][:k - len(want)]
+            assert idx[t].tolist() == want
+            if len(finite) == 0:
+                assert np.isnan(w[t]).all()
+                continue
+            p = np.zeros(E)
+            p[finite] = softmax(row[finite])
+            ref = p[idx[t]]
+            if normalize:
+                ref = ref / ref.sum()
+            np.testing.assert_allclose(w[t], ref, rtol=1e-14, atol=0)
+    # grouped selection ignores NaN members when scoring a group
+    lg = np.array([[np.nan, -5.0, 1.0, 0.5, np.nan, np.nan, 0.0, -1.0]])
+    # group scores: {0,1} -5, {2,3} 1, {4,5} -inf (all NaN), {6,7} 0
+    idx, _ = oracle.route(lg, 3, True, 4, 2)
+    assert idx[0].tolist() == [2, 3, 6]
+    idx, _ = oracle.route(lg, 5, True, 4, 3)
+    assert idx[0].tolist() == [2, 3, 6, 7, 1]
+    idx, _ = oracle.route(lg, 8, True, 4, 4)
+    assert idx[0].tolist() == [2, 3, 6, 7, 1, 0, 4, 5]
+
+
 def test_k_equals_E_is_the_softmax():
     rng = np.random.default_rng(3)
     E = 7

@@ -43,10 +43,13 @@ def _forward_both(cfg, seed, path=None):
 def test_noalloc_matches_workspace_forward_twice(cuda_device, path):
     cfg = gen.MoEConfig(T=12, H=256, I=192, E=8, k=2, bits=4, block_size=64, fusion=2,
                         has_fc1_bias=True, has_fc2_bias=True, has_shared=True)
-    ref, outs, _ = _forward_both(cfg, 41, path)
+    ref, outs, m = _forward_both(cfg, 41, path)
     for y in outs:
         assert np.isfinite(y).all()
         assert max_rel(y, ref) <= TOL_BF16
+    # the device status word of the no-alloc forward lives in the fixed array
+    from weight_only_quantized_warp_b200 import qmoe
+    assert qmoe.qmoe_noalloc_read_device_status(m.handle) == qmoe.QMOE_OK
 
 
 def test_noalloc_rejects_calls_above_the_fixed_scratch(cuda_device):

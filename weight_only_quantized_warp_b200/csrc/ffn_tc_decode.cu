@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 // the run's activations: rows [seg0 + tt*bn, +BN), 64-k chunks from
                 // ks_lo*2; the box spans the largest split (out-of-range rows and
                 // chunks arrive as zeros)
-                if (!warp_wait(smem_u32(bempty), bph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                if (!warp_wait(smem_u32(bempty), bph ^ 1u, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
                 bph ^= 1u;
                 const int box_ch = ((nks + a.splits - 1) / a.splits) * (kDBK / 64);
                 mbar_expect_tx_e(smem_u32(bfull), uint32_t(box_ch * BN * 128), e);
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
             prev = it;
             const int64_t blk = int64_t(it.e) * nrb + it.rb;
             for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
-                if (!warp_wait(smem_u32(&pempty[ps]), pph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                if (!warp_wait(smem_u32(&pempty[ps]), pph ^ 1u, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
                 const uint32_t fb = smem_u32(&pfull[ps]);
                 mbar_expect_tx_e(fb, uint32_t(C::kPacked), e);
                 const int g = ks * (kDBK / kgroup_of(BITS));
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 if (++ps == PS) { ps = 0; pph ^= 1u; }
                 if (SMODE != 0) {
                     // the stage's scale blocks [sb0, sb0 + SP): contiguous, 128 scales each
-                    if (!warp_wait(smem_u32(&sempty[ss]), sph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                    if (!warp_wait(smem_u32(&sempty[ss]), sph ^ 1u, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
                     const uint32_t sb = smem_u32(&sfull[ss]);
                     mbar_expect_tx_e(sb, uint32_t(SSLOT), e);
                     const int sb0 = (ks * kDBK) >> bs_log2;
@@ -258,20 +258,20 @@ __global__ void __launch_bounds__(kDThreads, 1)
         for (int i = i_lo; ok && i < i_hi; ++i) {
             const Item it = item_at_stream(i, prefix, a, nrb, nks);
             if (prev.e < 0 || !same_run(prev, it)) {
-                if (!warp_wait(smem_u32(bfull), bph, abort_flag, a.status)) break;
+                if (!warp_wait(smem_u32(bfull), bph, abort_flag, a.status, a.timeout_ns)) break;
                 bph ^= 1u;
             }
             prev = it;
             const uint32_t idesc = idesc_bf16(((it.rows + 15) / 16) * 16);
             if (SMODE == 0) {
                 // one accumulator slot for the whole item
-                if (!warp_wait(smem_u32(&cempty[pr]), cph ^ 1u, abort_flag, a.status)) break;
+                if (!warp_wait(smem_u32(&cempty[pr]), cph ^ 1u, abort_flag, a.status, a.timeout_ns)) break;
                 tc_fence_after();
             }
             for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
                 // with per-stage partials, a full A slot also means a free partial
                 // slot: the dequantise warps waited for it before signalling
-                if (!warp_wait(smem_u32(&afull[as]), aph, abort_flag, a.status)) { ok = false; break; }
+                if (!warp_wait(smem_u32(&afull[as]), aph, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t at = tmem + uint32_t(C::kACol0 + as * kDAStageCols);
                 const uint32_t d0 = tmem + uint32_t(pr * C::kPC);
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
             const Item it = item_at_stream(i, prefix, a, nrb, nks);
             for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
                 if (((sn++) & 1) != par) continue;
-                if (!warp_wait(smem_u32(&pfull[ps]), pph, abort_flag, a.status)) { ok = false; break; }
+                if (!warp_wait(smem_u32(&pfull[ps]), pph, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
                 uint4 wq[GROUPS];
                 const uint8_t* pk = psm + ps * C::kPacked;
 #pragma unroll
@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 if (lane == 0) mbar_arrive(smem_u32(&pempty[ps]));
                 ps += 2;
                 if (ps >= PS) { ps -= PS; pph ^= 1u; }
-                if (!warp_wait(smem_u32(&aempty[as]), aph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                if (!warp_wait(smem_u32(&aempty[as]), aph ^ 1u, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t at = tmem + lane_addr + uint32_t(C::kACol0 + as * kDAStageCols);
 #pragma unroll
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                     // (stage s uses slot s % PR, phase (s / PR) & 1), so the MMA
                     // needs only this one barrier
                     const int s = sn - 1;
-                    if (!warp_wait(smem_u32(&cempty[s % PR]), ((s / PR) & 1) ^ 1u, abort_flag, a.status)) {
+                    if (!warp_wait(smem_u32(&cempty[s % PR]), ((s / PR) & 1) ^ 1u, abort_flag, a.status, a.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
             for (int n = 0; n < BN; ++n) acc[n] = 0.0f;
             if (SMODE == 0) {
-                if (!warp_wait(smem_u32(&cfull[pr]), cph, abort_flag, a.status)) break;
+                if (!warp_wait(smem_u32(&cfull[pr]), cph, abort_flag, a.status, a.timeout_ns)) break;
                 tc_fence_after();
                 const int64_t si = (int64_t(it.e) * nrb + it.rb) * kBlockRows + spos;
                 const float s = !valid ? 0.0f
@@ -431,8 +431,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 if (++pr == PR) { pr = 0; cph ^= 1u; }
             } else {
                 for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
-                    if (!warp_wait(smem_u32(&sfull[ss]), sph, abort_flag, a.status) ||
-                        !warp_wait(smem_u32(&cfull[pr]), cph, abort_flag, a.status)) {
+                    if (!warp_wait(smem_u32(&sfull[ss]), sph, abort_flag, a.status, a.timeout_ns) ||
+                        !warp_wait(smem_u32(&cfull[pr]), cph, abort_flag, a.status, a.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -605,6 +605,8 @@ cudaError_t launch_ffn_tc_decode(const FfnArgs& f, int bn, int32_t* status, cuda
     a.limit = f.limit;
     a.splits = f.splits;
     a.scale_bf16 = f.scale_bf16;
+    a.timeout_ns = f.timeout_ns;
+    a.withhold = f.withhold;
     a.bn = bn;
     // packed ring: 8 slots (int4) / 4 (int8), 64 KB either way; the scale ring
     // takes what is left, up to 24 stages (one slot per stage)

@@ -57,6 +57,17 @@ qmoe_status qmoe_forward_noalloc(const qmoe_handle* h, int64_t T, const void* x,
     {
         std::lock_guard<std::mutex> lock(g_setup_mu);
         if (!g_scratch_addr[dev]) {
+            // the address lookup is not a stream operation; under stream
+            // capture it may fail or invalidate the capture, so the first call
+            // on a device must come before any capture
+            cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+            err = cudaStreamIsCapturing((cudaStream_t)stream, &cs);
+            if (err != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+                h->last_error =
+                    "qmoe_forward_noalloc: the first call on a device looks up the scratch array's address and "
+                    "must not run under stream capture; make one call on this device before capturing";
+                return QMOE_INVALID_ARGUMENT;
+            }
             void* p = nullptr;
             err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
             if (err != cudaSuccess || !p) {
@@ -68,6 +79,26 @@ qmoe_status qmoe_forward_noalloc(const qmoe_handle* h, int64_t T, const void* x,
         scratch = g_scratch_addr[dev];
     }
     return qmoe_forward(h, T, x, router_logits, shared_output, y, scratch, kNoAllocScratchBytes, stream);
+}
+
+qmoe_status qmoe_noalloc_read_device_status(const qmoe_handle* h, void* stream) {
+    if (!h) return QMOE_INVALID_ARGUMENT;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        h->last_error = "qmoe_noalloc_read_device_status: no usable current device";
+        return QMOE_CUDA_ERROR;
+    }
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_setup_mu);
+        scratch = g_scratch_addr[dev];
+    }
+    if (!scratch) {
+        h->last_error = "qmoe_noalloc_read_device_status: no qmoe_forward_noalloc call has run on this device";
+        return QMOE_INVALID_ARGUMENT;
+    }
+    // the status word sits at the same offset for every T
+    return qmoe_read_device_status(h, scratch, stream);
 }
 
 }  // extern "C"

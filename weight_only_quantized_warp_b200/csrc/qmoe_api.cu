@@ -396,6 +396,17 @@ qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t value) {
         h->path_override = int(value);
         return QMOE_OK;
     }
+    if (option == QMOE_OPT_WAIT_LIMIT_NS) {
+        if (value < 100000 || value > int64_t(60) * 1000000000)
+            return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_WAIT_LIMIT_NS must lie in [1e5, 6e10] ns");
+        h->wait_limit_ns = uint64_t(value);
+        return QMOE_OK;
+    }
+    if (option == QMOE_OPT_TEST_WITHHOLD) {
+        if (value != 0 && value != 1) return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_TEST_WITHHOLD must be 0 or 1");
+        h->withhold = int(value);
+        return QMOE_OK;
+    }
     return fail(h, QMOE_INVALID_ARGUMENT, "unknown option %d", int(option));
 }
 
@@ -515,6 +526,8 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     f1.fp4 = c.weight_format == QMOE_WEIGHTS_MXFP4;
     f1.act_bf16 = bf16;
     f1.nt = p.nt;
+    f1.timeout_ns = h->wait_limit_ns;
+    f1.withhold = h->withhold;
     FfnArgs f2 = f1;
     f2.W = h->w2;
     f2.S = h->s2;

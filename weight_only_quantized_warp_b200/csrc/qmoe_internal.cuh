@@ -83,6 +83,8 @@ struct qmoe_handle {
     float* b2 = nullptr;  // [E, H] fp32, nullptr when no fc2 bias
     int device = -1;
     int path_override = -1;  // QMOE_OPT_PATH; -1 = choose by shape
+    uint64_t wait_limit_ns = 2000000000ull;  // QMOE_OPT_WAIT_LIMIT_NS
+    int withhold = 0;        // QMOE_OPT_TEST_WITHHOLD
     mutable std::mutex mu;
     mutable std::string last_error;
 };
@@ -153,6 +155,10 @@ struct FfnArgs {
     // per-block scales [rows, K / block_size]; rows indexed like `act`
     const int8_t* aq;
     const float* as;
+    // tcgen05 kernels: limit of every bounded device wait, and the test-only
+    // withheld accumulator signal (QMOE_OPT_WAIT_LIMIT_NS, QMOE_OPT_TEST_WITHHOLD)
+    uint64_t timeout_ns;
+    int withhold;
 };
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
 // Shared memory of one decode CTA (staged activation rows) and its limit;

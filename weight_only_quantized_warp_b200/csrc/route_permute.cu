@@ -7,7 +7,7 @@
 // Readings: selection is by raw logit (exact in any precision, so the
 // selection is bit-identical to any other exact implementation), ties go to
 // the lower expert id, and the list is ordered by (logit descending, id
-// ascending). The weights are the softmax over all E logits restricted to the
+// ascending); a NaN logit reads as -inf. The weights are the softmax over all E logits restricted to the
 // selection, renormalised over the k when asked.
 //
 // The permutation groups the T*k (token, slot) pairs into per-expert
@@ -41,6 +41,10 @@ __device__ __forceinline__ void route_token(const void* logits, int act_bf16, in
         if (i < per && e < E) {
             v[i] = act_bf16 ? __bfloat162float(((const __nv_bfloat16*)logits)[t * E + e])
                             : ((const float*)logits)[t * E + e];
+            // a NaN logit never wins a comparison; read as -inf it still
+            // loses to every number and ties resolve by id, so every
+            // selected index is a real expert
+            if (isnan(v[i])) v[i] = -INFINITY;
         }
     }
     // max over all E

@@ -12,6 +12,7 @@
 namespace qmoe {
 namespace {
 
+// Default limit of every bounded device wait (QMOE_OPT_WAIT_LIMIT_NS).
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 struct TcArgs {
@@ -26,6 +27,8 @@ struct TcArgs {
     float alpha, beta, limit;
     int splits, scale_bf16, bn;
     int ring, stage_bytes, sring;  // streaming decode: packed-ring slots, scale-slot bytes, scale-ring slots
+    uint64_t timeout_ns;     // limit of every bounded wait
+    int withhold;            // test only: the MMA warp keeps back its first item's accumulator signal
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -80,17 +83,17 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait on a phase parity. Returns false (after raising the CTA's
-// abort flag and the workspace status) when the wait gives up or another role
-// already aborted.
+// abort flag and the workspace status) when the wait gives up after
+// limit_ns, or another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
+                                          int32_t* status, uint64_t limit_ns) {
     if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = now_ns();
     for (uint32_t spin = 1;; ++spin) {
         if (mbar_try(bar, parity)) return true;
         if ((spin & 15u) == 0u) {
             if (*abort_flag) return false;
-            if (now_ns() - t0 > kTimeoutNs) {
+            if (now_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 atomicExch(status, int32_t(QMOE_TIMEOUT));
                 return false;
@@ -102,8 +105,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Wait by a whole warp: every lane polls, and the warp continues only if all
 // lanes saw the phase complete (a timeout in any lane stops the whole warp).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
-    const bool ok = mbar_wait(bar, parity, abort_flag, status);
+                                          int32_t* status, uint64_t limit_ns) {
+    const bool ok = mbar_wait(bar, parity, abort_flag, status, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
 

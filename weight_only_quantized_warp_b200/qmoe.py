@@ -39,8 +39,9 @@ EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forwa
            "qmoe_status_string", "qmoe_last_error", "qmoe_path_for", "qmoe_launches_for",
            "qmoe_token_tile_for",
            "qmoe_set_option", "qmoe_forward_noalloc", "qmoe_noalloc_scratch_bytes",
+           "qmoe_noalloc_read_device_status",
            "qmoe_quantize_act_i8")
-QMOE_OPT_PATH = 1
+QMOE_OPT_PATH, QMOE_OPT_WAIT_LIMIT_NS, QMOE_OPT_TEST_WITHHOLD = 1, 2, 3
 
 
 class qmoe_config(ctypes.Structure):
@@ -89,6 +90,8 @@ lib.qmoe_forward_noalloc.restype = ctypes.c_int
 lib.qmoe_forward_noalloc.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp]
 lib.qmoe_noalloc_scratch_bytes.restype = _sz
 lib.qmoe_noalloc_scratch_bytes.argtypes = []
+lib.qmoe_noalloc_read_device_status.restype = ctypes.c_int
+lib.qmoe_noalloc_read_device_status.argtypes = [_vp, _vp]
 lib.qmoe_set_option.restype = ctypes.c_int
 lib.qmoe_set_option.argtypes = [_vp, ctypes.c_int32, _i64]
 lib.qmoe_launches_for.restype = ctypes.c_int32
@@ -182,6 +185,11 @@ def qmoe_forward_noalloc(h, T, x, router_logits, shared_output, y, stream=None):
 
 def qmoe_noalloc_scratch_bytes() -> int:
     return int(lib.qmoe_noalloc_scratch_bytes())
+
+
+def qmoe_noalloc_read_device_status(h, stream=None) -> int:
+    """Device status word of the last no-alloc forward on the current device."""
+    return int(lib.qmoe_noalloc_read_device_status(h, _stream(stream)))
 
 
 def qmoe_forward_profiled(h, T, x, router_logits, shared_output, y, workspace, workspace_bytes,
