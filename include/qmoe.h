@@ -63,7 +63,7 @@ typedef enum qmoe_status {
 /* activation_type, in the order the QMoE page lists them. */
 enum {
     QMOE_ACT_RELU = 0,
-    QMOE_ACT_GELU = 1, /* erf form */
+    QMOE_ACT_GELU = 1, /* erf form, or the tanh form with gelu_mode QMOE_GELU_TANH */
     QMOE_ACT_SILU = 2,
     QMOE_ACT_SWIGLU = 3,
     QMOE_ACT_IDENTITY = 4
@@ -153,7 +153,17 @@ typedef struct qmoe_config {
     int32_t apply_router_weight_on_input;
     int32_t weight_format;        /* QMOE_WEIGHTS_* */
     int32_t compute_mode;         /* QMOE_COMPUTE_* */
+    /* Options the "MoE" page names without formulas; readings:
+     *   expert_output_scale -- multiplies every expert's output (its fc2 bias
+     *     included) before the router weighting; 0 reads as 1; finite, >= 0.
+     *   gelu_mode -- QMOE_GELU_ERF (default) or QMOE_GELU_TANH, the form of
+     *     activation_type GELU (plain or gated): erf, or the tanh form
+     *     0.5 a (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3))). */
+    float expert_output_scale;
+    int32_t gelu_mode;
 } qmoe_config;
+
+enum { QMOE_GELU_ERF = 0, QMOE_GELU_TANH = 1 };
 
 typedef struct qmoe_handle qmoe_handle;
 
@@ -190,6 +200,23 @@ QMOE_API qmoe_status qmoe_set_weights(qmoe_handle* h,
                              const void* fc2_w, const void* fc2_s, const void* fc2_b,
                              const void* fc3_w, const void* fc3_s, const void* fc3_b,
                              void* stream);
+
+/*
+ * qmoe_set_score_correction_bias -- the e_score_correction_bias tensor of
+ * "ClikaRT::nn::QMoEWoQ" / the QMoEWoQ Python page, set_weights(); the pages
+ * give no formula. Reading: the bias moves the expert selection only. Every
+ * forward then ranks experts (and, with grouped top-k, groups by their
+ * largest key) by the fp32 sum logit + bias[e], one single-precision
+ * addition, ties to the lower id; the router weights stay the softmax of the
+ * unbiased logits over all E, restricted to the selection.
+ *
+ *   bias  [E] fp32, a DEVICE pointer aligned to 4 bytes, or NULL to clear
+ *
+ * The values are copied into handle-owned device memory (the call waits for
+ * the copy on `stream`); the caller may free its buffer afterwards. A NaN
+ * key reads as -inf. QMOE_INVALID_ARGUMENT for a misaligned pointer.
+ */
+QMOE_API qmoe_status qmoe_set_score_correction_bias(qmoe_handle* h, const void* bias, void* stream);
 
 /*
  * qmoe_workspace_size -- bytes of device scratch that qmoe_forward needs for

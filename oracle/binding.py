@@ -32,7 +32,9 @@ class _Cfg(ctypes.Structure):
                 ("apply_router_weight_on_input", ctypes.c_int32),
                 ("routed_scaling_factor", ctypes.c_double),
                 ("mxfp4", ctypes.c_int32), ("act_bf16", ctypes.c_int32),
-                ("int8_block", ctypes.c_int32)]
+                ("int8_block", ctypes.c_int32), ("pad_", ctypes.c_int32),
+                ("expert_output_scale", ctypes.c_double),
+                ("score_bias", ctypes.c_void_p)]
 
 
 def _load():
@@ -97,14 +99,18 @@ def dequant(packed: np.ndarray, scales: np.ndarray, N: int, K: int, bits: int,
     return w
 
 
-def route(logits: np.ndarray, k: int, normalize: bool, n_group: int = 0, topk_group: int = 0):
+def route(logits: np.ndarray, k: int, normalize: bool, n_group: int = 0, topk_group: int = 0,
+          score_bias: Optional[np.ndarray] = None):
+    """Top-k routing of ``logits`` [T, E]; ``score_bias`` [E] (fp32 values,
+    the e_score_correction_bias) shifts the selection keys only."""
     lg = to_f64(logits)
     T, E = lg.shape
+    sb = None if score_bias is None else to_f64(np.asarray(score_bias, dtype=np.float32))
     idx = np.empty((T, k), dtype=np.int32)
     w = np.empty((T, k), dtype=np.float64)
     _load().oracle_route(_p(lg, _f64p), ctypes.c_int64(T), ctypes.c_int64(E), ctypes.c_int64(k),
                          ctypes.c_int32(int(normalize)), ctypes.c_int32(n_group), ctypes.c_int32(topk_group),
-                         _p(idx, _i32p), _p(w, _f64p))
+                         _p(sb, _f64p), _p(idx, _i32p), _p(w, _f64p))
     return idx, w
 
 
@@ -188,8 +194,12 @@ def forward(inp, tokens: Optional[Sequence[int]] = None, want_h: bool = False) -
         x, lg = np.ascontiguousarray(x[tokens]), np.ascontiguousarray(lg[tokens])
         sh = None if sh is None else np.ascontiguousarray(sh[tokens])
     T = x.shape[0]
+    sb = getattr(inp, "score_bias", None)
+    sb = None if sb is None else to_f64(np.asarray(sb, dtype=np.float32))
+    eos = float(getattr(c, "expert_output_scale", 1.0) or 1.0)
+    act = 5 if (c.act == 1 and int(getattr(c, "gelu_mode", 0)) == 1) else c.act  # GELU, tanh form
     cfg = _Cfg(T=T, H=c.H, I=c.I, E=c.E, k=c.k, bits=c.bits, block_size=c.block_size,
-               act=c.act, fusion=c.fusion, normalize=int(c.normalize), has_fc3=int(c.has_fc3),
+               act=act, fusion=c.fusion, normalize=int(c.normalize), has_fc3=int(c.has_fc3),
                alpha=float(c.alpha), beta=float(c.beta),
                limit=float(c.limit) if c.limit is not None else math.inf,
                n_group=int(c.n_group), topk_group=int(c.topk_group),
@@ -197,7 +207,8 @@ def forward(inp, tokens: Optional[Sequence[int]] = None, want_h: bool = False) -
                routed_scaling_factor=float(c.routed_scaling_factor) if c.routed_scaling_factor else 1.0,
                mxfp4=int(c.weight_format == 1),
                act_bf16=int(np.asarray(inp.x).dtype == np.uint16),
-               int8_block=int(getattr(c, "compute_mode", 0) == 1))
+               int8_block=int(getattr(c, "compute_mode", 0) == 1),
+               expert_output_scale=eos, score_bias=None if sb is None else sb.ctypes.data)
     y = np.empty((T, c.H), dtype=np.float64)
     idx = np.empty((T, c.k), dtype=np.int32)
     w = np.empty((T, c.k), dtype=np.float64)

@@ -12,8 +12,11 @@ gated FFN, weighted combine), the "QLinearWoQ" summary (x @ dequant(W).T + b)
 and "ClikaRT::nn::QMoEWoQ" forward() (shared_output folds into the combine),
 plus its class description's int8 block tier (compute_mode 1: per-block
 int8 rounding of each expert input row, decided with numpy float32 scalars,
-and integer dots per block). Grouped routing, the router weight on the
-input, routed scaling and MXFP4 are left to the C oracle.
+and integer dots per block), the routing bias of set_weights
+(e_score_correction_bias: selection on float32 logit + bias, weights from the
+unbiased logits), expert_output_scale and the tanh form of GELU. Grouped
+routing, the router weight on the input, routed scaling and MXFP4 are left to
+the C oracle.
 """
 from __future__ import annotations
 
@@ -119,20 +122,24 @@ def dot_i8(packed_row, scales_row, K, bits, bs, codes, xs):
     return tot
 
 
-def activation(act, g, u, alpha, beta, limit, gated):
+def _gelu(a, tanh_form):
+    if tanh_form:
+        return 0.5 * a * (1 + math.tanh(math.sqrt(2 / math.pi) * (a + 0.044715 * a ** 3)))
+    return 0.5 * a * (1 + math.erf(a / math.sqrt(2)))
+
+
+def activation(act, g, u, alpha, beta, limit, gated, gelu_tanh=False):
     sig = lambda v: 1.0 / (1.0 + math.exp(-v))  # noqa: E731
     if not gated:
         a = g
-        return {0: max(a, 0.0), 1: 0.5 * a * (1 + math.erf(a / math.sqrt(2))),
-                2: a * sig(a), 4: a}[act]
+        return {0: max(a, 0.0), 1: _gelu(a, gelu_tanh), 2: a * sig(a), 4: a}[act]
     if act == 3:
         al = 1.0 if alpha == 0 else alpha
         if math.isfinite(limit) and limit > 0:
             g = min(g, limit)
             u = max(-limit, min(limit, u))
         return (u + beta) * g * sig(al * g)
-    base = {0: max(g, 0.0), 1: 0.5 * g * (1 + math.erf(g / math.sqrt(2))),
-            2: g * sig(g), 4: g}[act]
+    base = {0: max(g, 0.0), 1: _gelu(g, gelu_tanh), 2: g * sig(g), 4: g}[act]
     return base * u
 
 
@@ -163,11 +170,21 @@ def forward(inp):
     S1, S2 = scl(inp.fc1_s), scl(inp.fc2_s)
     S3 = scl(inp.fc3_s) if c.has_fc3 else None
 
+    gt = int(getattr(c, "gelu_mode", 0)) == 1
+    eos = float(getattr(c, "expert_output_scale", 1.0) or 1.0)
+    sbias = getattr(inp, "score_bias", None)
     y = np.zeros((c.T, c.H))
     sels, wts = [], []
     for t in range(c.T):
         row = lg[t].tolist()
-        sel = select_experts(row, c.k)
+        if sbias is None:
+            sel = select_experts(row, c.k)
+        else:
+            # selection keys: one float32 addition of logit and bias (numpy's
+            # IEEE single precision); the weights use the unbiased logits
+            keys = [float(np.float32(v) + np.float32(b)) for v, b in zip(np.asarray(lg[t], dtype=np.float32),
+                                                                       np.asarray(sbias, dtype=np.float32))]
+            sel = select_experts(keys, c.k)
         w = route_weights(row, sel, c.normalize)
         sels.append(sel)
         wts.append(w)
@@ -183,7 +200,7 @@ def forward(inp):
             h = []
             for i in range(c.I):
                 if not gated:
-                    h.append(activation(c.act, a[i], None, c.alpha, c.beta, c.limit, False))
+                    h.append(activation(c.act, a[i], None, c.alpha, c.beta, c.limit, False, gt))
                     continue
                 if c.fusion == 1:
                     g, u = a[2 * i], a[2 * i + 1]
@@ -195,7 +212,7 @@ def forward(inp):
                         u = dot_i8(inp.fc3_w[e][i], S3[e][i], c.H, c.bits, c.block_size, qx, sx) + b3[i]
                     else:
                         u = sum(xt[kk] * W3[e][i][kk] for kk in range(c.H)) + b3[i]
-                h.append(activation(c.act, g, u, c.alpha, c.beta, c.limit, True))
+                h.append(activation(c.act, g, u, c.alpha, c.beta, c.limit, True, gt))
             if i8:
                 qh, sh_ = quantize_row([round_act(v, bf16) for v in h], c.block_size)
             for m in range(c.H):
@@ -203,7 +220,7 @@ def forward(inp):
                     o = dot_i8(inp.fc2_w[e][m], S2[e][m], c.I, c.bits, c.block_size, qh, sh_) + b2[m]
                 else:
                     o = sum(h[i] * W2[e][m][i] for i in range(c.I)) + b2[m]
-                y[t, m] += w[j] * o
+                y[t, m] += w[j] * (eos * o)
         if sh is not None:
             y[t] += sh[t]
     return dict(y=y, topk_idx=np.array(sels, dtype=np.int32), topk_w=np.array(wts))

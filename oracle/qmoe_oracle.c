@@ -33,7 +33,8 @@
  *     rows, up = last I rows; fusion 0 with fc3: gate = fc1, up = fc3.
  *
  * Routing options the "MoE" page names without formulas (n_group,
- * topk_group, routed_scaling_factor, apply_router_weight_on_input), read as:
+ * topk_group, routed_scaling_factor, apply_router_weight_on_input,
+ * expert_output_scale, gelu_mode), read as:
  *   - grouped top-k: the E experts form n_group consecutive groups of
  *     E / n_group; a group's score is the largest raw logit among its
  *     experts; the topk_group groups with the highest scores are kept (ties
@@ -42,7 +43,11 @@
  *   - routed_scaling_factor multiplies the router-weighted sum of the expert
  *     outputs, not the shared output;
  *   - apply_router_weight_on_input: the router weight multiplies the
- *     expert's input row instead of its output.
+ *     expert's input row instead of its output;
+ *   - expert_output_scale multiplies every expert's output (its fc2 bias
+ *     included) before the router weighting;
+ *   - gelu_mode "tanh" selects the tanh form of GELU (see plain_act).
+ * e_score_correction_bias: see oracle_route.
  *
  * MXFP4 weights (the block format the QMoEWoQ page names for its gpt-oss
  * checkpoint), read as OCP microscaling FP4: a 4-bit code is e2m1 -- sign
@@ -65,6 +70,7 @@
  * Every sum is a serial fp64 loop in index order, so the result does not
  * depend on the thread count.
  */
+#define _GNU_SOURCE
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -74,7 +80,8 @@
 #include <omp.h>
 #endif
 
-enum { O_RELU = 0, O_GELU = 1, O_SILU = 2, O_SWIGLU = 3, O_IDENTITY = 4 };
+/* O_GELU_TANH: GELU in its tanh form (gelu_mode "tanh"). */
+enum { O_RELU = 0, O_GELU = 1, O_SILU = 2, O_SWIGLU = 3, O_IDENTITY = 4, O_GELU_TANH = 5 };
 
 typedef struct oracle_cfg {
     int64_t T, H, I, E, k;
@@ -91,6 +98,9 @@ typedef struct oracle_cfg {
     int32_t mxfp4;                       /* codes are e2m1, no zero point */
     int32_t act_bf16;                    /* activation dtype: 1 bf16, 0 fp32 */
     int32_t int8_block;                  /* int8 block compute tier */
+    int32_t pad_;
+    double expert_output_scale;          /* multiplies every expert output (with its bias) */
+    const double* score_bias;            /* e_score_correction_bias [E], or NULL */
 } oracle_cfg;
 
 int oracle_num_threads(void) {
@@ -140,17 +150,33 @@ void oracle_dequant(const uint8_t* packed, const double* scales, int64_t N, int6
 /* Routing ("MoE" page summary; QMoE page attributes k and
  * normalize_routing_weights). A NaN logit reads as -inf: it loses to every
  * number, and among equal values the lower id wins, so every selected index
- * names an expert. */
+ * names an expert.
+ *
+ * e_score_correction_bias (QMoEWoQ pages, a set_weights tensor without a
+ * formula), read as: the bias moves the selection only. Experts (and groups)
+ * are ranked by the key fp32(logit + bias[e]) -- one IEEE single-precision
+ * addition of the stored logit and the fp32 bias, a NaN key reading as -inf
+ * -- while the weights stay the softmax of the unbiased logits over all E,
+ * restricted to the selection. */
 void oracle_route(const double* logits, int64_t T, int64_t E, int64_t k, int32_t normalize,
-                  int32_t n_group, int32_t topk_group, int32_t* idx, double* w) {
+                  int32_t n_group, int32_t topk_group, const double* score_bias, int32_t* idx, double* w) {
     char* taken = (char*)malloc((size_t)E);
     char* allowed = (char*)malloc((size_t)E);
     double* p = (double*)malloc(sizeof(double) * (size_t)E);
-    double* l = (double*)malloc(sizeof(double) * (size_t)E);
+    double* lv = (double*)malloc(sizeof(double) * (size_t)E);  /* logits, NaN as -inf */
+    double* l = (double*)malloc(sizeof(double) * (size_t)E);   /* selection keys */
     const int64_t G = n_group > 1 ? n_group : 1, gsize = E / G;
     char* kept = (char*)malloc((size_t)G);
     for (int64_t t = 0; t < T; ++t) {
-        for (int64_t e = 0; e < E; ++e) l[e] = isnan(logits[t * E + e]) ? -INFINITY : logits[t * E + e];
+        for (int64_t e = 0; e < E; ++e) {
+            lv[e] = isnan(logits[t * E + e]) ? -INFINITY : logits[t * E + e];
+            if (score_bias) {
+                const float key = (float)lv[e] + (float)score_bias[e];
+                l[e] = isnan(key) ? -INFINITY : (double)key;
+            } else {
+                l[e] = lv[e];
+            }
+        }
         /* groups: keep the topk_group groups of largest member logit */
         memset(kept, G == 1, (size_t)G);
         for (int64_t r = 0; G > 1 && r < topk_group; ++r) {
@@ -177,12 +203,12 @@ void oracle_route(const double* logits, int64_t T, int64_t E, int64_t k, int32_t
             taken[best] = 1;
             idx[t * k + j] = (int32_t)best;
         }
-        double mx = l[0];
+        double mx = lv[0];
         for (int64_t e = 1; e < E; ++e)
-            if (l[e] > mx) mx = l[e];
+            if (lv[e] > mx) mx = lv[e];
         double z = 0.0;
-        for (int64_t e = 0; e < E; ++e) z += exp(l[e] - mx);
-        for (int64_t e = 0; e < E; ++e) p[e] = exp(l[e] - mx) / z;
+        for (int64_t e = 0; e < E; ++e) z += exp(lv[e] - mx);
+        for (int64_t e = 0; e < E; ++e) p[e] = exp(lv[e] - mx) / z;
         double sel = 0.0;
         for (int64_t j = 0; j < k; ++j) sel += p[idx[t * k + j]];
         for (int64_t j = 0; j < k; ++j)
@@ -193,6 +219,7 @@ void oracle_route(const double* logits, int64_t T, int64_t E, int64_t k, int32_t
     free(kept);
     free(p);
     free(l);
+    free(lv);
 }
 
 /* Token -> expert permutation: segments in expert order, tokens ascending
@@ -215,10 +242,15 @@ void oracle_permute(const int32_t* idx, int64_t T, int64_t E, int64_t k, int32_t
 
 static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
 
+/* activation_type of the QMoE page; GELU in its erf form, or (gelu_mode
+ * "tanh", named by the MoE page's options without a formula) in the tanh
+ * form of the GELU paper (Hendrycks and Gimpel):
+ * 0.5 a (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3))). */
 static double plain_act(int act, double a) {
     switch (act) {
         case O_RELU: return a > 0.0 ? a : 0.0;
         case O_GELU: return 0.5 * a * (1.0 + erf(a / sqrt(2.0)));
+        case O_GELU_TANH: return 0.5 * a * (1.0 + tanh(sqrt(2.0 / M_PI) * (a + 0.044715 * a * a * a)));
         case O_SILU: return a * sigmoid(a);
         default: return a; /* identity */
     }
@@ -324,8 +356,9 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
     const int64_t pk1 = H * bits / 8, pk2 = I * bits / 8;
     const int64_t sc1 = bs > 0 ? H / bs : 1, sc2 = bs > 0 ? I / bs : 1;
 
-    oracle_route(logits, T, E, k, c->normalize, c->n_group, c->topk_group, topk_idx, topk_w);
+    oracle_route(logits, T, E, k, c->normalize, c->n_group, c->topk_group, c->score_bias, topk_idx, topk_w);
     const double rsf = c->routed_scaling_factor;
+    const double eos = c->expert_output_scale;
 
     double* a1 = (double*)calloc((size_t)(R * N1), sizeof(double)); /* fc1 pre-activation */
     double* a3 = c->has_fc3 ? (double*)calloc((size_t)(R * I), sizeof(double)) : NULL;
@@ -428,7 +461,7 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
         free(q1);
         free(qs1);
 
-        /* FC2: o[r, m] = sum_i h[r, i] * W2[m, i] + b2[m] */
+        /* FC2: o[r, m] = eos * (sum_i h[r, i] * W2[m, i] + b2[m]) */
         const uint8_t* w2 = fc2_w + e * H * pk2;
         const double* s2 = fc2_s + e * H * sc2;
         /* int8 tier: h rounded to the activation dtype, then per block to int8 */
@@ -459,7 +492,7 @@ int oracle_forward(const oracle_cfg* c, const double* x, const double* logits,
                     else
                         for (int64_t kk = 0; kk < I; ++kk) acc += h[r * I + kk] * wrow[kk];
                     if (fc2_b) acc += fc2_b[e * H + n];
-                    o[r * H + n] = acc;
+                    o[r * H + n] = eos * acc;
                 }
             }
             free(wrow);

@@ -39,7 +39,9 @@ def test_library_exports_every_declared_symbol(q):
 
 
 def test_config_struct_layout(q):
-    assert ctypes.sizeof(q.qmoe_config) == 120
+    assert ctypes.sizeof(q.qmoe_config) == 128
+    assert q.qmoe_config.expert_output_scale.offset == 120
+    assert q.qmoe_config.gelu_mode.offset == 124
     assert q.qmoe_config.expert_weight_bits.offset == 32
     assert q.qmoe_config.activation_alpha.offset == 48
     assert q.qmoe_config.reserved.offset == 92
@@ -83,6 +85,8 @@ BAD = [
     (dict(weight_format=1, block_size=64, scale_dtype=2), 1),   # ... and block_size 32
     (dict(weight_format=1, expert_weight_bits=8, block_size=32, scale_dtype=2), 1),
     (dict(scale_dtype=2), 1),                                   # E8M0 only with MXFP4
+    (dict(expert_output_scale=-0.5), 1), (dict(expert_output_scale=math.inf), 1),
+    (dict(gelu_mode=2), 1), (dict(gelu_mode=-1), 1),
 ]
 
 
@@ -178,6 +182,16 @@ def test_noalloc_status_before_any_noalloc_call(q):
     try:
         assert q.lib.qmoe_noalloc_read_device_status(h, None) in (q.QMOE_INVALID_ARGUMENT, q.QMOE_CUDA_ERROR)
         assert q.lib.qmoe_noalloc_read_device_status(None, None) == q.QMOE_INVALID_ARGUMENT
+    finally:
+        q.qmoe_destroy(h)
+
+
+def test_score_bias_setter_rejects_before_device_work(q):
+    h = q.qmoe_create(_cfg(q))
+    try:
+        assert q.lib.qmoe_set_score_correction_bias(h, 258, None) == q.QMOE_INVALID_ARGUMENT  # misaligned
+        assert q.lib.qmoe_set_score_correction_bias(h, None, None) == q.QMOE_OK              # clear: no-op
+        assert q.lib.qmoe_set_score_correction_bias(None, None, None) == q.QMOE_INVALID_ARGUMENT
     finally:
         q.qmoe_destroy(h)
 

@@ -131,6 +131,8 @@ CASES = {
     "two_tiles_per_expert": dict(T=40),
     "four_tiles_two_passes": dict(T=150),
     "unfused_routing": dict(T=300, E=4),
+    "score_bias_gelu_tanh_eos": dict(fusion=1, act=gen.ACT_GELU, gelu_mode=1, has_score_bias=True,
+                                     expert_output_scale=0.5, E=16, k=3),
 }
 
 

@@ -94,6 +94,16 @@ CASES = {
                                       normalize=False, routed_scaling_factor=0.5),
     "fp32_weight_on_input_scaled": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, apply_router_weight_on_input=True,
                                         routed_scaling_factor=0.75, normalize=False, block_size=32),
+    # e_score_correction_bias (selection keys fp32(logit + bias)), expert_output_scale, tanh GELU
+    "score_bias": dict(T=40, E=16, k=4, has_score_bias=True, normalize=False),
+    "score_bias_grouped_eos": dict(T=40, E=16, k=4, n_group=4, topk_group=2, has_score_bias=True,
+                                   expert_output_scale=1.75, has_fc2_bias=True),
+    "score_bias_wide_tile": dict(T=300, E=2, k=1, H=256, I=384, has_score_bias=True),
+    "gelu_tanh_plain_bias": dict(fusion=0, act=gen.ACT_GELU, gelu_mode=1, has_fc1_bias=True),
+    "gelu_tanh_gated_int8": dict(fusion=1, act=gen.ACT_GELU, gelu_mode=1, bits=8, block_size=64),
+    "gelu_tanh_wide_tile": dict(T=300, E=2, k=1, H=256, I=384, fusion=0, act=gen.ACT_GELU, gelu_mode=1),
+    "gelu_tanh_fp32_eos": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, fusion=0, act=gen.ACT_GELU,
+                               gelu_mode=1, expert_output_scale=0.25, has_shared=True),
     # MXFP4 expert weights (e2m1 codes, E8M0 scale per 32)
     "mxfp4_swiglu_bias": dict(weight_format=gen.WEIGHTS_MXFP4, block_size=32, scale_dtype=gen.DT_E8M0, fusion=1,
                               alpha=1.702, beta=1.0, limit=7.0, has_fc1_bias=True, has_fc2_bias=True),

@@ -229,6 +229,94 @@ def test_unnormalised_weights_are_softmax_probabilities():
     np.testing.assert_allclose(w2.sum(axis=1), 1.0, rtol=1e-15)
 
 
+# ------------------------------------------- e_score_correction_bias (QMoEWoQ pages)
+
+def test_golden_score_bias_examples():
+    for case in _golden("routing_bias.json")["cases"]:
+        lg = np.array([case["logits"]], dtype=np.float32)
+        idx, w = oracle.route(lg, case["k"], case["normalize"], score_bias=np.array(case["bias"], dtype=np.float32))
+        assert idx[0].tolist() == case["sel"], case
+        np.testing.assert_allclose(w[0], [_eval(s) for s in case["weights"]], rtol=1e-14)
+
+
+@pytest.mark.parametrize("E,G,TG,k", [(8, 0, 0, 2), (16, 0, 0, 5), (16, 4, 2, 4), (32, 8, 3, 6)])
+def test_score_bias_against_float32_keys(E, G, TG, k):
+    """Selection = top-k of numpy float32(logit) + float32(bias) (IEEE single
+    additions), groups scored by their largest key; weights = the unbiased
+    softmax restricted to the selection."""
+    rng = np.random.default_rng(E * 3 + k)
+    lg = rng.standard_normal((150, E)).astype(np.float32)
+    b = (rng.standard_normal(E) * 0.7).astype(np.float32)
+    keys = lg + b                      # float32 + float32 -> float32
+    for normalize in (True, False):
+        idx, w = oracle.route(lg, k, normalize, G, TG, score_bias=b)
+        p = softmax(lg.astype(np.float64), axis=1)
+        for t in range(lg.shape[0]):
+            allowed = np.ones(E, dtype=bool)
+            if G > 1:
+                gs = keys[t].reshape(G, E // G).max(axis=1)
+                order = sorted(range(G), key=lambda g: (-gs[g], g))[:TG]
+                allowed = np.isin(np.arange(E) // (E // G), order)
+            cand = [e for e in range(E) if allowed[e]]
+            want = sorted(cand, key=lambda e: (-keys[t, e], e))[:k]
+            assert idx[t].tolist() == want
+            ref = p[t, want]
+            if normalize:
+                ref = ref / ref.sum()
+            np.testing.assert_allclose(w[t], ref, rtol=1e-14)
+    # a zero bias changes nothing
+    i0, w0 = oracle.route(lg, k, True, G, TG)
+    i1, w1 = oracle.route(lg, k, True, G, TG, score_bias=np.zeros(E, dtype=np.float32))
+    np.testing.assert_array_equal(i0, i1)
+    np.testing.assert_array_equal(w0, w1)
+
+
+# ------------------------------------------------- gelu_mode, expert_output_scale
+
+def test_gelu_tanh_form_against_torch():
+    """The tanh form of GELU equals torch's gelu(approximate="tanh") in fp64,
+    stays within 1e-3 of the erf form, and keeps gelu(a) - gelu(-a) = a."""
+    import torch
+    a = np.linspace(-8.0, 8.0, 641)
+    ref = torch.nn.functional.gelu(torch.from_numpy(a), approximate="tanh").numpy()
+    got = np.array([oracle.plain_act(5, v) for v in a])
+    np.testing.assert_allclose(got, ref, rtol=1e-14, atol=1e-15)
+    erf = np.array([oracle.plain_act(gen.ACT_GELU, v) for v in a])
+    assert np.abs(got - erf).max() < 1e-3
+    neg = np.array([oracle.plain_act(5, -v) for v in a])
+    np.testing.assert_allclose(got - neg, a, rtol=0, atol=1e-14)
+    # gated use: act(g) * u with the same form
+    assert oracle.gated_act(5, 1.25, -0.5, 0.0, 0.0, math.inf) == oracle.plain_act(5, 1.25) * -0.5
+
+
+def test_gelu_mode_selects_the_form_in_the_forward():
+    cfg = _tiny_cfg(T=5, fusion=0, act=gen.ACT_GELU, has_fc1_bias=True)
+    inp = gen.make_inputs(cfg, seed=23, bias_std=0.1)
+    y_erf = oracle.forward(inp, want_h=True)
+    inp_t = dataclasses.replace(inp, cfg=dataclasses.replace(cfg, gelu_mode=1))
+    y_tanh = oracle.forward(inp_t, want_h=True)
+    assert not np.array_equal(y_erf["h"], y_tanh["h"])
+    np.testing.assert_allclose(y_tanh["h"], y_erf["h"], rtol=0, atol=1e-3 * np.abs(y_erf["h"]).max() + 1e-3)
+
+
+def test_expert_output_scale_scales_every_expert_output():
+    """eos multiplies each expert output (with its fc2 bias) before the
+    router weighting: y - shared scales by eos, the same as
+    routed_scaling_factor, and a forced single expert gives eos times the
+    two-layer QLinear chain."""
+    cfg = _tiny_cfg(T=6, has_fc2_bias=True, has_shared=True)
+    inp = gen.make_inputs(cfg, seed=24, bias_std=0.1)
+    sh = oracle.to_f64(inp.shared)
+    y1 = oracle.forward(inp)["y"]
+    y3 = oracle.forward(dataclasses.replace(inp, cfg=dataclasses.replace(cfg, expert_output_scale=3.0)))["y"]
+    r3 = oracle.forward(dataclasses.replace(inp, cfg=dataclasses.replace(cfg, routed_scaling_factor=3.0)))["y"]
+    np.testing.assert_allclose(y3 - sh, 3.0 * (y1 - sh), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(y3, r3, rtol=1e-14, atol=1e-14)
+    # 0 reads as 1
+    y0 = oracle.forward(dataclasses.replace(inp, cfg=dataclasses.replace(cfg, expert_output_scale=0.0)))["y"]
+    np.testing.assert_array_equal(y0, y1)
+
+
 # -------------------------------------------------------- routing options (MoE page)
 
 def test_golden_grouped_routing_examples():
@@ -516,6 +604,9 @@ LITERAL_CASES = [
     dict(fusion=0, act=gen.ACT_IDENTITY, bits=8, block_size=16),
     dict(alpha=1.702, beta=1.0, limit=0.5, has_fc1_bias=True, has_fc2_bias=True, has_shared=True),
     dict(act_dtype=gen.DT_BF16, scale_dtype=gen.DT_BF16, k=3, E=5),
+    dict(has_score_bias=True, k=3, E=6, normalize=False),
+    dict(fusion=0, act=gen.ACT_GELU, gelu_mode=1, has_fc1_bias=True, expert_output_scale=1.5, has_fc2_bias=True),
+    dict(fusion=1, act=gen.ACT_GELU, gelu_mode=1, has_score_bias=True, expert_output_scale=0.5),
 ]
 
 

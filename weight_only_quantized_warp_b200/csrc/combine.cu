@@ -2,7 +2,8 @@
 //
 // y[t] = rsf * sum_j w[t, j] * (o[inv[t, j]] + b2[e_j]) + shared[t], j in
 // list order, fp32, rounded once to the output dtype (rsf: the
-// routed_scaling_factor; w = 1 when the weights scaled the expert inputs). The "MoE" page
+// routed_scaling_factor times the expert_output_scale; w = 1 when the
+// weights scaled the expert inputs). The "MoE" page
 // (clika_runtime.nn) combines the expert outputs under the router weights;
 // "ClikaRT::nn::QMoEWoQ" forward() folds the optional shared_output into this
 // routed combine (no separate add pass). Reading: the fc2 bias belongs to the

@@ -215,6 +215,10 @@ qmoe_status validate(const qmoe_config& c, std::string& why) {
         return bad(QMOE_INVALID_ARGUMENT, "apply_router_weight_on_input must be 0 or 1");
     if (!(c.routed_scaling_factor >= 0.0f) || !std::isfinite(c.routed_scaling_factor))
         return bad(QMOE_INVALID_ARGUMENT, "routed_scaling_factor must be finite and >= 0");
+    if (!(c.expert_output_scale >= 0.0f) || !std::isfinite(c.expert_output_scale))
+        return bad(QMOE_INVALID_ARGUMENT, "expert_output_scale must be finite and >= 0");
+    if (c.gelu_mode != QMOE_GELU_ERF && c.gelu_mode != QMOE_GELU_TANH)
+        return bad(QMOE_INVALID_ARGUMENT, "gelu_mode must be QMOE_GELU_ERF or QMOE_GELU_TANH");
     return QMOE_OK;
 }
 
@@ -273,7 +277,35 @@ qmoe_status qmoe_create(const qmoe_config* cfg, qmoe_handle** out) {
 void qmoe_destroy(qmoe_handle* h) {
     if (!h) return;
     free_pack(h->w1, h->s1, h->b1, h->w2, h->s2, h->b2);
+    cudaFree(h->score_bias);
     delete h;
+}
+
+qmoe_status qmoe_set_score_correction_bias(qmoe_handle* h, const void* bias, void* stream) {
+    if (!h) return QMOE_INVALID_ARGUMENT;
+    std::lock_guard<std::mutex> lock(h->mu);
+    if (reinterpret_cast<uintptr_t>(bias) & 3)
+        return fail(h, QMOE_INVALID_ARGUMENT, "e_score_correction_bias must be 4-byte aligned");
+    if (!bias) {
+        cudaFree(h->score_bias);
+        h->score_bias = nullptr;
+        return QMOE_OK;
+    }
+    const size_t n = size_t(h->cfg.num_experts) * sizeof(float);
+    float* dst = h->score_bias;
+    cudaError_t err = cudaSuccess;
+    if (!dst && (err = cudaMalloc((void**)&dst, n)) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(h, QMOE_OUT_OF_MEMORY, "cudaMalloc for e_score_correction_bias: %s", cudaGetErrorString(err));
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((err = cudaMemcpyAsync(dst, bias, n, cudaMemcpyDeviceToDevice, st)) != cudaSuccess ||
+        (err = cudaStreamSynchronize(st)) != cudaSuccess) {
+        if (dst != h->score_bias) cudaFree(dst);
+        return cuda_fail(h, err, "e_score_correction_bias copy");
+    }
+    h->score_bias = dst;
+    return QMOE_OK;
 }
 
 qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_s,
@@ -490,11 +522,12 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
     if (p.fused_route) {
         if ((err = launch_route_permute(router_logits, bf16, T, E, k, c.normalize_routing_weights, c.n_group,
-                                        c.topk_group, idx, tw, offsets, perm, inv, status, st)) != cudaSuccess)
+                                        c.topk_group, h->score_bias, idx, tw, offsets, perm, inv, status, st)) !=
+            cudaSuccess)
             return cuda_fail(h, err, "route+permute");
     } else {
         if ((err = launch_route(router_logits, bf16, T, E, k, c.normalize_routing_weights, c.n_group, c.topk_group,
-                                idx, tw, status, st)) != cudaSuccess)
+                                h->score_bias, idx, tw, status, st)) != cudaSuccess)
             return cuda_fail(h, err, "route");
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
         if ((err = launch_permute(idx, T, E, k, offsets, perm, inv, st)) != cudaSuccess)
@@ -517,7 +550,8 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     f1.block_size = c.block_size;
     f1.gated = h->gated;
     f1.is_fc1 = 1;
-    f1.act_type = c.activation_type;
+    f1.act_type = (c.activation_type == QMOE_ACT_GELU && c.gelu_mode == QMOE_GELU_TANH) ? kActGeluTanh
+                                                                                       : c.activation_type;
     f1.alpha = resolved_alpha(c.activation_alpha);
     f1.beta = c.activation_beta;
     f1.limit = resolved_limit(c.swiglu_limit);
@@ -599,7 +633,11 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     ca.R = p.R;
     ca.k = k;
     ca.splits = p.fc2_splits;
-    ca.rsf = c.routed_scaling_factor > 0.0f ? c.routed_scaling_factor : 1.0f;
+    // the routed sum's multiplier: routed_scaling_factor times
+    // expert_output_scale (each 0 reads as 1); both scale the expert outputs
+    // linearly, so one fp32 product applies them
+    ca.rsf = (c.routed_scaling_factor > 0.0f ? c.routed_scaling_factor : 1.0f) *
+             (c.expert_output_scale > 0.0f ? c.expert_output_scale : 1.0f);
     ca.weights_on_input = c.apply_router_weight_on_input;
     ca.act_bf16 = bf16;
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");

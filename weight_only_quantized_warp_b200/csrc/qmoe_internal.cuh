@@ -47,6 +47,11 @@ __host__ __device__ constexpr int64_t padded_rows(int64_t n) {
     return (n + kBlockRows - 1) / kBlockRows * kBlockRows;
 }
 
+// Activation code passed to the kernels for GELU in its tanh form
+// (activation_type GELU with gelu_mode QMOE_GELU_TANH); the other codes are
+// the public QMOE_ACT_* values.
+constexpr int kActGeluTanh = 5;
+
 // Hot-path selection.
 enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2, kPathTcDecode = 3, kPathI8 = 4 };
 
@@ -83,6 +88,7 @@ struct qmoe_handle {
     float* b2 = nullptr;  // [E, H] fp32, nullptr when no fc2 bias
     int device = -1;
     int path_override = -1;  // QMOE_OPT_PATH; -1 = choose by shape
+    float* score_bias = nullptr;  // e_score_correction_bias [E] fp32, or nullptr
     uint64_t wait_limit_ns = 2000000000ull;  // QMOE_OPT_WAIT_LIMIT_NS
     int withhold = 0;        // QMOE_OPT_TEST_WITHHOLD
     mutable std::mutex mu;
@@ -117,14 +123,17 @@ struct PackArgs {
 };
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t st);
 
-// Top-k softmax routing: warp per token.
+// Top-k softmax routing: warp per token. sbias (nullable): per-expert bias of
+// the selection keys.
 cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int n_group,
-                         int topk_group, int32_t* topk_idx, float* topk_w, int32_t* status, cudaStream_t st);
+                         int topk_group, const float* sbias, int32_t* topk_idx, float* topk_w, int32_t* status,
+                         cudaStream_t st);
 // Routing and permutation of at most kFusedRouteTokens tokens in one launch.
 constexpr int64_t kFusedRouteTokens = 64;
 cudaError_t launch_route_permute(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
-                                 int n_group, int topk_group, int32_t* topk_idx, float* topk_w, int32_t* offsets,
-                                 int32_t* perm_tok, int32_t* inv, int32_t* status, cudaStream_t st);
+                                 int n_group, int topk_group, const float* sbias, int32_t* topk_idx, float* topk_w,
+                                 int32_t* offsets, int32_t* perm_tok, int32_t* inv, int32_t* status,
+                                 cudaStream_t st);
 
 // Histogram, scan and stable scatter into per-expert segments (one CTA).
 // prepare_route_permute() raises the permute kernel's shared-memory limit on

@@ -28,22 +28,29 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
 // Route token t with one warp (lane = this thread's lane). With n_group > 1
 // the experts form n_group consecutive groups; only the topk_group groups of
 // largest member logit (ties to the lower group id) may be selected.
+// sbias (nullable): the e_score_correction_bias. It moves the selection
+// only: experts and groups are ranked by the key fp32(logit + bias), the
+// weights stay the softmax of the unbiased logits.
 __device__ __forceinline__ void route_token(const void* logits, int act_bf16, int64_t t, int E, int k,
                                             int normalize, int n_group, int topk_group,
+                                            const float* __restrict__ sbias,
                                             int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                                             int lane) {
-    float v[kMaxPerLane];
+    float v[kMaxPerLane];   // selection keys
+    float lv[kMaxPerLane];  // logits
     const int per = (E + 31) >> 5;
 #pragma unroll
     for (int i = 0; i < kMaxPerLane; ++i) {
         const int e = lane + 32 * i;
-        v[i] = 0.0f;
+        v[i] = lv[i] = 0.0f;
         if (i < per && e < E) {
-            v[i] = act_bf16 ? __bfloat162float(((const __nv_bfloat16*)logits)[t * E + e])
-                            : ((const float*)logits)[t * E + e];
+            lv[i] = act_bf16 ? __bfloat162float(((const __nv_bfloat16*)logits)[t * E + e])
+                             : ((const float*)logits)[t * E + e];
             // a NaN logit never wins a comparison; read as -inf it still
             // loses to every number and ties resolve by id, so every
             // selected index is a real expert
+            if (isnan(lv[i])) lv[i] = -INFINITY;
+            v[i] = sbias ? __fadd_rn(lv[i], sbias[e]) : lv[i];
             if (isnan(v[i])) v[i] = -INFINITY;
         }
     }
@@ -51,14 +58,20 @@ __device__ __forceinline__ void route_token(const void* logits, int act_bf16, in
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kMaxPerLane; ++i)
-        if (i < per && lane + 32 * i < E) mx = fmaxf(mx, v[i]);
+        if (i < per && lane + 32 * i < E) mx = fmaxf(mx, lv[i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    // softmax denominator over all E (fixed reduction tree)
+    // softmax numerators and denominator over all E (fixed reduction tree)
+    float ex[kMaxPerLane];
     float z = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i)
-        if (i < per && lane + 32 * i < E) z += expf(v[i] - mx);
+    for (int i = 0; i < kMaxPerLane; ++i) {
+        ex[i] = 0.0f;
+        if (i < per && lane + 32 * i < E) {
+            ex[i] = expf(lv[i] - mx);
+            z += ex[i];
+        }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
 
@@ -125,7 +138,12 @@ __device__ __forceinline__ void route_token(const void* logits, int act_bf16, in
             }
         }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        const float p = expf(bv - mx);
+        // the selected expert's softmax numerator, from the lane that holds it
+        float mine = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kMaxPerLane; ++i)
+            if (i == (be >> 5)) mine = ex[i];
+        const float p = __shfl_sync(0xffffffffu, mine, be & 31);
         sel += p;
         if ((j & 31) == lane) p_keep[j >> 5] = p;
         if (lane == 0) topk_idx[t * k + j] = be;
@@ -141,12 +159,13 @@ __device__ __forceinline__ void route_token(const void* logits, int act_bf16, in
 // One warp per token. Thread 0 also clears the workspace status word, which
 // no kernel of the forward has written yet.
 __global__ void route_kernel(const void* logits, int act_bf16, int64_t T, int E, int k,
-                             int normalize, int n_group, int topk_group, int32_t* __restrict__ topk_idx,
-                             float* __restrict__ topk_w, int32_t* __restrict__ status) {
+                             int normalize, int n_group, int topk_group, const float* __restrict__ sbias,
+                             int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                             int32_t* __restrict__ status) {
     if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
     const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
-    route_token(logits, act_bf16, t, E, k, normalize, n_group, topk_group, topk_idx, topk_w,
+    route_token(logits, act_bf16, t, E, k, normalize, n_group, topk_group, sbias, topk_idx, topk_w,
                 threadIdx.x & 31);
 }
 
@@ -286,13 +305,14 @@ __device__ __forceinline__ void permute_warp(const int32_t* __restrict__ topk_id
 // first.
 __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
     const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int n_group, int topk_group,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv, int32_t* __restrict__ status) {
+    const float* __restrict__ sbias, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv,
+    int32_t* __restrict__ status) {
     extern __shared__ uint32_t sm[];
     if (threadIdx.x == 0) *status = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int64_t t = warp; t < T; t += kWarps)
-        route_token(logits, act_bf16, t, E, k, normalize, n_group, topk_group, topk_idx, topk_w, lane);
+        route_token(logits, act_bf16, t, E, k, normalize, n_group, topk_group, sbias, topk_idx, topk_w, lane);
     __syncthreads();
     if (warp == 0) {
         int32_t* cnt = reinterpret_cast<int32_t*>(sm);
@@ -303,12 +323,13 @@ __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
 }  // namespace
 
 cudaError_t launch_route(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize, int n_group,
-                         int topk_group, int32_t* topk_idx, float* topk_w, int32_t* status, cudaStream_t st) {
+                         int topk_group, const float* sbias, int32_t* topk_idx, float* topk_w, int32_t* status,
+                         cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int threads = 256;
     const int64_t blocks = (T * 32 + threads - 1) / threads;
     route_kernel<<<unsigned(blocks), threads, 0, st>>>(logits, act_bf16, T, E, k, normalize, n_group, topk_group,
-                                                       topk_idx, topk_w, status);
+                                                       sbias, topk_idx, topk_w, status);
     return cudaGetLastError();
 }
 
@@ -317,10 +338,12 @@ size_t permute_smem_bytes(int E) {
 }
 
 cudaError_t launch_route_permute(const void* logits, int act_bf16, int64_t T, int E, int k, int normalize,
-                                 int n_group, int topk_group, int32_t* topk_idx, float* topk_w, int32_t* offsets,
-                                 int32_t* perm_tok, int32_t* inv, int32_t* status, cudaStream_t st) {
+                                 int n_group, int topk_group, const float* sbias, int32_t* topk_idx, float* topk_w,
+                                 int32_t* offsets, int32_t* perm_tok, int32_t* inv, int32_t* status,
+                                 cudaStream_t st) {
     route_permute_kernel<<<1, kPermThreads, permute_smem_bytes(E), st>>>(
-        logits, act_bf16, T, E, k, normalize, n_group, topk_group, topk_idx, topk_w, offsets, perm_tok, inv, status);
+        logits, act_bf16, T, E, k, normalize, n_group, topk_group, sbias, topk_idx, topk_w, offsets, perm_tok, inv,
+        status);
     return cudaGetLastError();
 }
 

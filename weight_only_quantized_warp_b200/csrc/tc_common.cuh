@@ -299,6 +299,7 @@ __device__ __forceinline__ float act_plain(int t, float a) {
     switch (t) {
         case QMOE_ACT_RELU: return fmaxf(a, 0.0f);
         case QMOE_ACT_GELU: return 0.5f * a * (1.0f + erff(a * 0.70710678118654752f));
+        case kActGeluTanh: return 0.5f * a * (1.0f + tanhf(0.79788456080286536f * (a + 0.044715f * a * a * a)));
         case QMOE_ACT_SILU: return a * sigmoidf_(a);
         default: return a;
     }

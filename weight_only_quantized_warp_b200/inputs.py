@@ -81,6 +81,12 @@ class MoEConfig:
     weight_format: int = WEIGHTS_INT
     # COMPUTE_INT8_BLOCK: the activations are rounded per K block to int8
     compute_mode: int = COMPUTE_FLOAT
+    # MoE page options: a multiplier of every expert output (0 reads as 1)
+    # and the GELU form (0 erf, 1 tanh); set_weights' e_score_correction_bias
+    # ([E] fp32, drawn when has_score_bias)
+    expert_output_scale: float = 1.0
+    gelu_mode: int = 0
+    has_score_bias: bool = False
 
     @property
     def gated(self) -> bool:
@@ -107,6 +113,7 @@ class MoEInputs:
     fc3_s: Optional[np.ndarray] = None
     fc3_b: Optional[np.ndarray] = None
     shared: Optional[np.ndarray] = None
+    score_bias: Optional[np.ndarray] = None   # [E] float32
 
 
 def _store(a: np.ndarray, dtype: int) -> np.ndarray:
@@ -182,6 +189,8 @@ def make_inputs(cfg: MoEConfig, seed: int, logits: str = "normal",
         inp.fc3_b = _store(rng.standard_normal((E, I)) * bias_std, cfg.act_dtype)
     if cfg.has_shared:
         inp.shared = _store(rng.standard_normal((T, H)), cfg.act_dtype)
+    if cfg.has_score_bias:
+        inp.score_bias = (rng.standard_normal(E) * 0.5).astype(np.float32)
     return inp
 
 

@@ -30,6 +30,7 @@ ACT_RELU, ACT_GELU, ACT_SILU, ACT_SWIGLU, ACT_IDENTITY = 0, 1, 2, 3, 4
 DTYPE_F32, DTYPE_BF16, DTYPE_E8M0 = 0, 1, 2
 WEIGHTS_INT, WEIGHTS_MXFP4 = 0, 1
 COMPUTE_FLOAT, COMPUTE_INT8_BLOCK = 0, 1
+GELU_ERF, GELU_TANH = 0, 1
 PATH_SIMT, PATH_DECODE, PATH_TC, PATH_TC_DECODE, PATH_INT8 = 0, 1, 2, 3, 4
 
 # Every function the header declares (checked against include/qmoe.h by the tests).
@@ -39,7 +40,7 @@ EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forwa
            "qmoe_status_string", "qmoe_last_error", "qmoe_path_for", "qmoe_launches_for",
            "qmoe_token_tile_for",
            "qmoe_set_option", "qmoe_forward_noalloc", "qmoe_noalloc_scratch_bytes",
-           "qmoe_noalloc_read_device_status",
+           "qmoe_noalloc_read_device_status", "qmoe_set_score_correction_bias",
            "qmoe_quantize_act_i8")
 QMOE_OPT_PATH, QMOE_OPT_WAIT_LIMIT_NS, QMOE_OPT_TEST_WITHHOLD = 1, 2, 3
 
@@ -57,7 +58,8 @@ class qmoe_config(ctypes.Structure):
                 ("use_sparse_mixer", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
                 ("routed_scaling_factor", ctypes.c_float), ("apply_router_weight_on_input", ctypes.c_int32),
-                ("weight_format", ctypes.c_int32), ("compute_mode", ctypes.c_int32)]
+                ("weight_format", ctypes.c_int32), ("compute_mode", ctypes.c_int32),
+                ("expert_output_scale", ctypes.c_float), ("gelu_mode", ctypes.c_int32)]
 
 
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
@@ -92,6 +94,8 @@ lib.qmoe_noalloc_scratch_bytes.restype = _sz
 lib.qmoe_noalloc_scratch_bytes.argtypes = []
 lib.qmoe_noalloc_read_device_status.restype = ctypes.c_int
 lib.qmoe_noalloc_read_device_status.argtypes = [_vp, _vp]
+lib.qmoe_set_score_correction_bias.restype = ctypes.c_int
+lib.qmoe_set_score_correction_bias.argtypes = [_vp, _vp, _vp]
 lib.qmoe_set_option.restype = ctypes.c_int
 lib.qmoe_set_option.argtypes = [_vp, ctypes.c_int32, _i64]
 lib.qmoe_launches_for.restype = ctypes.c_int32
@@ -152,7 +156,9 @@ def make_config(cfg) -> qmoe_config:
         routed_scaling_factor=float(getattr(cfg, "routed_scaling_factor", 1.0)),
         apply_router_weight_on_input=int(getattr(cfg, "apply_router_weight_on_input", False)),
         weight_format=int(getattr(cfg, "weight_format", 0)),
-        compute_mode=int(getattr(cfg, "compute_mode", 0)))
+        compute_mode=int(getattr(cfg, "compute_mode", 0)),
+        expert_output_scale=float(getattr(cfg, "expert_output_scale", 1.0)),
+        gelu_mode=int(getattr(cfg, "gelu_mode", 0)))
 
 
 def qmoe_create(cfg: qmoe_config) -> int:
@@ -165,6 +171,12 @@ def qmoe_set_weights(h, fc1_w, fc1_s, fc1_b, fc2_w, fc2_s, fc2_b, fc3_w=None, fc
                      fc3_b=None, stream=None):
     _check(lib.qmoe_set_weights(h, _ptr(fc1_w), _ptr(fc1_s), _ptr(fc1_b), _ptr(fc2_w), _ptr(fc2_s),
                                 _ptr(fc2_b), _ptr(fc3_w), _ptr(fc3_s), _ptr(fc3_b), _stream(stream)), h)
+
+
+def qmoe_set_score_correction_bias(h, bias, stream=None):
+    """Bind the e_score_correction_bias ([E] fp32 device tensor, or None to
+    clear); it moves the expert selection only."""
+    _check(lib.qmoe_set_score_correction_bias(h, _ptr(bias), _stream(stream)), h)
 
 
 def qmoe_workspace_size(h, T: int) -> int:
@@ -287,6 +299,8 @@ class QMoE:
              ("fc1_w", "fc1_s", "fc1_b", "fc2_w", "fc2_s", "fc2_b", "fc3_w", "fc3_s", "fc3_b")}
         self.set_weights(t["fc1_w"], t["fc1_s"], t["fc2_w"], t["fc2_s"], t["fc1_b"], t["fc2_b"],
                          t["fc3_w"], t["fc3_s"], t["fc3_b"], stream)
+        sb = getattr(inp, "score_bias", None)
+        qmoe_set_score_correction_bias(self.handle, to_device(sb, d) if sb is not None else None, stream)
 
     def workspace(self, T: int):
         import torch
