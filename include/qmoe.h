@@ -378,6 +378,12 @@ enum { QMOE_OPT_PATH = 1 };
  * forward with the option back at 0 is a normal one. */
 enum { QMOE_OPT_WAIT_LIMIT_NS = 2, QMOE_OPT_TEST_WITHHOLD = 3 };
 
+/* QMOE_OPT_PDL (0 or 1, default 1): launch the weight-streaming kernels of
+ * path 1 and the combine as programmatic dependents of the kernel before
+ * them, so each starts streaming its weights while the previous one drains;
+ * 0 launches every kernel in plain stream order. Results are identical. */
+enum { QMOE_OPT_PDL = 4 };
+
 /* qmoe_set_option -- set a tunable option on the handle. QMOE_INVALID_ARGUMENT
  * for an unknown option or value. Not thread-safe against concurrent
  * qmoe_forward calls on the same handle. */

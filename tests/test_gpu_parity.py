@@ -237,6 +237,28 @@ def test_repeated_forward_is_bitwise_deterministic(cuda_device, path):
     np.testing.assert_array_equal(a.hidden, b.hidden)
 
 
+@pytest.mark.parametrize("name", ["mixtral_decode", "sweep_int8_T16"])
+def test_dependent_launch_changes_nothing(cuda_device, name):
+    """The weight-streaming kernels launched as programmatic dependents (the
+    default) give bitwise the same output as plain stream-ordered launches."""
+    import torch
+    from weight_only_quantized_warp_b200 import qmoe
+    cfg, seed, kw = gen.workload(name)
+    inp = gen.make_inputs(cfg, seed, **kw)
+    m = qmoe.QMoE(cfg, "cuda:0")
+    m.set_weights_from(inp)
+    x = qmoe.to_device(inp.x, "cuda:0")
+    lg = qmoe.to_device(inp.logits, "cuda:0")
+    outs = []
+    for pdl in (1, 0, 1):
+        qmoe.qmoe_set_option(m.handle, qmoe.QMOE_OPT_PDL, pdl)
+        for _ in range(3):
+            y = m.forward(x, lg)
+        torch.cuda.synchronize()
+        outs.append(y.clone())
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
 def test_rebind_replaces_the_pack(cuda_device):
     import torch
     from weight_only_quantized_warp_b200 import qmoe

@@ -22,6 +22,7 @@ constexpr int kCombineChunk = kCombineThreads * 4;  // elements of one row per b
 // loads of all k rows and splits are independent, so they are in flight
 // together.
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineArgs a) {
+    pdl_wait();  // every input comes from earlier kernels of the forward
     const float* __restrict__ o = a.o;
     const int nchunk = int((a.H + kCombineChunk - 1) / kCombineChunk);
     const int64_t nblk = a.T * nchunk;
@@ -87,8 +88,7 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
     if (a.T == 0) return cudaSuccess;
     int64_t blocks = a.T * ((a.H + kCombineChunk - 1) / kCombineChunk);
     if (blocks > 148 * 16) blocks = 148 * 16;
-    combine_kernel<<<unsigned(blocks), kCombineThreads, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(combine_kernel, dim3(unsigned(blocks)), dim3(kCombineThreads), 0, st, a.pdl != 0, a);
 }
 
 }  // namespace qmoe

@@ -151,9 +151,6 @@ __global__ void __launch_bounds__(kWarps * 32, 3) ffn_decode_kernel(const FfnArg
     const int64_t nrb = padded_rows(a.N) / kBlockRows;
     const int64_t rt = rb * kTilesPerBlock + warp;
     const bool active = rt < nrt;
-    const int64_t seg0 = a.offsets[e];
-    const int M = a.offsets[e + 1] - int(seg0);
-    if (M <= 0) return;  // uniform over the CTA
     const int64_t ngr = a.K / KG;
     const int64_t nsb = a.block_size > 0 ? a.K / a.block_size : 1;
     const int lg_bs = a.block_size > 0 ? __ffs(a.block_size) - 1 : 0;
@@ -185,9 +182,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3) ffn_decode_kernel(const FfnArg
     float s0 = 1.0f, s1 = 1.0f;  // per-column scales
     if (SMODE == 0 && active) ScaleRaw<SF32>::load(sbase, 0).get(s0, s1);
 
-    for (int p0 = 0; p0 < M; p0 += ROWS) {
-        uint4 wr[D];
-        ScaleRaw<SF32> sr[D / P];
+    // the first D k-groups of a pass (and their scales) in flight
+    uint4 wr[D];
+    ScaleRaw<SF32> sr[D / P];
+    auto fill = [&]() {
         if (active) {
 #pragma unroll
             for (int i = 0; i < D; ++i) {
@@ -197,6 +195,20 @@ __global__ void __launch_bounds__(kWarps * 32, 3) ffn_decode_kernel(const FfnArg
                 }
             }
         }
+    };
+    // The weights depend on nothing the forward computes, so the first pass's
+    // loads go out before the wait on the kernel before this one (routing or
+    // FC1) when launched as its programmatic dependent; the segment offsets,
+    // the row map and the activations are read only after it.
+    fill();
+    pdl_trigger();
+    pdl_wait();
+    const int64_t seg0 = a.offsets[e];
+    const int M = a.offsets[e + 1] - int(seg0);
+    if (M <= 0) return;  // uniform over the CTA
+
+    for (int p0 = 0; p0 < M; p0 += ROWS) {
+        if (p0 > 0) fill();
         // stage the activation rows of tokens p0 .. p0 + ROWS - 1 (clamped):
         // one warp per row, lanes over its 16-byte chunks
         for (int row = warp; row < ROWS; row += kWarps) {
@@ -531,8 +543,8 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
 
 template <int BITS, int SMODE, bool SF32, int NT, int P>
 cudaError_t launch_one(const FfnArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
-    ffn_decode_kernel<BITS, SMODE, SF32, NT, P><<<grid, kWarps * 32, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(ffn_decode_kernel<BITS, SMODE, SF32, NT, P>, grid, dim3(kWarps * 32), smem, st, a.pdl != 0,
+                         a);
 }
 
 template <int BITS, int SMODE, bool SF32, int P>

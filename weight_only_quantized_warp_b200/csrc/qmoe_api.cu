@@ -434,6 +434,11 @@ qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t value) {
         h->wait_limit_ns = uint64_t(value);
         return QMOE_OK;
     }
+    if (option == QMOE_OPT_PDL) {
+        if (value != 0 && value != 1) return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_PDL must be 0 or 1");
+        h->pdl = int(value);
+        return QMOE_OK;
+    }
     if (option == QMOE_OPT_TEST_WITHHOLD) {
         if (value != 0 && value != 1) return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_TEST_WITHHOLD must be 0 or 1");
         h->withhold = int(value);
@@ -562,6 +567,9 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     f1.nt = p.nt;
     f1.timeout_ns = h->wait_limit_ns;
     f1.withhold = h->withhold;
+    // the weight-streaming kernels prefetch their first weights while the
+    // kernel before them finishes (routing / gather before FC1, FC1 before FC2)
+    f1.pdl = h->pdl && p.path == kPathDecode;
     FfnArgs f2 = f1;
     f2.W = h->w2;
     f2.S = h->s2;
@@ -639,6 +647,7 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
     ca.rsf = (c.routed_scaling_factor > 0.0f ? c.routed_scaling_factor : 1.0f) *
              (c.expert_output_scale > 0.0f ? c.expert_output_scale : 1.0f);
     ca.weights_on_input = c.apply_router_weight_on_input;
+    ca.pdl = h->pdl;
     ca.act_bf16 = bf16;
     if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
     if ((err = launch_combine(ca, st)) != cudaSuccess) return cuda_fail(h, err, "combine");

@@ -9,10 +9,37 @@
 
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "qmoe.h"
 
 namespace qmoe {
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with pdl = true may start
+// while the kernel before it on the stream is still running; it must call
+// pdl_wait() before it reads anything that kernel (or an earlier one) wrote.
+// pdl_trigger() lets the next kernel's launch begin once every CTA of this
+// grid has called it or exited. Both are no-ops when no such launch is
+// involved.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 bool pdl, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------------------
 // Packed weight layout ("fragment order").
@@ -91,6 +118,7 @@ struct qmoe_handle {
     float* score_bias = nullptr;  // e_score_correction_bias [E] fp32, or nullptr
     uint64_t wait_limit_ns = 2000000000ull;  // QMOE_OPT_WAIT_LIMIT_NS
     int withhold = 0;        // QMOE_OPT_TEST_WITHHOLD
+    int pdl = 1;             // QMOE_OPT_PDL
     mutable std::mutex mu;
     mutable std::string last_error;
 };
@@ -168,6 +196,9 @@ struct FfnArgs {
     // withheld accumulator signal (QMOE_OPT_WAIT_LIMIT_NS, QMOE_OPT_TEST_WITHHOLD)
     uint64_t timeout_ns;
     int withhold;
+    // weight-streaming decode kernel: launched as a programmatic dependent of
+    // the kernel before it (prefetches weights, then waits for its inputs)
+    int pdl;
 };
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
 // Shared memory of one decode CTA (staged activation rows) and its limit;
@@ -224,6 +255,7 @@ struct CombineArgs {
     int k, splits, act_bf16;
     float rsf;               // routed_scaling_factor (1 when unset)
     int weights_on_input;    // the router weights already scaled FC1's input rows
+    int pdl;                 // launched as a programmatic dependent of FC2
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 

@@ -248,6 +248,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
     const int32_t* __restrict__ topk_idx, int64_t T, int E, int k, int32_t* __restrict__ offsets,
     int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv) {
     extern __shared__ uint32_t sm[];
+    pdl_trigger();  // the expert kernels may launch and prefetch weights meanwhile
     permute_block(topk_idx, T, E, k, offsets, perm_tok, inv, sm);
 }
 
@@ -309,6 +310,7 @@ __global__ void __launch_bounds__(kPermThreads) route_permute_kernel(
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv,
     int32_t* __restrict__ status) {
     extern __shared__ uint32_t sm[];
+    pdl_trigger();  // the expert kernels may launch and prefetch weights meanwhile
     if (threadIdx.x == 0) *status = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int64_t t = warp; t < T; t += kWarps)
