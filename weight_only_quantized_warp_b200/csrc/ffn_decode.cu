@@ -132,8 +132,11 @@ constexpr int kRing = 8;               // weight loads in flight per lane
 // has its first kRing weight loads in flight. The k-group loop has a steady
 // part (loads always in range, no guards), one guarded drain round and a
 // tail; all shared-memory, weight and scale addresses advance by constants.
+// Resident CTAs per SM the kernel is built for: three for one 8-token tile
+// (80 registers hold it), two for two or four tiles (whose accumulators and
+// activation fragments would spill at 80).
 template <int BITS, int SMODE, bool SF32, int NT, int P>
-__global__ void __launch_bounds__(kWarps * 32, 3) ffn_decode_kernel(const FfnArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, NT == 1 ? 3 : 2) ffn_decode_kernel(const FfnArgs a) {
     constexpr int KG = kgroup_of(BITS);
     constexpr int D = kRing;
     static_assert(D % P == 0, "scale chunk must divide the ring");

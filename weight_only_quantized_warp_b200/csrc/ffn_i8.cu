@@ -150,7 +150,7 @@ __host__ __device__ constexpr int64_t staged_row_bytes_i8(int64_t kr) { return k
 // has a steady part (loads always in range), one guarded drain round and a
 // tail, as in the bf16 decode kernels.
 template <int BITS, bool SF32, int NT, int P>
-__global__ void __launch_bounds__(kWarps * 32, 3) ffn_i8_kernel(const FfnArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, NT == 1 ? 3 : 2) ffn_i8_kernel(const FfnArgs a) {
     constexpr int KG = kgroup_of(BITS);
     constexpr int D = kRing;
     static_assert(D % P == 0, "scale chunk must divide the ring");
