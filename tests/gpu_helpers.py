@@ -88,7 +88,8 @@ def run_gpu(inp: gen.MoEInputs, device="cuda:0", repeat: int = 1, path=None, hid
 
 def check_routing(inp: gen.MoEInputs, g: GpuRun):
     c = inp.cfg
-    idx, w = oracle.route(inp.logits, c.k, c.normalize, c.n_group, c.topk_group)
+    idx, w = oracle.route(inp.logits, c.k, c.normalize, c.n_group, c.topk_group,
+                          score_bias=getattr(inp, "score_bias", None))
     np.testing.assert_array_equal(g.topk_idx, idx)
     np.testing.assert_allclose(g.topk_w, w, rtol=TOL_ROUTE_W, atol=1e-30)
     off, perm, inv = oracle.permute(idx, c.E)

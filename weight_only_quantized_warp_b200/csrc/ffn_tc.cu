@@ -12,18 +12,20 @@
 // dimension the routed tokens of one expert (a multiple of 16, up to 128), so
 // a small expert segment wastes no tensor work on padding rows.
 //
-// Warp roles of one persistent CTA (608 threads, one CTA per SM):
-//   warps 0-7   dequantise: packed codes (shared) -> bf16 A tile written
+// Warp roles of one persistent CTA (864 threads, one CTA per SM):
+//   warps 0-15  dequantise: packed codes (shared) -> bf16 A tile written
 //               straight into tensor memory (tcgen05.st), one 16-row tile per
-//               warp; the A operand never touches shared memory
-//   warp 8      activation producer: 64-row TMA boxes of the activations
+//               warp; two groups of eight warps take alternate stages, so two
+//               stages are decoded at once; the A operand never touches
+//               shared memory
+//   warp 16     activation producer: 64-row TMA boxes of the activations
 //               (bf16, 128-byte swizzle), as many as the tile has rows
-//   warp 18     weight producer: one bulk copy of the packed 128 x 64 tile
+//   warp 26     weight producer: one bulk copy of the packed 128 x 64 tile
 //               (4 KB int4, 8 KB int8) and one of its scales
-//   warp 9      allocates TMEM and issues tcgen05.mma (A from TMEM, B from
+//   warp 17     allocates TMEM and issues tcgen05.mma (A from TMEM, B from
 //               shared memory); producers and MMA run their loops as whole
 //               warps and predicate each issue on one elected lane
-//   warps 10-17 epilogue: TMEM -> registers (tcgen05.ld), scale / bias /
+//   warps 18-25 epilogue: TMEM -> registers (tcgen05.ld), scale / bias /
 //               activation, global stores; two warps per TMEM lane quarter
 // Stages cycle through an S-deep ring guarded by mbarriers (full: copies
 // landed; deq: A tile written to TMEM; empty: the MMAs reading the stage are
@@ -48,10 +50,10 @@
 namespace qmoe {
 namespace {
 
-constexpr int kDeqWarps = 8;
-constexpr int kWarpProd = 8;
-constexpr int kWarpMma = 9;
-constexpr int kWarpEpi0 = 10;
+constexpr int kDeqWarps = 16;                            // two groups of 8, alternate stages
+constexpr int kWarpProd = 16;
+constexpr int kWarpMma = 17;
+constexpr int kWarpEpi0 = 18;
 constexpr int kEpiWarps = 8;
 constexpr int kWarpProd2 = kWarpEpi0 + kEpiWarps;          // second producer (weights)
 constexpr int kTcThreads = (kWarpProd2 + 1) * 32;           // 608
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&full[s]), 2);  // one arrival per producer warp
-            mbar_init(smem_u32(&deq[s]), kDeqWarps);
+            mbar_init(smem_u32(&deq[s]), kDeqWarps / 2);  // one group decodes a stage
             mbar_init(smem_u32(&empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -221,9 +223,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp < kDeqWarps) {
         // ------------------------------------------------------- dequantise
-        // warp w writes row tile t = 2*(w%4) + w/4 (TMEM lanes 16t..16t+15,
-        // inside the lane quarter w%4 it may access)
-        const int tile = 2 * (warp & 3) + (warp >> 2);
+        // warp w writes row tile t = 2*(w%4) + (w/4)%2 (TMEM lanes 16t..16t+15,
+        // inside the lane quarter w%4 it may access) of the stages of parity
+        // w / 8: two groups of eight warps decode alternate stages
+        const int tile = 2 * (warp & 3) + ((warp >> 2) & 1), grp = warp >> 3;
+        int seen = 0;  // stages seen by this warp, both parities
         const int r0 = lane >> 2, c = lane & 3;
         const uint32_t lane_addr = uint32_t(16 * tile) << 16;
         int st = 0;
@@ -236,6 +240,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
             const Item it = item_at(i, prefix, a, nrb, nks);
             for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
+                if ((seen++ & 1) != grp) {  // the other group's stage
+                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                    continue;
+                }
                 if (!warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
                 const uint8_t* sb = smem + st * C::kStage;
                 const uint8_t* pk = sb + C::kB;

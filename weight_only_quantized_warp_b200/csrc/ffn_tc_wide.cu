@@ -12,13 +12,14 @@
 // MMA's shared-memory descriptor reads) instead of TMEM, and the MMA takes
 // both operands from shared memory.
 //
-// Warp roles (608 threads, one CTA per SM):
-//   warps 0-7   dequantise: one 16-row tile each, bf16 A tile into a ring of
-//               shared-memory slots (st.shared, then an async-proxy fence)
-//   warp 8      activation producer: 64-row TMA boxes (up to four per stage)
-//   warp 18     weight producer: packed 128 x 64 tile and its scales (bulk)
-//   warp 9      TMEM allocation and MMA issue (converged warp, elected lane)
-//   warps 10-17 epilogue, shared with ffn_tc.cu
+// Warp roles (864 threads, one CTA per SM):
+//   warps 0-15  dequantise: two groups of eight take alternate stages; a warp
+//               decodes one 16-row tile into a ring of shared-memory A slots
+//               (st.shared, then an async-proxy fence)
+//   warp 16     activation producer: 64-row TMA boxes (up to four per stage)
+//   warp 26     weight producer: packed 128 x 64 tile and its scales (bulk)
+//   warp 17     TMEM allocation and MMA issue (converged warp, elected lane)
+//   warps 18-25 epilogue, shared with ffn_tc.cu
 // Every wait is bounded (about two seconds, then QMOE_TIMEOUT in the
 // workspace status word; every role leaves its loop and the CTA frees TMEM).
 #include "qmoe_internal.cuh"
@@ -30,10 +31,10 @@ namespace {
 
 constexpr int kWBK = 64;             // k per stage
 constexpr int kWN = 256;             // token-tile width (MMA N)
-constexpr int kWDeqWarps = 8;
-constexpr int kWWarpProd = 8;
-constexpr int kWWarpMma = 9;
-constexpr int kWEpi0 = 10;
+constexpr int kWDeqWarps = 16;            // two groups of 8, alternate stages
+constexpr int kWWarpProd = 16;
+constexpr int kWWarpMma = 17;
+constexpr int kWEpi0 = 18;
 constexpr int kWEpiWarps = 8;
 constexpr int kWWarpProd2 = kWEpi0 + kWEpiWarps;  // 18
 constexpr int kWThreads = (kWWarpProd2 + 1) * 32;  // 608
@@ -46,8 +47,8 @@ struct WideCfg {
     static constexpr int kPacked = kBlockRows * kWBK * BITS / 8;
     static constexpr int kStage = kB + kPacked + kWScaleMax;   // activations, codes, scales
     static constexpr int kA = kBlockRows * 128;                // decoded A tile, 16 KB
-    static constexpr int kAS = 3;                              // A-tile slots
-    static constexpr int kStages = (220 * 1024 - kAS * kA) / kStage;  // 4 (int4) / 4 (int8)
+    static constexpr int kAS = BITS == 4 ? 4 : 3;              // A-tile slots
+    static constexpr int kStages = (222 * 1024 - kAS * kA) / kStage;  // 4 (int4) / 4 (int8)
     static constexpr int kAOff = kStages * kStage;             // multiple of 1024
     static constexpr int kBarOff = kAOff + kAS * kA;
     static constexpr int kBarBytes = 2048;
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
             mbar_init(smem_u32(&empty[s]), 1);
         }
         for (int s = 0; s < AS; ++s) {
-            mbar_init(smem_u32(&afull[s]), kWDeqWarps);
+            mbar_init(smem_u32(&afull[s]), kWDeqWarps / 2);  // one group writes a slot
             mbar_init(smem_u32(&aempty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -204,8 +205,11 @@ __global__ void __launch_bounds__(kWThreads, 1)
         }
     } else if (warp < kWDeqWarps) {
         // ------------------------------------------------------- dequantise
-        // warp w decodes row tile w (rows 16w .. 16w + 15 of the 128-row block)
-        const int tile = warp;
+        // warp w decodes row tile w % 8 (rows 16 (w % 8) .. + 15 of the 128-row
+        // block) of the stages of parity w / 8: two groups of eight warps take
+        // alternate stages, so two stages are decoded at once
+        const int tile = warp & 7, grp = warp >> 3;
+        int seen = 0;  // stages seen by this warp, both parities
         const int r0 = lane >> 2, c = lane & 3;
         const int rA = 16 * tile + r0;  // and rA + 8; both have (row & 7) == r0
         int st = 0, as = 0;
@@ -216,6 +220,11 @@ __global__ void __launch_bounds__(kWThreads, 1)
         for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
             const Item it = item_at(i, prefix, a, nrb, nks);
             for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
+                if ((seen++ & 1) != grp) {  // the other group's stage
+                    if (++st == ST) { st = 0; ph ^= 1u; }
+                    if (++as == AS) { as = 0; aph ^= 1u; }
+                    continue;
+                }
                 if (!warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status, a.timeout_ns) ||
                     !warp_wait(smem_u32(&aempty[as]), aph ^ 1u, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
                 const uint8_t* pk = smem + st * C::kStage + C::kB;

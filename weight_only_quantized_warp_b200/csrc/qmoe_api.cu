@@ -63,16 +63,30 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         p.nt = per_expert <= 8 ? 1 : (per_expert <= 16 ? 2 : 4);
         // FC1 runs unsplit; keep its staged rows small enough for at least two CTAs per SM
         while (p.nt > 1 && smem(H, 1, p.nt) > kDecodeSmemTarget) p.nt /= 2;
-        // enough FC2 warps (one per 16-row tile per touched expert per split)
-        // to give every SM several resident warps
-        const int64_t warps = touched * (H / kTileRows);
-        const int64_t want = kSms * 48;
+        // FC2 split-K: every CTA (one 128-row block of one touched expert and
+        // one split) streams the same bytes, so the launch takes about
+        // ceil(CTAs / slots) rounds of the resident CTA slots; take the split
+        // count (1..8, staged rows within the shared-memory target) whose
+        // CTAs fill those rounds best, the fewest splits on a tie
         const int64_t ngr = I / kgroup_of(bits);
-        int64_t s = ceil_div(want, warps);
-        s = std::min<int64_t>(s, 8);
-        while (s < ngr && smem(I, int(s), p.nt) > kDecodeSmemTarget) ++s;
-        s = std::min<int64_t>(s, ngr);
-        p.fc2_splits = int(std::max<int64_t>(s, 1));
+        const int64_t slots = kSms * (p.nt == 1 ? 3 : 2);
+        const int64_t blocks = touched * (padded_rows(H) / kBlockRows);
+        int64_t best = 0;
+        double best_eff = -1.0;
+        for (int64_t s = 1; s <= std::min<int64_t>(8, ngr); ++s) {
+            if (smem(I, int(s), p.nt) > kDecodeSmemTarget) continue;
+            const int64_t ctas = blocks * s;
+            const double eff = double(ctas) / double(slots * ceil_div(ctas, slots));
+            if (eff > best_eff + 1e-9) {
+                best_eff = eff;
+                best = s;
+            }
+        }
+        if (best == 0) {  // no split count fits the target: the smallest that fits the limit
+            best = 1;
+            while (best < ngr && smem(I, int(best), p.nt) > kDecodeSmemTarget) ++best;
+        }
+        p.fc2_splits = int(best);
         p.ok = smem(H, 1, p.nt) <= int64_t(kDecodeSmemLimit) &&
                smem(I, p.fc2_splits, p.nt) <= int64_t(kDecodeSmemLimit);
     } else if (p.path == kPathTc) {
