@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT == 1 ? 3 : 2) ffn_decode_kerne
                     v[2] *= s1;
                     v[3] *= s1;
                 }
-                epilogue(a, rt, r0, c, seg0, M, p0 + 8 * n, v, split, true);
+                epilogue(a, e, rt, r0, c, seg0, M, p0 + 8 * n, v, split, true);
             }
         }
         __syncthreads();  // the next pass restages xs
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_simt_kernel(const FfnArgs a) 
                 v[3] = acc[n][1];
             }
         }
-        epilogue(a, rt, r0, c, seg0, M, p0, v, split, false);
+        epilogue(a, e, rt, r0, c, seg0, M, p0, v, split, false);
     }
 }
 

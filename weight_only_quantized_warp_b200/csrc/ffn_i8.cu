@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kWarps * 32, NT == 1 ? 3 : 2) ffn_i8_kernel(co
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
                 const float v[4] = {acc[n][0], acc[n][1], acc[n][2], acc[n][3]};
-                epilogue(a, rt, r0, c, seg0, M, p0 + 8 * n, v, split, a.act_bf16 != 0);
+                epilogue(a, e, rt, r0, c, seg0, M, p0 + 8 * n, v, split, a.act_bf16 != 0);
             }
         }
         __syncthreads();  // the next pass restages xs

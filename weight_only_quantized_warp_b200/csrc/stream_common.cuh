@@ -53,16 +53,17 @@ __device__ __forceinline__ void store_act(void* p, int64_t i, float v, bool bf16
 
 // Shared epilogue. v[0..3] are the MMA C-fragment values of lane (r0, c):
 // (row r0, token 2c), (row r0, token 2c+1), (row r0+8, token 2c),
-// (row r0+8, token 2c+1) of one 8-token tile starting at segment row p.
-__device__ __forceinline__ void epilogue(const FfnArgs& a, int64_t rt, int r0, int c, int64_t seg0,
+// (row r0+8, token 2c+1) of one 8-token tile starting at segment row p of
+// expert e.
+__device__ __forceinline__ void epilogue(const FfnArgs& a, int e, int64_t rt, int r0, int c, int64_t seg0,
                                          int M, int p, const float (&v)[4], int split, bool out_bf16) {
     const int tA = p + 2 * c, tB = tA + 1;
     if (a.is_fc1) {
         if (a.gated) {
             const int64_t I = a.N / 2;
             const int64_t i = rt * 8 + r0;
-            const float bg = a.bias ? a.bias[(int64_t)blockIdx.y * a.N + rt * 16 + r0] : 0.0f;
-            const float bu = a.bias ? a.bias[(int64_t)blockIdx.y * a.N + rt * 16 + r0 + 8] : 0.0f;
+            const float bg = a.bias ? a.bias[(int64_t)e * a.N + rt * 16 + r0] : 0.0f;
+            const float bu = a.bias ? a.bias[(int64_t)e * a.N + rt * 16 + r0 + 8] : 0.0f;
             if (tA < M)
                 store_act(a.out, (seg0 + tA) * I + i,
                           act_gated(a.act_type, v[0] + bg, v[2] + bu, a.alpha, a.beta, a.limit),
@@ -74,8 +75,8 @@ __device__ __forceinline__ void epilogue(const FfnArgs& a, int64_t rt, int r0, i
         } else {
             const int64_t I = a.N;
             const int64_t m0 = rt * 16 + r0, m1 = m0 + 8;
-            const float b0 = a.bias ? a.bias[(int64_t)blockIdx.y * a.N + m0] : 0.0f;
-            const float b1 = a.bias ? a.bias[(int64_t)blockIdx.y * a.N + m1] : 0.0f;
+            const float b0 = a.bias ? a.bias[(int64_t)e * a.N + m0] : 0.0f;
+            const float b1 = a.bias ? a.bias[(int64_t)e * a.N + m1] : 0.0f;
             if (tA < M) {
                 store_act(a.out, (seg0 + tA) * I + m0, act_plain(a.act_type, v[0] + b0), out_bf16);
                 store_act(a.out, (seg0 + tA) * I + m1, act_plain(a.act_type, v[2] + b1), out_bf16);
