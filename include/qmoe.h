@@ -384,6 +384,14 @@ enum { QMOE_OPT_WAIT_LIMIT_NS = 2, QMOE_OPT_TEST_WITHHOLD = 3 };
  * 0 launches every kernel in plain stream order. Results are identical. */
 enum { QMOE_OPT_PDL = 4 };
 
+/* QMOE_OPT_DECODE_TILES (0, 1, 2 or 4; default 0): 8-token tiles per pass of
+ * the weight-streaming kernels (paths 1 and 4); 0 chooses by the average rows
+ * per expert. Fewer are taken where the staged activation rows of a pass
+ * would not fit two CTAs per SM. An expert segment longer than one pass
+ * streams its weights once per pass. Results agree with the oracle for every
+ * value. */
+enum { QMOE_OPT_DECODE_TILES = 5 };
+
 /* qmoe_set_option -- set a tunable option on the handle. QMOE_INVALID_ARGUMENT
  * for an unknown option or value. Not thread-safe against concurrent
  * qmoe_forward calls on the same handle. */

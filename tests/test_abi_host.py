@@ -106,8 +106,10 @@ def test_create_accepts_and_plans_without_gpu(q):
         assert q.qmoe_workspace_size(h, -1) == 0
         assert q.qmoe_path_for(h, 8) == q.PATH_DECODE
         assert q.qmoe_launches_for(h, 8) == 4     # route+permute, FC1, FC2, combine
-        assert q.qmoe_launches_for(h, 64) == 4
-        assert q.qmoe_launches_for(h, 65) == 6    # tensor-core path: route, permute, gather, ...
+        assert q.qmoe_launches_for(h, 32) == 4
+        assert q.qmoe_launches_for(h, 33) == 5    # tensor-core path: route+permute, gather, FC1, FC2, combine
+        assert q.qmoe_launches_for(h, 64) == 5
+        assert q.qmoe_launches_for(h, 65) == 6    # route, permute, gather, ...
         assert q.qmoe_launches_for(h, 0) == 0
         assert q.qmoe_token_tile_for(h, 8) == 0  # decode path: no token tile
         assert q.qmoe_token_tile_for(h, -1) == -1
@@ -119,10 +121,12 @@ def test_create_accepts_and_plans_without_gpu(q):
     q.qmoe_destroy(None)  # no-op
 
 
-@pytest.mark.parametrize("T,path,tile", [(8, 1, 0), (96, 2, 32), (384, 2, 128), (2048, 2, 256)])
+@pytest.mark.parametrize("T,path,tile", [(8, 1, 0), (32, 1, 0), (33, 2, 16), (96, 2, 32), (128, 2, 64),
+                                         (384, 2, 128), (2048, 2, 256)])
 def test_plan_token_tile_covers_the_average_segment(q, T, path, tile):
-    # 8 experts, k = 2: T*2/8 rows per expert on average; the tile is the
-    # power of two covering 4/3 of that, at most 256
+    # 8 experts, k = 2: T*2/8 rows per expert on average; up to 8 the weights
+    # stream (no token tile), above it the tile is the power of two covering
+    # 4/3 of that, at most 256
     h = q.qmoe_create(_cfg(q))
     try:
         assert q.qmoe_path_for(h, T) == path
@@ -167,10 +171,12 @@ def test_wait_limit_and_withhold_options_are_validated(q):
     h = q.qmoe_create(_cfg(q))
     try:
         for opt, val in [(q.QMOE_OPT_WAIT_LIMIT_NS, 99999), (q.QMOE_OPT_WAIT_LIMIT_NS, 61 * 10**9),
-                         (q.QMOE_OPT_TEST_WITHHOLD, 2), (q.QMOE_OPT_TEST_WITHHOLD, -1), (99, 0)]:
+                         (q.QMOE_OPT_TEST_WITHHOLD, 2), (q.QMOE_OPT_TEST_WITHHOLD, -1), (99, 0),
+                         (q.QMOE_OPT_DECODE_TILES, 3), (q.QMOE_OPT_DECODE_TILES, 8), (q.QMOE_OPT_DECODE_TILES, -1)]:
             assert q.lib.qmoe_set_option(h, opt, val) == q.QMOE_INVALID_ARGUMENT
         for opt, val in [(q.QMOE_OPT_WAIT_LIMIT_NS, 10**6), (q.QMOE_OPT_WAIT_LIMIT_NS, 2 * 10**9),
-                         (q.QMOE_OPT_TEST_WITHHOLD, 1), (q.QMOE_OPT_TEST_WITHHOLD, 0)]:
+                         (q.QMOE_OPT_TEST_WITHHOLD, 1), (q.QMOE_OPT_TEST_WITHHOLD, 0),
+                         (q.QMOE_OPT_DECODE_TILES, 4), (q.QMOE_OPT_DECODE_TILES, 0)]:
             assert q.lib.qmoe_set_option(h, opt, val) == q.QMOE_OK
     finally:
         q.qmoe_destroy(h)
@@ -253,7 +259,7 @@ def test_quantize_entry_rejects_bad_dtype_alignment_and_null(q):
 
 
 @pytest.mark.parametrize("kw,T,path", [
-    (dict(), 8, 1), (dict(), 65, 2), (dict(), 4096, 2),
+    (dict(), 8, 1), (dict(), 40, 2), (dict(), 65, 2), (dict(), 4096, 2),
     (dict(compute_mode=1), 8, 4), (dict(compute_mode=1), 300, 4),
     (dict(compute_mode=1, apply_router_weight_on_input=1), 8, 4),
     (dict(apply_router_weight_on_input=1), 8, 1),

@@ -73,6 +73,15 @@ CASES = {
                                act=gen.ACT_SILU),
     "k128_int8_percol_relu": dict(H=256, I=384, bits=8, block_size=0, fusion=0, act=gen.ACT_RELU),
     "k128_t32_tile32": dict(H=256, I=384, T=96, E=8, k=2),
+    # long K ranges: staged rows near the shared-memory target (fewer token
+    # tiles per pass on the streaming path), several tiles and passes, and the
+    # zero-point fold's per-column and per-chunk sums over thousands of k
+    "long_k_int4_bs128": dict(T=60, E=4, k=2, H=2048, I=1152, block_size=128),
+    "long_k_int4_bs32_f32scales": dict(T=60, E=4, k=2, H=2048, I=384, block_size=32,
+                                       scale_dtype=gen.DT_F32, has_fc1_bias=True),
+    "long_k_int8_percol": dict(T=28, E=4, k=2, H=4096, I=256, bits=8, block_size=0),
+    "long_k_one_tile_fold_percol": dict(T=4, E=2, k=1, H=5120, I=256, block_size=0),
+    "long_k_one_tile_fold_bs64": dict(T=4, E=2, k=1, H=5120, I=256, block_size=64, has_fc2_bias=True),
     # more than 128 rows per expert: 256-wide token tiles on the tensor-core path
     "wide_tile_int4_bs32_bias": dict(T=300, E=2, k=1, H=256, I=384, block_size=32, fusion=1, alpha=1.702,
                                      beta=1.0, limit=7.0, has_fc1_bias=True, has_fc2_bias=True),

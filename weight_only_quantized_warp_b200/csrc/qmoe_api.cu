@@ -61,6 +61,7 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
                                      : decode_smem_bytes(K, bits, bs, splits, nt);
         };
         p.nt = per_expert <= 8 ? 1 : (per_expert <= 16 ? 2 : 4);
+        if (h.decode_tiles > 0) p.nt = h.decode_tiles;
         // FC1 runs unsplit; keep its staged rows small enough for at least two CTAs per SM
         while (p.nt > 1 && smem(H, 1, p.nt) > kDecodeSmemTarget) p.nt /= 2;
         // FC2 split-K: every CTA (one 128-row block of one touched expert and
@@ -451,6 +452,12 @@ qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t value) {
     if (option == QMOE_OPT_PDL) {
         if (value != 0 && value != 1) return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_PDL must be 0 or 1");
         h->pdl = int(value);
+        return QMOE_OK;
+    }
+    if (option == QMOE_OPT_DECODE_TILES) {
+        if (value != 0 && value != 1 && value != 2 && value != 4)
+            return fail(h, QMOE_INVALID_ARGUMENT, "QMOE_OPT_DECODE_TILES must be 0, 1, 2 or 4");
+        h->decode_tiles = int(value);
         return QMOE_OK;
     }
     if (option == QMOE_OPT_TEST_WITHHOLD) {

@@ -115,6 +115,7 @@ struct qmoe_handle {
     float* b2 = nullptr;  // [E, H] fp32, nullptr when no fc2 bias
     int device = -1;
     int path_override = -1;  // QMOE_OPT_PATH; -1 = choose by shape
+    int decode_tiles = 0;    // QMOE_OPT_DECODE_TILES; 0 = choose by shape
     float* score_bias = nullptr;  // e_score_correction_bias [E] fp32, or nullptr
     uint64_t wait_limit_ns = 2000000000ull;  // QMOE_OPT_WAIT_LIMIT_NS
     int withhold = 0;        // QMOE_OPT_TEST_WITHHOLD
@@ -205,8 +206,11 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t st);
 // prepare_ffn_decode() raises the kernels' limit on the current device.
 constexpr size_t kDecodeSmemLimit = 200 * 1024;
 constexpr int64_t kDecodeSmemTarget = 112 * 1024;  // at least two CTAs per SM (three fit below 75 KB)
-// Rows per expert up to which the weight-streaming kernels are chosen.
-constexpr int64_t kDecodeRowsPerExpert = 16;
+// Rows per expert up to which the weight-streaming kernels are chosen (one
+// 8-token tile per pass; above it the tensor-core GEMM decodes each weight
+// once per token tile of up to 256 rows, measured faster from 16 rows per
+// expert on).
+constexpr int64_t kDecodeRowsPerExpert = 8;
 int64_t decode_smem_bytes(int64_t K, int bits, int block_size, int splits, int nt);
 cudaError_t prepare_ffn_decode();
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);

@@ -42,7 +42,7 @@ EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forwa
            "qmoe_set_option", "qmoe_forward_noalloc", "qmoe_noalloc_scratch_bytes",
            "qmoe_noalloc_read_device_status", "qmoe_set_score_correction_bias",
            "qmoe_quantize_act_i8")
-QMOE_OPT_PATH, QMOE_OPT_WAIT_LIMIT_NS, QMOE_OPT_TEST_WITHHOLD, QMOE_OPT_PDL = 1, 2, 3, 4
+QMOE_OPT_PATH, QMOE_OPT_WAIT_LIMIT_NS, QMOE_OPT_TEST_WITHHOLD, QMOE_OPT_PDL, QMOE_OPT_DECODE_TILES = 1, 2, 3, 4, 5
 
 
 class qmoe_config(ctypes.Structure):
