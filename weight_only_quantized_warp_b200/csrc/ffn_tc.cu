@@ -80,6 +80,10 @@ template <int BITS, bool PERCOL, int BNMAX, int STAGES, bool FP4>
 __global__ void __launch_bounds__(kTcThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap bmap, const TcArgs a) {
     using C = TcCfg<BITS, PERCOL, BNMAX, STAGES>;
+    // stages a role tests at once: within one lap of the ring (a dequantise
+    // group's own stages are every other one)
+    constexpr int kLook = STAGES - 1 < 4 ? STAGES - 1 : 4;
+    constexpr int kLookDeq = (STAGES - 1) / 2 + 1 < 4 ? (STAGES - 1) / 2 + 1 : 4;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -157,6 +161,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int st = 0;
         uint32_t ph = 0;
         bool ok = true;
+        int ready = 0;  // free stages found ahead by the last batched test
         const int ngr = int(a.K / kgroup_of(BITS));
         const int bs_log2 = PERCOL ? 0 : __ffs(a.block_size) - 1;
         for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
@@ -166,7 +171,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int y0 = int(it.seg0) + it.tt * a.bn;
             const int64_t blk = int64_t(it.e) * nrb + it.rb;
             for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
-                if (!warp_wait(smem_u32(&empty[st]), ph ^ 1u, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
+                if (ready == 0) {
+                    ready = ready_run<kLook>(empty, nullptr, st, ph ^ 1u, 1, STAGES);
+                    if (ready == 0) {
+                        if (!warp_wait(smem_u32(&empty[st]), ph ^ 1u, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
+                        ready = 1;
+                    }
+                }
+                --ready;
                 uint8_t* sb = smem + st * C::kStage;
                 const uint32_t fb = smem_u32(&full[st]);
                 mbar_expect_tx_e(fb, bytes, e);
@@ -194,6 +206,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int st = 0, acc = 0;
             uint32_t ph = 0, aph = 0;
             bool ok = true;
+            int ready = 0;  // decoded stages found ahead by the last batched test
             for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
                 const Item it = item_at(i, prefix, a, nrb, nks);
                 const int n = ((it.rows + 15) / 16) * 16;
@@ -202,8 +215,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
                 const uint32_t d = tmem + uint32_t(acc * BNMAX);
                 for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
-                    if (!warp_wait(smem_u32(&deq[st]), ph, abort_flag, a.status, a.timeout_ns) ||
-                        !warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
+                    // a stage is ready when decoded (A) and landed (B)
+                    if (ready == 0) {
+                        ready = ready_run<kLook>(deq, full, st, ph, 1, STAGES);
+                        if (ready == 0) {
+                            if (!warp_wait(smem_u32(&deq[st]), ph, abort_flag, a.status, a.timeout_ns) ||
+                                !warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
+                            ready = 1;
+                        }
+                    }
+                    --ready;
                     tc_fence_after();
                     const uint32_t at = tmem + uint32_t(C::kACol0 + st * kAStageCols);
                     const uint64_t bd = desc_sw128(smem_u32(smem + st * C::kStage));
@@ -227,7 +248,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // inside the lane quarter w%4 it may access) of the stages of parity
         // w / 8: two groups of eight warps decode alternate stages
         const int tile = 2 * (warp & 3) + ((warp >> 2) & 1), grp = warp >> 3;
-        int seen = 0;  // stages seen by this warp, both parities
         const int r0 = lane >> 2, c = lane & 3;
         const uint32_t lane_addr = uint32_t(16 * tile) << 16;
         int st = 0;
@@ -237,18 +257,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // scale block (within the stage) of a k offset: blocks of 64 k or more
         // cover the whole stage
         const int bs_shift = a.block_size >= kBK ? 30 : __ffs(a.block_size) - 1;
-        for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+        const bool stage_scale = a.block_size >= kBK;
+        int ready = 0;  // this group's landed stages found ahead by the last batched test
+        // The decode of a stage depends on nothing but its buffers, so the
+        // group walks its own stages (every other one of the CTA's sequence)
+        // directly: the stage count of the CTA's items, then a flat loop.
+        int nstages = 0;
+        for (int i = blockIdx.x; i < total; i += gridDim.x) {
             const Item it = item_at(i, prefix, a, nrb, nks);
-            for (int ks = it.ks_lo; ks < it.ks_hi; ++ks) {
-                if ((seen++ & 1) != grp) {  // the other group's stage
-                    if (++st == STAGES) { st = 0; ph ^= 1u; }
-                    continue;
+            nstages += it.ks_hi - it.ks_lo;
+        }
+        if (grp == 1) st = 1;
+        for (int n = grp; ok && n < nstages; n += 2) {
+            {
+                if (ready == 0) {
+                    ready = ready_run<kLookDeq>(full, nullptr, st, ph, 2, STAGES);
+                    if (ready == 0) {
+                        if (!warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
+                        ready = 1;
+                    }
                 }
-                if (!warp_wait(smem_u32(&full[st]), ph, abort_flag, a.status, a.timeout_ns)) { ok = false; break; }
+                --ready;
                 const uint8_t* sb = smem + st * C::kStage;
                 const uint8_t* pk = sb + C::kB;
                 const uint8_t* sc = pk + C::kPacked;
                 const uint32_t at = tmem + lane_addr + uint32_t(C::kACol0 + st * kAStageCols);
+                // bf16 scale of rows r0 / r0 + 8 (in both halves) of the block
+                // holding stage-relative k offset kl
+                auto scale_pair = [&](int kl, uint32_t& sa2, uint32_t& sb2) {
+                    const int si = ((kl >> bs_shift) * kTilesPerBlock + tile) * 16 + 2 * r0;
+                    if (a.scale_bf16) {
+                        const uint32_t raw = *reinterpret_cast<const uint32_t*>(sc + si * 2);
+                        sa2 = __byte_perm(raw, 0u, 0x1010);
+                        sb2 = __byte_perm(raw, 0u, 0x3232);
+                    } else {
+                        const float2 f = *reinterpret_cast<const float2*>(sc + si * 4);
+                        sa2 = bf2_bcast(f.x);
+                        sb2 = bf2_bcast(f.y);
+                    }
+                };
+                // blocks of 64 k or more: one scale pair for the whole stage
+                uint32_t sa_st = 0, sb_st = 0;
+                if (!PERCOL && stage_scale) scale_pair(0, sa_st, sb_st);
                 constexpr int GROUPS = kBK / kgroup_of(BITS);  // 1 (int4) or 2 (int8)
 #pragma unroll
                 for (int gg = 0; gg < GROUPS; ++gg) {
@@ -281,18 +331,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                         if (!PERCOL) {
                             // scale block of this k-step (k = 64*ks + 32*gg + 16j + 4c + ...)
-                            const int kl = 32 * gg * (BITS == 8) + 16 * j + 4 * c;
-                            const int si = ((kl >> bs_shift) * kTilesPerBlock + tile) * 16 + 2 * r0;
-                            uint32_t sa2, sb2;  // bf16 scale of row r0 / r0 + 8, in both halves
-                            if (a.scale_bf16) {
-                                const uint32_t raw = *reinterpret_cast<const uint32_t*>(sc + si * 2);
-                                sa2 = __byte_perm(raw, 0u, 0x1010);
-                                sb2 = __byte_perm(raw, 0u, 0x3232);
-                            } else {
-                                const float2 f = *reinterpret_cast<const float2*>(sc + si * 4);
-                                sa2 = bf2_bcast(f.x);
-                                sb2 = bf2_bcast(f.y);
-                            }
+                            uint32_t sa2 = sa_st, sb2 = sb_st;
+                            if (!stage_scale) scale_pair(32 * gg * (BITS == 8) + 16 * j + 4 * c, sa2, sb2);
                             A[0] = bf2_mul(A[0], sa2);
                             A[2] = bf2_mul(A[2], sa2);
                             A[1] = bf2_mul(A[1], sb2);
@@ -314,7 +354,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&deq[st]));
-                if (++st == STAGES) { st = 0; ph ^= 1u; }
+                st += 2;
+                if (st >= STAGES) {
+                    st -= STAGES;
+                    ph ^= 1u;
+                }
             }
         }
     } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + kEpiWarps) {

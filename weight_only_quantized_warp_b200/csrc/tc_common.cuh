@@ -102,6 +102,32 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Run of completed phases, by a whole warp without blocking: tests the ring
+// stages st, st + step, ... (up to L of them, the parity flipping where the
+// ring wraps) on bars0 (and bars1 when given) and returns how many leading
+// ones have completed. The tests are independent, so their shared-memory
+// round trips overlap; a role that finds several stages ready consumes them
+// without testing again. Valid while the stages tested lie within one lap of
+// the ring: (L - 1) * step < stages. Lane 0's view is taken by every lane.
+template <int L>
+__device__ __forceinline__ int ready_run(const uint64_t* bars0, const uint64_t* bars1, int st, uint32_t parity,
+                                         int step, int stages) {
+    uint32_t mask = 0;
+#pragma unroll
+    for (int j = 0; j < L; ++j) {
+        bool ok = mbar_test(smem_u32(&bars0[st]), parity);
+        if (bars1 != nullptr) ok = mbar_test(smem_u32(&bars1[st]), parity) & ok;
+        mask |= uint32_t(ok) << j;
+        st += step;
+        if (st >= stages) {
+            st -= stages;
+            parity ^= 1u;
+        }
+    }
+    mask = __shfl_sync(0xffffffffu, mask, 0);
+    return __ffs(~mask) - 1;
+}
+
 // Wait by a whole warp: every lane polls, and the warp continues only if all
 // lanes saw the phase complete (a timeout in any lane stops the whole warp).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
