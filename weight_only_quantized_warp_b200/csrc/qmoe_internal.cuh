@@ -215,16 +215,6 @@ int64_t decode_smem_bytes(int64_t K, int bits, int block_size, int splits, int n
 cudaError_t prepare_ffn_decode();
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
 
-// Weight streaming through a shared-memory slab ring (persistent, one CTA per
-// SM): integer codes with per-column scales or block scales of at least one
-// k-group, bf16 activations, one or two 8-token tiles per pass.
-// stream_smem_bytes also reports the ring slabs that fit (stages_out).
-constexpr size_t kStreamSmemLimit = 224 * 1024;
-bool stream_supports(int bits, int block_size, int fp4, int nt);
-int64_t stream_smem_bytes(int64_t K, int bits, int block_size, int splits, int nt, int* stages_out);
-cudaError_t prepare_ffn_stream();
-cudaError_t launch_ffn_stream(const FfnArgs& a, int32_t* status, cudaStream_t st);
-
 // Tensor-core (tcgen05) expert FFN layer over the segments; bn = token tile.
 // prepare_ffn_tc() raises the kernels' shared-memory limit on the current
 // device. launch_gather_rows copies the routed rows of x into segment order.
