@@ -120,8 +120,9 @@ def launch_names(path, launches, weights_on_input):
     the row gather (tensor-core paths, or router weights on the input), the
     int8 tier's two rounding launches, FC1, FC2 and the combine."""
     from weight_only_quantized_warp_b200 import qmoe
-    gather = path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE) or weights_on_input
-    ffn = ["quantize_x", "fc1", "quantize_h", "fc2"] if path == qmoe.PATH_INT8 else ["fc1", "fc2"]
+    gather = path in (qmoe.PATH_TC, qmoe.PATH_TC_DECODE, qmoe.PATH_INT8_TC) or weights_on_input
+    int8_tier = path in (qmoe.PATH_INT8, qmoe.PATH_INT8_TC)
+    ffn = ["quantize_x", "fc1", "quantize_h", "fc2"] if int8_tier else ["fc1", "fc2"]
     routing = launches - int(gather) - len(ffn) - 1
     if routing not in (1, 2):
         raise ValueError(f"{launches} launches do not fit path {path}")
@@ -169,6 +170,9 @@ def roofline_of(cfg, alg, fc1_ms, peaks, peaks_kind, kname, traffic):
     binds."""
     hbm_peak = float(peaks["hbm_gbs"])
     tc_peak, tc_kind = tc_peak_of(peaks)
+    if kname.startswith("ffn_tc_i8_kernel"):
+        # integer MMAs: the bf16 figure times the nominal int8 / bf16 ratio (4.5 / 2.25)
+        tc_peak, tc_kind = 2.0 * tc_peak, tc_kind + " x 2 for int8"
     t_hbm = alg["fc1_bytes"] / (hbm_peak * 1e9)
     t_tc = alg["fc1_flops"] / (tc_peak * 1e12)
     if t_hbm >= t_tc:
@@ -262,7 +266,7 @@ def fc1_kernel_name(qmoe, path, tile):
     if path == qmoe.PATH_TC:
         return "ffn_tc_wide_kernel" if tile > 128 else "ffn_tc_kernel"
     return {qmoe.PATH_TC_DECODE: "ffn_tc_decode_kernel", qmoe.PATH_SIMT: "ffn_simt_kernel",
-            qmoe.PATH_INT8: "ffn_i8_kernel"}.get(path, "ffn_decode_kernel")
+            qmoe.PATH_INT8: "ffn_i8_kernel", qmoe.PATH_INT8_TC: "ffn_tc_i8_kernel"}.get(path, "ffn_decode_kernel")
 
 
 # ---------------------------------------------------------------- reference arm

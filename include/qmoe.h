@@ -361,8 +361,11 @@ QMOE_API qmoe_status qmoe_quantize_act_i8(const void* x, int32_t dtype, int64_t 
  * tcgen05 streaming decode kernels (falls back to 1 for shapes they do not
  * cover: more than 32 rows per expert, K not a multiple of 128, or a K range
  * whose resident activations exceed 128 KB). fp32 activations always take
- * the fp32 path (0); compute_mode INT8_BLOCK always takes path 4 and ignores
- * this option. */
+ * the fp32 path (0). Under compute_mode INT8_BLOCK the option chooses within
+ * the tier: 1 (or 3) forces the streaming integer kernels (path 4), 2 the
+ * tcgen05 integer GEMM (path 5; falls back to 4 for fp32 activations or
+ * blocks of fewer than 32 codes); by default path 5 is taken for blocks of
+ * 128 or more codes beyond 32 rows per expert, path 4 otherwise. */
 enum { QMOE_OPT_PATH = 1 };
 
 /* QMOE_OPT_WAIT_LIMIT_NS: the limit, in nanoseconds, of every bounded
@@ -400,7 +403,9 @@ QMOE_API qmoe_status qmoe_set_option(qmoe_handle* h, int32_t option, int64_t val
 /* The forward path qmoe_forward takes for T tokens: 0 = fp32 SIMT path,
  * 1 = weight-streaming decode path (mma.sync), 2 = tcgen05 grouped GEMM,
  * 3 = tcgen05 streaming decode, 4 = int8 block tier (weight-streaming
- * integer mma.sync). -1 for a NULL handle. */
+ * integer mma.sync), 5 = int8 block tier on the tcgen05 integer GEMM
+ * (kind::i8, int32 accumulators in tensor memory folded per K block).
+ * -1 for a NULL handle. */
 QMOE_API int32_t qmoe_path_for(const qmoe_handle* h, int64_t T);
 
 /* Number of kernel launches qmoe_forward enqueues for T tokens: routing and
@@ -412,7 +417,8 @@ QMOE_API int32_t qmoe_launches_for(const qmoe_handle* h, int64_t T);
 /* Token-tile width (the MMA N dimension, rows of one expert per work item)
  * of the tensor-core paths for T tokens: 16..128 run the 128-wide tcgen05
  * kernel with the decoded weights in TMEM, 256 the wide kernel with them in
- * shared memory; 16 or 32 on path 3. 0 on paths 0 and 1, -1 for a NULL
+ * shared memory; 16 or 32 on path 3; 16..64 on path 5. 0 on paths 0, 1 and
+ * 4, -1 for a NULL
  * handle or T < 0. No counterpart on the pages: it only reports the plan. */
 QMOE_API int32_t qmoe_token_tile_for(const qmoe_handle* h, int64_t T);
 

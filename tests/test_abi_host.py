@@ -210,26 +210,43 @@ def test_status_strings(q):
 
 
 def test_int8_tier_plan(q):
-    # compute_mode INT8_BLOCK: path 4 for every T, the two rounding launches
-    # added, and the code buffers in the workspace
+    # compute_mode INT8_BLOCK: the streaming kernel (path 4), and with K
+    # blocks of 128 or more beyond 32 rows per expert the integer tensor-core
+    # GEMM (path 5, with the row gather and a token tile of at most 64); the
+    # two rounding launches added, and the code buffers in the workspace
     h = q.qmoe_create(_cfg(q, compute_mode=q.COMPUTE_INT8_BLOCK))
+    h128 = q.qmoe_create(_cfg(q, compute_mode=q.COMPUTE_INT8_BLOCK, block_size=128))
     hf = q.qmoe_create(_cfg(q))
     ha = q.qmoe_create(_cfg(q, compute_mode=q.COMPUTE_INT8_BLOCK, apply_router_weight_on_input=1))
     try:
-        for T in (1, 8, 64, 65, 4096):
+        for T in (1, 8, 64, 65, 4096):  # 64-code blocks: the streaming kernel
             assert q.qmoe_path_for(h, T) == q.PATH_INT8
             assert q.qmoe_token_tile_for(h, T) == 0
+        for T in (8, 128):
+            assert q.qmoe_path_for(h128, T) == q.PATH_INT8
+        for T, tile in ((129, 64), (4096, 64)):
+            assert q.qmoe_path_for(h128, T) == q.PATH_INT8_TC
+            assert q.qmoe_token_tile_for(h128, T) == tile
         assert q.qmoe_launches_for(h, 8) == 6     # route+permute, quantize x, FC1, quantize h, FC2, combine
         assert q.qmoe_launches_for(h, 65) == 7    # routing and permutation apart
+        assert q.qmoe_launches_for(h128, 129) == 8  # plus the row gather
         assert q.qmoe_launches_for(ha, 8) == 7    # plus the weighted row gather
         # codes and scales of x [T, H] and h [T*k, I] on top of the float plan
         T, H, I, k, bs = 8, 256, 512, 2, 64
         extra = T * H + T * (H // bs) * 4 + T * k * I + T * k * (I // bs) * 4
         assert q.qmoe_workspace_size(h, T) >= q.qmoe_workspace_size(hf, T) + extra
-        q.qmoe_set_option(h, q.QMOE_OPT_PATH, 2)  # ignored on the int8 tier
-        assert q.qmoe_path_for(h, 8) == q.PATH_INT8
+        q.qmoe_set_option(h, q.QMOE_OPT_PATH, 2)  # the tensor-core GEMM at any T
+        assert q.qmoe_path_for(h, 8) == q.PATH_INT8_TC
+        q.qmoe_set_option(h, q.QMOE_OPT_PATH, 1)  # the streaming kernel at any T
+        assert q.qmoe_path_for(h, 4096) == q.PATH_INT8
+        for v in (1, 3):  # 1 and 3 both keep the tier on the streaming kernel
+            q.qmoe_set_option(h128, q.QMOE_OPT_PATH, v)
+            assert q.qmoe_path_for(h128, 4096) == q.PATH_INT8
+        q.qmoe_set_option(h128, q.QMOE_OPT_PATH, -1)
+        assert q.qmoe_path_for(h128, 4096) == q.PATH_INT8_TC
     finally:
         q.qmoe_destroy(h)
+        q.qmoe_destroy(h128)
         q.qmoe_destroy(hf)
         q.qmoe_destroy(ha)
     hs = q.qmoe_create(_cfg(q, compute_mode=q.COMPUTE_INT8_BLOCK, act_dtype=q.DTYPE_F32,
@@ -260,7 +277,7 @@ def test_quantize_entry_rejects_bad_dtype_alignment_and_null(q):
 
 @pytest.mark.parametrize("kw,T,path", [
     (dict(), 8, 1), (dict(), 40, 2), (dict(), 65, 2), (dict(), 4096, 2),
-    (dict(compute_mode=1), 8, 4), (dict(compute_mode=1), 300, 4),
+    (dict(compute_mode=1), 8, 4), (dict(compute_mode=1), 300, 4), (dict(compute_mode=1, block_size=128), 300, 5),
     (dict(compute_mode=1, apply_router_weight_on_input=1), 8, 4),
     (dict(apply_router_weight_on_input=1), 8, 1),
     (dict(act_dtype=0, scale_dtype=0), 8, 0), (dict(act_dtype=0, scale_dtype=0), 100, 0),
@@ -276,8 +293,8 @@ def test_bench_launch_names_match_the_plan(q, kw, T, path):
         assert len(names) == n
         assert names[-1] == "combine" and names.index("fc1") < names.index("fc2")
         assert ("route_permute" in names) == (T <= 64)
-        assert ("quantize_x" in names) == (path == q.PATH_INT8)
-        assert ("gather" in names) == (path in (q.PATH_TC, q.PATH_TC_DECODE) or
+        assert ("quantize_x" in names) == (path in (q.PATH_INT8, q.PATH_INT8_TC))
+        assert ("gather" in names) == (path in (q.PATH_TC, q.PATH_TC_DECODE, q.PATH_INT8_TC) or
                                        bool(kw.get("apply_router_weight_on_input")))
     finally:
         q.qmoe_destroy(h)

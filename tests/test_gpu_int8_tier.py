@@ -1,4 +1,5 @@
-"""GPU parity of the int8 block compute tier (compute_mode INT8_BLOCK, path 4)
+"""GPU parity of the int8 block compute tier (compute_mode INT8_BLOCK: the
+streaming integer kernel, path 4, and the integer tensor-core GEMM, path 5)
 against the oracle.
 
 The activation rounding is compared bit for bit: codes and fp32 scales of
@@ -28,8 +29,21 @@ from gpu_helpers import TOL_BF16, TOL_F32, check_routing, check_sampled, max_rel
 
 pytestmark = pytest.mark.gpu
 
-PATH_INT8 = 4
+PATH_INT8, PATH_INT8_TC = 4, 5
 TOL_Y = 1e-2
+
+
+def _expected_path(cfg, forced=None):
+    """The tier's kernel: the tensor-core GEMM for bf16 activations (blocks
+    of at least 32 codes) when forced, and by shape with blocks of 128 or more
+    beyond 32 rows per expert; the streaming kernel otherwise."""
+    tc_ok = cfg.act_dtype == gen.DT_BF16 and cfg.block_size >= 32
+    per_expert = -(-max(cfg.T * cfg.k, 1) // cfg.E)
+    if forced == 1:
+        return PATH_INT8
+    if forced == 2:
+        return PATH_INT8_TC if tc_ok else PATH_INT8
+    return PATH_INT8_TC if tc_ok and per_expert > 32 and cfg.block_size >= 128 else PATH_INT8
 
 
 def _quant_rows(rng, rows, K, bs, bf16):
@@ -88,9 +102,9 @@ def _cfg(**kw):
     return gen.MoEConfig(**base)
 
 
-def _check(inp, g):
+def _check(inp, g, forced=None):
     c = inp.cfg
-    assert g.path == PATH_INT8
+    assert g.path == _expected_path(c, forced)
     check_routing(inp, g)
     ref = oracle.forward(inp, want_h=True)
     err = max_rel(g.y, ref["y"])
@@ -136,11 +150,14 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("path", [None, 1, 2], ids=["auto", "stream", "tc"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_int8_tier_parity_small(cuda_device, name):
+def test_int8_tier_parity_small(cuda_device, name, path):
     cfg = _cfg(**CASES[name])
+    if path is not None and _expected_path(cfg, path) == _expected_path(cfg):
+        pytest.skip("the forced kernel is the one chosen by shape")
     inp = gen.make_inputs(cfg, seed=300 + list(CASES).index(name), bias_std=0.1)
-    _check(inp, run_gpu(inp))
+    _check(inp, run_gpu(inp, path=path), forced=path)
 
 
 def test_int8_tier_zero_rows_and_blocks(cuda_device):
@@ -224,21 +241,21 @@ def test_int8_tier_full_size_decode(cuda_device, T):
     cfg, seed, kw = gen.workload("mixtral_decode_i8", T=T)
     inp = gen.make_inputs(cfg, seed, **kw)
     g = run_gpu(inp)
-    assert g.path == PATH_INT8
+    assert g.path == _expected_path(cfg)
     tokens = np.arange(T) if T <= 8 else np.sort(np.random.default_rng(T).choice(T, 8, replace=False))
     err = check_sampled(inp, g, tokens)
     assert err <= TOL_Y
 
 
-@pytest.mark.parametrize("bits,T", [(8, 16), (4, 128)])
+@pytest.mark.parametrize("bits,T", [(8, 16), (4, 128), (8, 128), (4, 1024), (8, 1024)])
 def test_int8_tier_full_size_sweep_shapes(cuda_device, bits, T):
     # the sweep's H=4096, I=14336 shapes on the int8 tier: int8 codes with
-    # 128-code blocks, and int4 with 64-code blocks at 32 rows per expert
-    # (two passes of the two-tile kernel)
+    # 128-code blocks and int4 with 64-code blocks, on the streaming kernel
+    # (16 tokens) and the integer tensor-core GEMM (32 and 256 rows per expert)
     cfg, seed, kw = gen.sweep(bits, T)
     cfg.compute_mode = gen.COMPUTE_INT8_BLOCK
     inp = gen.make_inputs(cfg, seed, **kw)
     g = run_gpu(inp)
-    assert g.path == PATH_INT8
-    tokens = np.sort(np.random.default_rng(seed).choice(T, 4, replace=False))
-    assert check_sampled(inp, g, tokens) <= TOL_Y
+    assert g.path == _expected_path(cfg)
+    tokens = np.sort(np.random.default_rng(seed).choice(T, 4 if T < 1024 else 8, replace=False))
+    assert check_sampled(inp, g, tokens, name=f"int8_tier_sweep_int{bits}_T{T}/path{g.path}") <= TOL_Y

@@ -74,7 +74,13 @@ __device__ __forceinline__ void mma_u8s8_zero(int (&d)[4], const uint32_t (&a)[4
 // is bs / 4 consecutive lanes. Pass 1 finds the block's absmax, pass 2
 // writes the codes (one 32-bit word per lane and step) and lane 0 of the
 // block its scale.
-template <bool IN_BF16, bool PERM>
+// LAYOUT: 0 natural order; 1 the middle two codes of every run of 4 swapped
+// (k + {0, 2, 1, 3}: the nibble order of 4-bit weight words, for
+// ffn_i8_kernel); 2 and 3 the tensor-core order of ffn_tc_i8_kernel: within
+// every 32-code chunk, the run of codes k = 4 r .. 4 r + 3 goes to run
+// 2 (r % 4) + r / 4, with the middle two codes swapped (2, 4-bit weights) or
+// not (3, 8-bit weights).
+template <bool IN_BF16, int LAYOUT>
 __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(const void* x, int64_t rows, int64_t K, int bs,
                                                                int8_t* q, float* s) {
     const int lane = threadIdx.x & 31;
@@ -127,9 +133,15 @@ __global__ void __launch_bounds__(256) quantize_rows_i8_kernel(const void* x, in
             c = max(-127, min(127, c));
             b[i] = uint32_t(c) & 0xFFu;
         }
-        const uint32_t word = PERM ? (b[0] | (b[2] << 8) | (b[1] << 16) | (b[3] << 24))
+        constexpr bool SWAP = LAYOUT == 1 || LAYOUT == 2;
+        const uint32_t word = SWAP ? (b[0] | (b[2] << 8) | (b[1] << 16) | (b[3] << 24))
                                    : (b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24));
-        *reinterpret_cast<uint32_t*>(q + row * K + k) = word;
+        int64_t kout = k;
+        if (LAYOUT >= 2) {
+            const int rq = lane & 7;  // run of 4 inside the lane's 32-code chunk
+            kout = k - 4 * rq + 4 * (2 * (rq & 3) + (rq >> 2));
+        }
+        *reinterpret_cast<uint32_t*>(q + row * K + kout) = word;
     }
     const int64_t kl = k0 + lane * 4;
     if ((lane & (G - 1)) == 0 && kl < K) s[row * (K / bs) + kl / bs] = sc;
@@ -438,23 +450,27 @@ cudaError_t launch_ffn_i8(const FfnArgs& a, cudaStream_t st) {
     return launch_sf<8, 8>(a, grid, smem, st);
 }
 
-cudaError_t launch_quantize_i8(const void* x, int act_bf16, int64_t rows, int64_t K, int bs, int perm, int8_t* q,
+template <bool IN_BF16>
+void launch_quantize_layout(int layout, unsigned grid, const void* x, int64_t rows, int64_t K, int bs, int8_t* q,
+                            float* s, cudaStream_t st) {
+    switch (layout) {
+        case 1: quantize_rows_i8_kernel<IN_BF16, 1><<<grid, 256, 0, st>>>(x, rows, K, bs, q, s); break;
+        case 2: quantize_rows_i8_kernel<IN_BF16, 2><<<grid, 256, 0, st>>>(x, rows, K, bs, q, s); break;
+        case 3: quantize_rows_i8_kernel<IN_BF16, 3><<<grid, 256, 0, st>>>(x, rows, K, bs, q, s); break;
+        default: quantize_rows_i8_kernel<IN_BF16, 0><<<grid, 256, 0, st>>>(x, rows, K, bs, q, s); break;
+    }
+}
+
+cudaError_t launch_quantize_i8(const void* x, int act_bf16, int64_t rows, int64_t K, int bs, int layout, int8_t* q,
                                float* s, cudaStream_t st) {
     if (rows <= 0) return cudaSuccess;
     const int64_t span = bs > 128 ? bs : 128;
     const int64_t warps = rows * ((K + span - 1) / span);
     const unsigned grid = unsigned((warps + 7) / 8);
-    if (act_bf16) {
-        if (perm)
-            quantize_rows_i8_kernel<true, true><<<grid, 256, 0, st>>>(x, rows, K, bs, q, s);
-        else
-            quantize_rows_i8_kernel<true, false><<<grid, 256, 0, st>>>(x, rows, K, bs, q, s);
-    } else {
-        if (perm)
-            quantize_rows_i8_kernel<false, true><<<grid, 256, 0, st>>>(x, rows, K, bs, q, s);
-        else
-            quantize_rows_i8_kernel<false, false><<<grid, 256, 0, st>>>(x, rows, K, bs, q, s);
-    }
+    if (act_bf16)
+        launch_quantize_layout<true>(layout, grid, x, rows, K, bs, q, s, st);
+    else
+        launch_quantize_layout<false>(layout, grid, x, rows, K, bs, q, s, st);
     return cudaGetLastError();
 }
 

@@ -40,8 +40,17 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
                                touched * (padded_rows(H) / kBlockRows) * tcd_s2 < 4 * kSms))
         ++tcd_s2;
     const bool tcd_ok = per_expert <= 32 && tc_decode_fits(H, 1, tcd_bn, bs) && tc_decode_fits(I, tcd_s2, tcd_bn, bs);
-    if (c.compute_mode == QMOE_COMPUTE_INT8_BLOCK)
-        p.path = kPathI8;
+    if (c.compute_mode == QMOE_COMPUTE_INT8_BLOCK) {
+        // the int8 tier: the integer tcgen05 GEMM for bf16 activations where
+        // it measured faster than the streaming integer mma.sync kernel -- K
+        // blocks of 128 or more (one partial fold per 128 k or fewer) and more
+        // than 32 rows per expert; QMOE_OPT_PATH 2 forces it, 1 and 3 the
+        // streaming kernel
+        const bool tc_ok = bf16 && tc_i8_supports(bits, bs, H, I);
+        const bool want_tc = h.path_override == kPathTc ||
+                             (h.path_override == -1 && per_expert > 32 && bs >= 128);
+        p.path = tc_ok && want_tc ? kPathI8Tc : kPathI8;
+    }
     else if (!bf16)
         p.path = kPathSimt;
     else if (h.path_override == kPathDecode || h.path_override == kPathTc)
@@ -90,26 +99,32 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
         p.fc2_splits = int(best);
         p.ok = smem(H, 1, p.nt) <= int64_t(kDecodeSmemLimit) &&
                smem(I, p.fc2_splits, p.nt) <= int64_t(kDecodeSmemLimit);
-    } else if (p.path == kPathTc) {
+    } else if (p.path == kPathTc || p.path == kPathI8Tc) {
         // token tile: the power of two covering the average segment with a
         // third to spare, so that most experts take one tile (the weights of
-        // an expert are decoded once per tile)
+        // an expert are decoded once per tile); at most 64 on the int8 tier,
+        // whose fold warps hold a tile's fp32 sums in registers
+        const int bnmax = p.path == kPathTc ? 256 : 64;
         int bn = 16;
-        while (bn < 256 && bn < ceil_div(4 * per_expert, 3)) bn *= 2;
+        while (bn < bnmax && bn < ceil_div(4 * per_expert, 3)) bn *= 2;
         p.bn = bn;
         // FC2 work items: touched experts x 128-row blocks x token tiles;
-        // split K until every SM has about two items
+        // split K until every SM has about two items. The int8 tier's
+        // 128-k stages split on K-block boundaries only for blocks up to 128.
         const int64_t items = touched * (padded_rows(H) / kBlockRows) * std::max<int64_t>(1, ceil_div(per_expert, bn));
+        const int64_t kstage = p.path == kPathTc ? 64 : 128;
         int64_t s = 1;
-        while (items * s < 2 * kSms && s < 8 && s * 2 <= I / 64) s *= 2;
+        if (p.path == kPathTc || bs <= 128)
+            while (items * s < 2 * kSms && s < 8 && s * 2 <= I / kstage) s *= 2;
         p.fc2_splits = int(s);
     }
     p.fused_route = T <= kFusedRouteTokens;
     // the row gather runs on the tensor-core paths, and on every path when
     // the router weights scale the expert inputs
-    p.gather = p.path == kPathTc || p.path == kPathTcDecode || c.apply_router_weight_on_input;
+    p.gather = p.path == kPathTc || p.path == kPathTcDecode || p.path == kPathI8Tc || c.apply_router_weight_on_input;
     // the int8 tier adds the rounding of FC1's input rows and of h
-    p.launches = (p.fused_route ? 1 : 2) + (p.gather ? 1 : 0) + 3 + (p.path == kPathI8 ? 2 : 0);
+    const bool i8 = p.path == kPathI8 || p.path == kPathI8Tc;
+    p.launches = (p.fused_route ? 1 : 2) + (p.gather ? 1 : 0) + 3 + (i8 ? 2 : 0);
     const size_t R = size_t(p.R);
     const size_t act = bf16 ? 2 : 4;
     size_t off = 0;
@@ -123,7 +138,7 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     p.off_xperm = off;
     off = align256(off + (p.gather ? R * size_t(H) * act : 0));
     p.off_o = off;       off = align256(off + size_t(p.fc2_splits) * R * size_t(H) * 4);
-    if (p.path == kPathI8) {
+    if (i8) {
         const size_t nsb1 = size_t(H / bs), nsb2 = size_t(I / bs);
         p.xq_rows = p.gather ? p.R : T;
         const size_t xr = size_t(p.xq_rows);
@@ -359,6 +374,7 @@ qmoe_status qmoe_set_weights(qmoe_handle* h, const void* fc1_w, const void* fc1_
     if (err == cudaSuccess) err = prepare_ffn_decode();
     if (err == cudaSuccess) err = prepare_ffn_tc();
     if (err == cudaSuccess) err = prepare_ffn_i8();
+    if (err == cudaSuccess) err = prepare_ffn_tc_i8();
     if (err != cudaSuccess) return cuda_fail(h, err, "prepare kernels");
 
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size, N1 = h->n1;
@@ -486,7 +502,7 @@ int32_t qmoe_launches_for(const qmoe_handle* h, int64_t T) {
 int32_t qmoe_token_tile_for(const qmoe_handle* h, int64_t T) {
     if (!h || T < 0) return -1;
     const Plan p = make_plan(*h, T);
-    return (p.path == kPathTc || p.path == kPathTcDecode) ? p.bn : 0;
+    return (p.path == kPathTc || p.path == kPathTcDecode || p.path == kPathI8Tc) ? p.bn : 0;
 }
 
 }  // extern "C"
@@ -613,9 +629,11 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
         f1.act = xp;
         f1.rowmap = nullptr;  // rows already in segment order
     }
-    if (p.path == kPathI8) {
-        // FC1's input rows (x by token, or the gathered rows) to int8 codes
-        const int perm = c.expert_weight_bits == 4;
+    if (p.path == kPathI8 || p.path == kPathI8Tc) {
+        // FC1's input rows (x by token, or the gathered rows) to int8 codes,
+        // in the order the chosen kernel reads them
+        const bool tc = p.path == kPathI8Tc;
+        const int perm = tc ? (c.expert_weight_bits == 4 ? 2 : 3) : (c.expert_weight_bits == 4 ? 1 : 0);
         int8_t* xq = (int8_t*)(ws + p.off_xq);
         float* xs = (float*)(ws + p.off_xs);
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
@@ -625,7 +643,8 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
         f1.aq = xq;
         f1.as = xs;
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        if ((err = launch_ffn_i8(f1, st)) != cudaSuccess) return cuda_fail(h, err, "fc1");
+        if ((err = tc ? launch_ffn_tc_i8(f1, p.bn, status, st) : launch_ffn_i8(f1, st)) != cudaSuccess)
+            return cuda_fail(h, err, "fc1");
         int8_t* hq = (int8_t*)(ws + p.off_hq);
         float* hs = (float*)(ws + p.off_hs);
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
@@ -634,7 +653,8 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
         f2.aq = hq;
         f2.as = hs;
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        if ((err = launch_ffn_i8(f2, st)) != cudaSuccess) return cuda_fail(h, err, "fc2");
+        if ((err = tc ? launch_ffn_tc_i8(f2, p.bn, status, st) : launch_ffn_i8(f2, st)) != cudaSuccess)
+            return cuda_fail(h, err, "fc2");
     } else {
         if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
         err = p.path == kPathSimt        ? launch_ffn_simt(f1, st)

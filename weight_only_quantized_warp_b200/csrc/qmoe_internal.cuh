@@ -80,7 +80,7 @@ __host__ __device__ constexpr int64_t padded_rows(int64_t n) {
 constexpr int kActGeluTanh = 5;
 
 // Hot-path selection.
-enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2, kPathTcDecode = 3, kPathI8 = 4 };
+enum Path : int { kPathSimt = 0, kPathDecode = 1, kPathTc = 2, kPathTcDecode = 3, kPathI8 = 4, kPathI8Tc = 5 };
 
 struct Plan {
     int path = kPathDecode;
@@ -215,6 +215,14 @@ int64_t decode_smem_bytes(int64_t K, int bits, int block_size, int splits, int n
 cudaError_t prepare_ffn_decode();
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
 
+// The int8 block tier on the tensor cores (tcgen05 kind::i8): activation
+// codes [R, K] in the tensor-core order of quantize layouts 2 / 3 (f.aq),
+// their block scales [R, K / block_size] (f.as), token tile bn <= 64.
+// tc_i8_supports: the shapes it takes (blocks of at least 32 codes).
+bool tc_i8_supports(int bits, int block_size, int64_t H, int64_t I);
+cudaError_t prepare_ffn_tc_i8();
+cudaError_t launch_ffn_tc_i8(const FfnArgs& f, int bn, int32_t* status, cudaStream_t st);
+
 // Tensor-core (tcgen05) expert FFN layer over the segments; bn = token tile.
 // prepare_ffn_tc() raises the kernels' shared-memory limit on the current
 // device. launch_gather_rows copies the routed rows of x into segment order.
@@ -238,9 +246,11 @@ cudaError_t launch_gather_rows_weighted(const void* x, const int32_t* perm, cons
                                         const float* topk_w, int k, void* xp, int64_t R, int64_t H, int act_bf16,
                                         cudaStream_t st);
 
-// Int8 block compute tier: per-block int8 rounding of activation rows (perm:
-// the 4-code order of 4-bit weights), and the expert FFN layer on the codes.
-cudaError_t launch_quantize_i8(const void* x, int act_bf16, int64_t rows, int64_t K, int bs, int perm, int8_t* q,
+// Int8 block compute tier: per-block int8 rounding of activation rows (layout
+// of the codes: 0 natural, 1 the 4-code order of 4-bit weights for the
+// streaming kernel, 2 / 3 the tensor-core order for 4- / 8-bit weights), and
+// the expert FFN layer on the codes.
+cudaError_t launch_quantize_i8(const void* x, int act_bf16, int64_t rows, int64_t K, int bs, int layout, int8_t* q,
                                float* s, cudaStream_t st);
 int64_t i8_smem_bytes(int64_t K, int bits, int block_size, int splits, int nt);
 cudaError_t prepare_ffn_i8();

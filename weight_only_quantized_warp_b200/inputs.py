@@ -297,6 +297,12 @@ WORKLOADS = {
 
 def workload(name: str, **kw):
     """Return ``(cfg, seed, gen_kwargs)`` for a named workload."""
+    if name.startswith("sweep_i8tier_int"):
+        # sweep_i8tier_int4_T1024: the sweep shape on the int8 block compute tier
+        bits = int(name[len("sweep_i8tier_int")])
+        cfg, seed, gkw = sweep(bits, int(name.split("_T")[1]))
+        cfg.compute_mode = COMPUTE_INT8_BLOCK
+        return cfg, seed, gkw
     if name.startswith("sweep_int"):
         # sweep_int4_T128
         bits = int(name[len("sweep_int")])

@@ -31,7 +31,7 @@ DTYPE_F32, DTYPE_BF16, DTYPE_E8M0 = 0, 1, 2
 WEIGHTS_INT, WEIGHTS_MXFP4 = 0, 1
 COMPUTE_FLOAT, COMPUTE_INT8_BLOCK = 0, 1
 GELU_ERF, GELU_TANH = 0, 1
-PATH_SIMT, PATH_DECODE, PATH_TC, PATH_TC_DECODE, PATH_INT8 = 0, 1, 2, 3, 4
+PATH_SIMT, PATH_DECODE, PATH_TC, PATH_TC_DECODE, PATH_INT8, PATH_INT8_TC = 0, 1, 2, 3, 4, 5
 
 # Every function the header declares (checked against include/qmoe.h by the tests).
 EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forward",
