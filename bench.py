@@ -542,37 +542,81 @@ def run_ours(args):
     if world > 1:
         dist.barrier(device_ids=[local])
 
-    # ---- end to end through the public call, host buffers, copies inside
+    # ---- end to end through the public call, host buffers, copies inside.
+    # As a serving loop does, two buffer slots and two copy streams let the
+    # copy engines bring step i+1's inputs in and take step i-1's result out
+    # while step i computes; every step's own copies lie inside the timed
+    # region, which runs from before the first input copy to after the last
+    # result copy. The same K steps with copies and compute in one stream
+    # give the serial figure reported beside it.
     x_h = torch.empty(b.x.shape, dtype=b.x.dtype, pin_memory=True).copy_(b.x.cpu())
     lg_h = torch.empty(b.lg.shape, dtype=b.lg.dtype, pin_memory=True).copy_(b.lg.cpu())
     sh_h = None if b.sh is None else torch.empty(b.sh.shape, dtype=b.sh.dtype, pin_memory=True).copy_(b.sh.cpu())
-    y_h = torch.empty(b.y.shape, dtype=b.y.dtype, pin_memory=True)
-    x_d, lg_d = torch.empty_like(b.x), torch.empty_like(b.lg)
-    sh_d = None if b.sh is None else torch.empty_like(b.sh)
+    y_h = [torch.empty(b.y.shape, dtype=b.y.dtype, pin_memory=True) for _ in range(2)]
+    x_d = [torch.empty_like(b.x) for _ in range(2)]
+    lg_d = [torch.empty_like(b.lg) for _ in range(2)]
+    sh_d = [None if b.sh is None else torch.empty_like(b.sh) for _ in range(2)]
+    y_d = [b.y, torch.empty_like(b.y)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
 
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        lg_d.copy_(lg_h, non_blocking=True)
-        if sh_d is not None:
-            sh_d.copy_(sh_h, non_blocking=True)
-        qmoe.qmoe_forward(h, T, x_d, lg_d, sh_d, b.y, b.ws, b.nws, stream)
-        y_h.copy_(b.y, non_blocking=True)
+    def e2e_step(i):
+        k = i % 2
+        with torch.cuda.stream(s_in):
+            if used[k]:
+                s_in.wait_event(ev_comp[k])  # the slot's previous forward has read its inputs
+            x_d[k].copy_(x_h, non_blocking=True)
+            lg_d[k].copy_(lg_h, non_blocking=True)
+            if sh_d[k] is not None:
+                sh_d[k].copy_(sh_h, non_blocking=True)
+            ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
+        if used[k]:
+            stream.wait_event(ev_out[k])  # the slot's previous result has left the device
+        qmoe.qmoe_forward(h, T, x_d[k], lg_d[k], sh_d[k], y_d[k], b.ws, b.nws, stream)
+        ev_comp[k].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[k])
+            y_h[k].copy_(y_d[k], non_blocking=True)
+            ev_out[k].record(s_out)
+        used[k] = True
 
-    for _ in range(3):
-        e2e_step()
+    def serial_step():
+        with torch.cuda.stream(stream):
+            x_d[0].copy_(x_h, non_blocking=True)
+            lg_d[0].copy_(lg_h, non_blocking=True)
+            if sh_d[0] is not None:
+                sh_d[0].copy_(sh_h, non_blocking=True)
+            qmoe.qmoe_forward(h, T, x_d[0], lg_d[0], sh_d[0], y_d[0], b.ws, b.nws, stream)
+            y_h[0].copy_(y_d[0], non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier(device_ids=[local])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(K):
+        e2e_step(3 + i)
+    e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = replicas.max_over_ranks([e0.elapsed_time(e1)], dev)[0]
+    for _ in range(3):
+        serial_step()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        serial_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    serial_ms = replicas.max_over_ranks([e0.elapsed_time(e1)], dev)[0]
     h2d = x_h.numel() * x_h.element_size() + lg_h.numel() * lg_h.element_size() + (
         0 if sh_h is None else sh_h.numel() * sh_h.element_size())
-    d2h = y_h.numel() * y_h.element_size()
+    d2h = y_h[0].numel() * y_h[0].element_size()
 
     if world > 1:
         dist.destroy_process_group()
@@ -631,7 +675,10 @@ def run_ours(args):
             "crossover": cross,
             "cpu_baseline": cpu,
             "e2e": {"value": replicas.job_tokens_per_s(T, world, K, e2e_ms), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "copies": "pinned host buffers; input and result copies of neighbouring steps "
+                              "overlap the forward on separate copy streams (two buffer slots)",
+                    "serial_value": replicas.job_tokens_per_s(T, world, K, serial_ms)},
             "gpu_launches": b.launches * K,
             "clocks": clk}
     print(json.dumps(line), flush=True)
