@@ -288,8 +288,9 @@ QMOE_API qmoe_status qmoe_debug_hidden(const qmoe_handle* h, int64_t T, const vo
 
 /*
  * qmoe_read_device_status -- wait for `stream`, then read the device-side
- * status word of `workspace` (QMOE_OK or QMOE_TIMEOUT when a bounded device
- * wait gave up in the last forward that used it).
+ * status word of `workspace` (QMOE_OK, QMOE_TIMEOUT when a bounded device
+ * wait gave up in the last forward that used it, or QMOE_INVALID_ARGUMENT
+ * when qmoe_ep_expert_rows met an expert id outside its handle's range).
  */
 QMOE_API qmoe_status qmoe_read_device_status(const qmoe_handle* h, const void* workspace, void* stream);
 
@@ -330,6 +331,61 @@ QMOE_API size_t qmoe_noalloc_scratch_bytes(void);
  * on the current device. (No counterpart on the pages.)
  */
 QMOE_API qmoe_status qmoe_noalloc_read_device_status(const qmoe_handle* h, void* stream);
+
+/*
+ * Expert parallel: the forward split at its two exchange points, for experts
+ * spread over ranks (each rank holds a contiguous range of experts in its own
+ * handle, every rank routes its own tokens). The pages fix no parallelism;
+ * the steps are those of qmoe_forward ("ClikaRT::nn::QMoEWoQ", forward();
+ * the "MoE" page's routed combine) with the rows moved between ranks by the
+ * caller (an all-to-all) after dispatch and again after the expert rows.
+ *
+ * qmoe_ep_dispatch -- on the token owner, with a handle of the full expert
+ * set (weights need not be bound: only the routing attributes and the score
+ * correction bias are used): route T tokens, sort their T*k routes by expert
+ * (stable, token order inside an expert) and write
+ *   rows       [T*k, H] act_dtype  x's row of every route, in that order
+ *                                  (scaled by the router weight and rounded
+ *                                  to act_dtype with apply_router_weight_on_input)
+ *   row_expert [T*k] int32         the global expert id of each row
+ *   offsets    [E+1] int32         rows of expert e are offsets[e] .. offsets[e+1]
+ *   state      qmoe_ep_state_bytes(h, T) bytes: the routing, for qmoe_ep_combine
+ * All DEVICE pointers; x and rows 16-byte aligned, state 256-byte aligned.
+ * The rows destined to one rank are one contiguous range (its experts'
+ * offsets). Enqueued on `stream`; T = 0 is a no-op.
+ */
+QMOE_API size_t qmoe_ep_state_bytes(const qmoe_handle* h, int64_t T);
+QMOE_API qmoe_status qmoe_ep_dispatch(const qmoe_handle* h, int64_t T, const void* x, const void* router_logits,
+                                      void* rows, int32_t* row_expert, int32_t* offsets, void* state,
+                                      size_t state_bytes, void* stream);
+
+/*
+ * qmoe_ep_expert_rows -- on the expert owner, with a handle holding experts
+ * expert_base .. expert_base + E_h - 1 (its num_experts = E_h, weights
+ * bound): for R rows of any order, out[r] [H] fp32 = FC2(act(FC1(rows[r])))
+ * + fc2 bias of expert row_expert[r] - expert_base (no router weight, no
+ * scaling factor: the token owner's combine applies them). The handle's
+ * routing attributes (k, normalisation, scaling, router weight on input) are
+ * not used. rows [R, H] act_dtype and out 16-byte aligned; workspace of
+ * qmoe_ep_rows_workspace_size(h, R) bytes, 256-byte aligned. An id outside
+ * the handle's range is not an index: the row is computed as expert 0 and
+ * the workspace status word reads QMOE_INVALID_ARGUMENT
+ * (qmoe_read_device_status). R = 0 is a no-op.
+ */
+QMOE_API size_t qmoe_ep_rows_workspace_size(const qmoe_handle* h, int64_t R);
+QMOE_API qmoe_status qmoe_ep_expert_rows(const qmoe_handle* h, int64_t R, const void* rows,
+                                         const int32_t* row_expert, int32_t expert_base, float* out,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qmoe_ep_combine -- on the token owner, after the expert outputs came back
+ * in dispatch order: y[t] = s * sum_j w[t, j] * expert_out[row of (t, j)] +
+ * shared_output[t], rounded once to act_dtype (s = routed_scaling_factor x
+ * expert_output_scale; w = 1 with apply_router_weight_on_input). expert_out
+ * [T*k, H] fp32, the state of the matching qmoe_ep_dispatch; same handle.
+ */
+QMOE_API qmoe_status qmoe_ep_combine(const qmoe_handle* h, int64_t T, const float* expert_out, const void* state,
+                                     const void* shared_output, void* y, void* stream);
 
 /* qmoe_destroy -- "ClikaRT::nn::QMoEWoQ", ~QMoEWoQ(): release the packed
  * weights and the handle. NULL is a no-op. */

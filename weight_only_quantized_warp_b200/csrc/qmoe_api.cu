@@ -21,11 +21,11 @@ static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Resident warps per SM assumed when sizing the FC2 split-K.
 static constexpr int64_t kSms = 148;
 
-Plan make_plan(const qmoe_handle& h, int64_t T) {
+Plan make_plan(const qmoe_handle& h, int64_t T, bool rows_mode) {
     const qmoe_config& c = h.cfg;
     Plan p;
     p.T = T;
-    p.R = T * c.k;
+    p.R = rows_mode ? T : T * c.k;
     const bool bf16 = c.act_dtype == QMOE_DTYPE_BF16;
     const int64_t E = c.num_experts, H = c.hidden_size, I = c.inter_size;
     const int bits = c.expert_weight_bits, bs = c.block_size;
@@ -121,7 +121,8 @@ Plan make_plan(const qmoe_handle& h, int64_t T) {
     p.fused_route = T <= kFusedRouteTokens;
     // the row gather runs on the tensor-core paths, and on every path when
     // the router weights scale the expert inputs
-    p.gather = p.path == kPathTc || p.path == kPathTcDecode || p.path == kPathI8Tc || c.apply_router_weight_on_input;
+    p.gather = p.path == kPathTc || p.path == kPathTcDecode || p.path == kPathI8Tc ||
+               (!rows_mode && c.apply_router_weight_on_input);
     // the int8 tier adds the rounding of FC1's input rows and of h
     const bool i8 = p.path == kPathI8 || p.path == kPathI8Tc;
     p.launches = (p.fused_route ? 1 : 2) + (p.gather ? 1 : 0) + 3 + (i8 ? 2 : 0);
@@ -507,6 +508,117 @@ int32_t qmoe_token_tile_for(const qmoe_handle* h, int64_t T) {
 
 }  // extern "C"
 
+// FC1 (+ activation) and FC2 of the routed rows: the row gather where the
+// plan wants it, the int8 tier's rounding launches, then the two expert
+// layers into the workspace (h, and FC2's fp32 split partials). Shared by
+// the whole forward and the expert-parallel rows entry.
+template <class Mark>
+static cudaError_t ffn_layers(const qmoe_handle* h, const Plan& p, const void* x, int32_t* perm, int32_t* inv,
+                              float* tw, int k, bool weighted_rows, char* ws, int32_t* status, cudaStream_t st,
+                              Mark& mark, const char** where) {
+    const qmoe_config& c = h->cfg;
+    const int E = int(c.num_experts);
+    const int bf16 = c.act_dtype == QMOE_DTYPE_BF16;
+    int32_t* offsets = (int32_t*)(ws + p.off_offsets);
+    void* hid = ws + p.off_h;
+    float* o = (float*)(ws + p.off_o);
+    cudaError_t err;
+    FfnArgs f1{};
+    f1.W = h->w1;
+    f1.S = h->s1;
+    f1.bias = h->b1;
+    f1.act = x;
+    f1.rowmap = perm;
+    f1.offsets = offsets;
+    f1.out = hid;
+    f1.N = h->n1;
+    f1.K = c.hidden_size;
+    f1.R = p.R;
+    f1.E = E;
+    f1.bits = c.expert_weight_bits;
+    f1.block_size = c.block_size;
+    f1.gated = h->gated;
+    f1.is_fc1 = 1;
+    f1.act_type = (c.activation_type == QMOE_ACT_GELU && c.gelu_mode == QMOE_GELU_TANH) ? kActGeluTanh
+                                                                                       : c.activation_type;
+    f1.alpha = resolved_alpha(c.activation_alpha);
+    f1.beta = c.activation_beta;
+    f1.limit = resolved_limit(c.swiglu_limit);
+    f1.splits = 1;
+    f1.scale_bf16 = c.scale_dtype != QMOE_DTYPE_F32;
+    f1.fp4 = c.weight_format == QMOE_WEIGHTS_MXFP4;
+    f1.act_bf16 = bf16;
+    f1.nt = p.nt;
+    f1.timeout_ns = h->wait_limit_ns;
+    f1.withhold = h->withhold;
+    // the weight-streaming kernels prefetch their first weights while the
+    // kernel before them finishes (routing / gather before FC1, FC1 before FC2)
+    f1.pdl = h->pdl && p.path == kPathDecode;
+    FfnArgs f2 = f1;
+    f2.W = h->w2;
+    f2.S = h->s2;
+    f2.bias = nullptr;
+    f2.act = hid;
+    f2.rowmap = nullptr;
+    f2.out = o;
+    f2.N = c.hidden_size;
+    f2.K = c.inter_size;
+    f2.gated = 0;
+    f2.is_fc1 = 0;
+    f2.splits = p.fc2_splits;
+    if (p.gather) {
+        if ((err = mark()) != cudaSuccess) { *where = "event"; return err; }
+        void* xp = ws + p.off_xperm;
+        err = weighted_rows
+                  ? launch_gather_rows_weighted(x, perm, inv, tw, k, xp, p.R, c.hidden_size, bf16, st)
+                  : launch_gather_rows(x, perm, xp, p.R, c.hidden_size * 2, st);
+        if (err != cudaSuccess) { *where = "gather"; return err; }
+        f1.act = xp;
+        f1.rowmap = nullptr;  // rows already in segment order
+    }
+    if (p.path == kPathI8 || p.path == kPathI8Tc) {
+        // FC1's input rows (x by token, or the gathered rows) to int8 codes,
+        // in the order the chosen kernel reads them
+        const bool tc = p.path == kPathI8Tc;
+        const int perm = tc ? (c.expert_weight_bits == 4 ? 2 : 3) : (c.expert_weight_bits == 4 ? 1 : 0);
+        int8_t* xq = (int8_t*)(ws + p.off_xq);
+        float* xs = (float*)(ws + p.off_xs);
+        if ((err = mark()) != cudaSuccess) { *where = "event"; return err; }
+        if ((err = launch_quantize_i8(f1.act, bf16, p.xq_rows, c.hidden_size, c.block_size, perm, xq, xs, st)) !=
+            cudaSuccess)
+            { *where = "quantize x"; return err; }
+        f1.aq = xq;
+        f1.as = xs;
+        if ((err = mark()) != cudaSuccess) { *where = "event"; return err; }
+        if ((err = tc ? launch_ffn_tc_i8(f1, p.bn, status, st) : launch_ffn_i8(f1, st)) != cudaSuccess)
+            { *where = "fc1"; return err; }
+        int8_t* hq = (int8_t*)(ws + p.off_hq);
+        float* hs = (float*)(ws + p.off_hs);
+        if ((err = mark()) != cudaSuccess) { *where = "event"; return err; }
+        if ((err = launch_quantize_i8(hid, bf16, p.R, c.inter_size, c.block_size, perm, hq, hs, st)) != cudaSuccess)
+            { *where = "quantize h"; return err; }
+        f2.aq = hq;
+        f2.as = hs;
+        if ((err = mark()) != cudaSuccess) { *where = "event"; return err; }
+        if ((err = tc ? launch_ffn_tc_i8(f2, p.bn, status, st) : launch_ffn_i8(f2, st)) != cudaSuccess)
+            { *where = "fc2"; return err; }
+    } else {
+        if ((err = mark()) != cudaSuccess) { *where = "event"; return err; }
+        err = p.path == kPathSimt        ? launch_ffn_simt(f1, st)
+              : p.path == kPathTc        ? launch_ffn_tc(f1, p.bn, status, st)
+              : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f1, p.bn, status, st)
+                                         : launch_ffn_decode(f1, st);
+        if (err != cudaSuccess) { *where = "fc1"; return err; }
+        if ((err = mark()) != cudaSuccess) { *where = "event"; return err; }
+        err = p.path == kPathSimt        ? launch_ffn_simt(f2, st)
+              : p.path == kPathTc        ? launch_ffn_tc(f2, p.bn, status, st)
+              : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f2, p.bn, status, st)
+                                         : launch_ffn_decode(f2, st);
+        if (err != cudaSuccess) { *where = "fc2"; return err; }
+    }
+    return cudaSuccess;
+}
+
 static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
                                 const void* router_logits, const void* shared_output, void* y,
                                 void* workspace, size_t workspace_bytes, void* stream,
@@ -576,99 +688,10 @@ static qmoe_status forward_impl(const qmoe_handle* h, int64_t T, const void* x,
             return cuda_fail(h, err, "permute");
     }
 
-    FfnArgs f1{};
-    f1.W = h->w1;
-    f1.S = h->s1;
-    f1.bias = h->b1;
-    f1.act = x;
-    f1.rowmap = perm;
-    f1.offsets = offsets;
-    f1.out = hid;
-    f1.N = h->n1;
-    f1.K = c.hidden_size;
-    f1.R = p.R;
-    f1.E = E;
-    f1.bits = c.expert_weight_bits;
-    f1.block_size = c.block_size;
-    f1.gated = h->gated;
-    f1.is_fc1 = 1;
-    f1.act_type = (c.activation_type == QMOE_ACT_GELU && c.gelu_mode == QMOE_GELU_TANH) ? kActGeluTanh
-                                                                                       : c.activation_type;
-    f1.alpha = resolved_alpha(c.activation_alpha);
-    f1.beta = c.activation_beta;
-    f1.limit = resolved_limit(c.swiglu_limit);
-    f1.splits = 1;
-    f1.scale_bf16 = c.scale_dtype != QMOE_DTYPE_F32;
-    f1.fp4 = c.weight_format == QMOE_WEIGHTS_MXFP4;
-    f1.act_bf16 = bf16;
-    f1.nt = p.nt;
-    f1.timeout_ns = h->wait_limit_ns;
-    f1.withhold = h->withhold;
-    // the weight-streaming kernels prefetch their first weights while the
-    // kernel before them finishes (routing / gather before FC1, FC1 before FC2)
-    f1.pdl = h->pdl && p.path == kPathDecode;
-    FfnArgs f2 = f1;
-    f2.W = h->w2;
-    f2.S = h->s2;
-    f2.bias = nullptr;
-    f2.act = hid;
-    f2.rowmap = nullptr;
-    f2.out = o;
-    f2.N = c.hidden_size;
-    f2.K = c.inter_size;
-    f2.gated = 0;
-    f2.is_fc1 = 0;
-    f2.splits = p.fc2_splits;
-    if (p.gather) {
-        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        void* xp = ws + p.off_xperm;
-        err = c.apply_router_weight_on_input
-                  ? launch_gather_rows_weighted(x, perm, inv, tw, k, xp, p.R, c.hidden_size, bf16, st)
-                  : launch_gather_rows(x, perm, xp, p.R, c.hidden_size * 2, st);
-        if (err != cudaSuccess) return cuda_fail(h, err, "gather");
-        f1.act = xp;
-        f1.rowmap = nullptr;  // rows already in segment order
-    }
-    if (p.path == kPathI8 || p.path == kPathI8Tc) {
-        // FC1's input rows (x by token, or the gathered rows) to int8 codes,
-        // in the order the chosen kernel reads them
-        const bool tc = p.path == kPathI8Tc;
-        const int perm = tc ? (c.expert_weight_bits == 4 ? 2 : 3) : (c.expert_weight_bits == 4 ? 1 : 0);
-        int8_t* xq = (int8_t*)(ws + p.off_xq);
-        float* xs = (float*)(ws + p.off_xs);
-        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        if ((err = launch_quantize_i8(f1.act, bf16, p.xq_rows, c.hidden_size, c.block_size, perm, xq, xs, st)) !=
-            cudaSuccess)
-            return cuda_fail(h, err, "quantize x");
-        f1.aq = xq;
-        f1.as = xs;
-        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        if ((err = tc ? launch_ffn_tc_i8(f1, p.bn, status, st) : launch_ffn_i8(f1, st)) != cudaSuccess)
-            return cuda_fail(h, err, "fc1");
-        int8_t* hq = (int8_t*)(ws + p.off_hq);
-        float* hs = (float*)(ws + p.off_hs);
-        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        if ((err = launch_quantize_i8(hid, bf16, p.R, c.inter_size, c.block_size, perm, hq, hs, st)) != cudaSuccess)
-            return cuda_fail(h, err, "quantize h");
-        f2.aq = hq;
-        f2.as = hs;
-        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        if ((err = tc ? launch_ffn_tc_i8(f2, p.bn, status, st) : launch_ffn_i8(f2, st)) != cudaSuccess)
-            return cuda_fail(h, err, "fc2");
-    } else {
-        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        err = p.path == kPathSimt        ? launch_ffn_simt(f1, st)
-              : p.path == kPathTc        ? launch_ffn_tc(f1, p.bn, status, st)
-              : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f1, p.bn, status, st)
-                                         : launch_ffn_decode(f1, st);
-        if (err != cudaSuccess) return cuda_fail(h, err, "fc1");
-        if ((err = mark()) != cudaSuccess) return cuda_fail(h, err, "event");
-        err = p.path == kPathSimt        ? launch_ffn_simt(f2, st)
-              : p.path == kPathTc        ? launch_ffn_tc(f2, p.bn, status, st)
-              : p.path == kPathTcDecode  ? launch_ffn_tc_decode(f2, p.bn, status, st)
-                                         : launch_ffn_decode(f2, st);
-        if (err != cudaSuccess) return cuda_fail(h, err, "fc2");
-    }
+    const char* where = "";
+    if ((err = ffn_layers(h, p, x, perm, inv, tw, k, c.apply_router_weight_on_input != 0, ws, status, st, mark,
+                          &where)) != cudaSuccess)
+        return cuda_fail(h, err, where);
     CombineArgs ca{};
     ca.o = o;
     ca.topk_idx = idx;
@@ -769,7 +792,203 @@ qmoe_status qmoe_read_device_status(const qmoe_handle* h, const void* workspace,
                                       cudaMemcpyDeviceToHost, (cudaStream_t)stream);
     if (err == cudaSuccess) err = cudaStreamSynchronize((cudaStream_t)stream);
     if (err != cudaSuccess) return cuda_fail(h, err, "read_device_status");
-    return v == 0 ? QMOE_OK : QMOE_TIMEOUT;
+    return v == 0 ? QMOE_OK : (v == QMOE_INVALID_ARGUMENT ? QMOE_INVALID_ARGUMENT : QMOE_TIMEOUT);
+}
+
+// ---------------------------------------------------------------- expert parallel
+// The forward split at its two exchange points: routing, permutation and the
+// row gather on the rank that owns the tokens (dispatch); the expert layers on
+// the rank that owns the experts (rows); the weighted combine back on the
+// token owner (combine). The rows in between travel between ranks in the
+// dispatch order, which is expert order, so each destination rank's rows are
+// one contiguous range.
+
+}  // extern "C"
+
+namespace {
+
+struct EpState {  // routing of one dispatch, kept for its combine
+    size_t off_status, off_idx, off_w, off_inv, off_perm, off_offsets, total;
+};
+
+EpState ep_state(const qmoe_handle& h, int64_t T) {
+    const size_t R = size_t(T) * size_t(h.cfg.k);
+    EpState s;
+    size_t off = 0;
+    s.off_status = off;  off = align256(off + 16);
+    s.off_idx = off;     off = align256(off + R * 4);
+    s.off_w = off;       off = align256(off + R * 4);
+    s.off_inv = off;     off = align256(off + R * 4);
+    s.off_perm = off;    off = align256(off + R * 4);
+    s.off_offsets = off; off = align256(off + size_t(h.cfg.num_experts + 1) * 4);
+    s.total = off;
+    return s;
+}
+
+bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
+
+qmoe_status on_device(const qmoe_handle* h) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(h, QMOE_CUDA_ERROR, "no current device");
+    if (h->device >= 0 && dev != h->device)  // a routing handle without weights runs on any device
+        return fail(h, QMOE_INVALID_ARGUMENT, "current device %d is not the handle's device (%d)", dev, h->device);
+    return QMOE_OK;
+}
+
+float routed_multiplier(const qmoe_config& c) {
+    return (c.routed_scaling_factor > 0.0f ? c.routed_scaling_factor : 1.0f) *
+           (c.expert_output_scale > 0.0f ? c.expert_output_scale : 1.0f);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t qmoe_ep_state_bytes(const qmoe_handle* h, int64_t T) {
+    if (!h || T < 0) return 0;
+    return ep_state(*h, T).total;
+}
+
+size_t qmoe_ep_rows_workspace_size(const qmoe_handle* h, int64_t R) {
+    if (!h || R < 0) return 0;
+    return make_plan(*h, R, true).total;
+}
+
+qmoe_status qmoe_ep_dispatch(const qmoe_handle* h, int64_t T, const void* x, const void* router_logits,
+                             void* rows, int32_t* row_expert, int32_t* offsets, void* state, size_t state_bytes,
+                             void* stream) {
+    if (!h) return QMOE_INVALID_ARGUMENT;
+    if (T < 0) return fail(h, QMOE_INVALID_ARGUMENT, "T must be >= 0");
+    if (T == 0) return QMOE_OK;
+    const qmoe_config& c = h->cfg;
+    const int bf16 = c.act_dtype == QMOE_DTYPE_BF16;
+    if (!x || !router_logits || !rows || !row_expert || !offsets || !state)
+        return fail(h, QMOE_INVALID_ARGUMENT, "x, router_logits, rows, row_expert, offsets and state are required");
+    if (misaligned(x, 16) || misaligned(rows, 16) || misaligned(router_logits, bf16 ? 2 : 4) ||
+        misaligned(row_expert, 4) || misaligned(offsets, 4) || misaligned(state, 256))
+        return fail(h, QMOE_INVALID_ARGUMENT, "x and rows 16-byte, state 256-byte, the rest element aligned");
+    if (T * c.k >= (int64_t(1) << 31)) return fail(h, QMOE_UNSUPPORTED, "T * k must stay below 2^31");
+    const EpState es = ep_state(*h, T);
+    if (state_bytes < es.total)
+        return fail(h, QMOE_INVALID_ARGUMENT, "state too small: %zu < %zu", state_bytes, es.total);
+    if (qmoe_status s = on_device(h)) return s;
+    char* sb = (char*)state;
+    int32_t* status = (int32_t*)(sb + es.off_status);
+    int32_t* idx = (int32_t*)(sb + es.off_idx);
+    float* tw = (float*)(sb + es.off_w);
+    int32_t* inv = (int32_t*)(sb + es.off_inv);
+    int32_t* perm = (int32_t*)(sb + es.off_perm);
+    int32_t* offs = (int32_t*)(sb + es.off_offsets);
+    const int E = int(c.num_experts), k = int(c.k);
+    const int64_t R = T * k;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t err;
+    if (T <= kFusedRouteTokens)
+        err = launch_route_permute(router_logits, bf16, T, E, k, c.normalize_routing_weights, c.n_group,
+                                   c.topk_group, h->score_bias, idx, tw, offs, perm, inv, status, st);
+    else if ((err = launch_route(router_logits, bf16, T, E, k, c.normalize_routing_weights, c.n_group,
+                                 c.topk_group, h->score_bias, idx, tw, status, st)) == cudaSuccess)
+        err = launch_permute(idx, T, E, k, offs, perm, inv, st);
+    if (err != cudaSuccess) return cuda_fail(h, err, "ep route");
+    err = c.apply_router_weight_on_input
+              ? launch_gather_rows_weighted(x, perm, inv, tw, k, rows, R, c.hidden_size, bf16, st)
+              : launch_gather_rows(x, perm, rows, R, c.hidden_size * (bf16 ? 2 : 4), st);
+    if (err == cudaSuccess) err = launch_scatter_row_experts(idx, inv, R, row_expert, st);
+    if (err == cudaSuccess)
+        err = cudaMemcpyAsync(offsets, offs, size_t(E + 1) * 4, cudaMemcpyDeviceToDevice, st);
+    return err == cudaSuccess ? QMOE_OK : cuda_fail(h, err, "ep dispatch");
+}
+
+qmoe_status qmoe_ep_expert_rows(const qmoe_handle* h, int64_t R, const void* rows, const int32_t* row_expert,
+                                int32_t expert_base, float* out, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+    if (!h) return QMOE_INVALID_ARGUMENT;
+    if (R < 0) return fail(h, QMOE_INVALID_ARGUMENT, "R must be >= 0");
+    if (!h->bound) return fail(h, QMOE_NOT_BOUND, "expert rows before set_weights bound the weights");
+    if (R == 0) return QMOE_OK;
+    if (!rows || !row_expert || !out || !workspace)
+        return fail(h, QMOE_INVALID_ARGUMENT, "rows, row_expert, out and workspace are required");
+    if (misaligned(rows, 16) || misaligned(out, 16) || misaligned(row_expert, 4) || misaligned(workspace, 256))
+        return fail(h, QMOE_INVALID_ARGUMENT, "rows and out 16-byte, workspace 256-byte, row_expert 4-byte aligned");
+    if (R >= (int64_t(1) << 31)) return fail(h, QMOE_UNSUPPORTED, "R must stay below 2^31");
+    const Plan p = make_plan(*h, R, true);
+    if (!p.ok) return fail(h, QMOE_UNSUPPORTED, "no kernel configuration fits this shape (hidden_size too large)");
+    if (workspace_bytes < p.total)
+        return fail(h, QMOE_INVALID_ARGUMENT, "workspace too small: %zu < %zu", workspace_bytes, p.total);
+    if (qmoe_status s = on_device(h)) return s;
+    const qmoe_config& c = h->cfg;
+    const int E = int(c.num_experts);
+    cudaStream_t st = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    int32_t* status = (int32_t*)(ws + p.off_status);
+    int32_t* idx = (int32_t*)(ws + p.off_idx);
+    float* tw = (float*)(ws + p.off_w);
+    int32_t* inv = (int32_t*)(ws + p.off_inv);
+    int32_t* perm = (int32_t*)(ws + p.off_perm);
+    int32_t* offs = (int32_t*)(ws + p.off_offsets);
+    cudaError_t err = cudaMemsetAsync(status, 0, 4, st);
+    if (err == cudaSuccess) err = launch_rebase_experts(row_expert, R, expert_base, E, idx, status, st);
+    if (err == cudaSuccess) err = launch_permute(idx, R, E, 1, offs, perm, inv, st);
+    if (err != cudaSuccess) return cuda_fail(h, err, "ep rows permute");
+    auto mark = []() -> cudaError_t { return cudaSuccess; };
+    const char* where = "";
+    if ((err = ffn_layers(h, p, rows, perm, inv, tw, 1, false, ws, status, st, mark, &where)) != cudaSuccess)
+        return cuda_fail(h, err, where);
+    // each row's expert output o + b2 in fp32: the combine with one route per
+    // row, unit weight and no scaling (the token owner's combine applies them)
+    CombineArgs ca{};
+    ca.o = (const float*)(ws + p.off_o);
+    ca.topk_idx = idx;
+    ca.topk_w = tw;
+    ca.inv = inv;
+    ca.b2 = h->b2;
+    ca.shared = nullptr;
+    ca.y = out;
+    ca.T = R;
+    ca.H = c.hidden_size;
+    ca.R = p.R;
+    ca.k = 1;
+    ca.splits = p.fc2_splits;
+    ca.rsf = 1.0f;
+    ca.weights_on_input = 1;
+    ca.pdl = h->pdl;
+    ca.act_bf16 = 0;
+    if ((err = launch_combine(ca, st)) != cudaSuccess) return cuda_fail(h, err, "ep rows output");
+    return QMOE_OK;
+}
+
+qmoe_status qmoe_ep_combine(const qmoe_handle* h, int64_t T, const float* expert_out, const void* state,
+                            const void* shared_output, void* y, void* stream) {
+    if (!h) return QMOE_INVALID_ARGUMENT;
+    if (T < 0) return fail(h, QMOE_INVALID_ARGUMENT, "T must be >= 0");
+    if (T == 0) return QMOE_OK;
+    if (!expert_out || !state || !y)
+        return fail(h, QMOE_INVALID_ARGUMENT, "expert_out, state and y are required");
+    if (misaligned(expert_out, 16) || misaligned(y, 16) || misaligned(shared_output, 16) || misaligned(state, 256))
+        return fail(h, QMOE_INVALID_ARGUMENT, "expert_out, shared_output and y 16-byte, state 256-byte aligned");
+    if (qmoe_status s = on_device(h)) return s;
+    const qmoe_config& c = h->cfg;
+    const EpState es = ep_state(*h, T);
+    const char* sb = (const char*)state;
+    CombineArgs ca{};
+    ca.o = expert_out;
+    ca.topk_idx = (const int32_t*)(sb + es.off_idx);
+    ca.topk_w = (const float*)(sb + es.off_w);
+    ca.inv = (const int32_t*)(sb + es.off_inv);
+    ca.b2 = nullptr;  // added with each expert output on the rank that computed it
+    ca.shared = shared_output;
+    ca.y = y;
+    ca.T = T;
+    ca.H = c.hidden_size;
+    ca.R = T * c.k;
+    ca.k = int(c.k);
+    ca.splits = 1;
+    ca.rsf = routed_multiplier(c);
+    ca.weights_on_input = c.apply_router_weight_on_input;
+    ca.pdl = 0;
+    ca.act_bf16 = c.act_dtype == QMOE_DTYPE_BF16;
+    const cudaError_t err = launch_combine(ca, (cudaStream_t)stream);
+    return err == cudaSuccess ? QMOE_OK : cuda_fail(h, err, "ep combine");
 }
 
 }  // extern "C"

@@ -126,7 +126,9 @@ struct qmoe_handle {
 
 namespace qmoe {
 
-Plan make_plan(const qmoe_handle& h, int64_t T);
+// rows_mode: T pre-routed rows, one expert each (the expert-parallel rows
+// entry): R = T, and no router-weighted gather.
+Plan make_plan(const qmoe_handle& h, int64_t T, bool rows_mode = false);
 
 // ----------------------------------------------------------------- launchers
 // Each returns the cudaError_t of its launch.
@@ -170,6 +172,15 @@ cudaError_t launch_route_permute(const void* logits, int act_bf16, int64_t T, in
 cudaError_t prepare_route_permute();
 cudaError_t launch_permute(const int32_t* topk_idx, int64_t T, int E, int k, int32_t* offsets,
                            int32_t* perm_tok, int32_t* inv, cudaStream_t st);
+// Expert parallel: the expert of every segment-ordered row
+// (row_expert[inv[s]] = topk_idx[s]), and caller-given global expert ids
+// rebased to a handle's local ids (id - base); an id outside [0, E) becomes
+// expert 0 and sets QMOE_INVALID_ARGUMENT in the status word, so no later
+// kernel indexes out of range.
+cudaError_t launch_scatter_row_experts(const int32_t* topk_idx, const int32_t* inv, int64_t R, int32_t* row_expert,
+                                       cudaStream_t st);
+cudaError_t launch_rebase_experts(const int32_t* ids, int64_t R, int32_t base, int E, int32_t* local,
+                                  int32_t* status, cudaStream_t st);
 
 // Expert FFN layer over the segments (decode / SIMT paths).
 struct FfnArgs {

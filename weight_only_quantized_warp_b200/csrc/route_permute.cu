@@ -366,4 +366,39 @@ cudaError_t launch_permute(const int32_t* topk_idx, int64_t T, int E, int k, int
     return cudaGetLastError();
 }
 
+namespace {
+
+__global__ void scatter_row_experts_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ inv,
+                                           int64_t R, int32_t* __restrict__ row_expert) {
+    for (int64_t s = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; s < R; s += int64_t(gridDim.x) * blockDim.x)
+        row_expert[inv[s]] = topk_idx[s];
+}
+
+__global__ void rebase_experts_kernel(const int32_t* __restrict__ ids, int64_t R, int32_t base, int E,
+                                      int32_t* __restrict__ local, int32_t* status) {
+    for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < R; r += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t e = int64_t(ids[r]) - base;
+        const bool ok = e >= 0 && e < E;
+        local[r] = ok ? int32_t(e) : 0;
+        if (!ok) atomicExch(status, int32_t(QMOE_INVALID_ARGUMENT));
+    }
+}
+
+int blocks_for(int64_t n) { return int(std::min<int64_t>((n + 255) / 256, 148 * 8)); }
+
+}  // namespace
+
+cudaError_t launch_scatter_row_experts(const int32_t* topk_idx, const int32_t* inv, int64_t R, int32_t* row_expert,
+                                       cudaStream_t st) {
+    if (R <= 0) return cudaSuccess;
+    scatter_row_experts_kernel<<<blocks_for(R), 256, 0, st>>>(topk_idx, inv, R, row_expert);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rebase_experts(const int32_t* ids, int64_t R, int32_t base, int E, int32_t* local,
+                                  int32_t* status, cudaStream_t st) {
+    rebase_experts_kernel<<<std::max(1, blocks_for(R)), 256, 0, st>>>(ids, R, base, E, local, status);
+    return cudaGetLastError();
+}
+
 }  // namespace qmoe

@@ -41,7 +41,8 @@ EXPORTS = ("qmoe_create", "qmoe_set_weights", "qmoe_workspace_size", "qmoe_forwa
            "qmoe_token_tile_for",
            "qmoe_set_option", "qmoe_forward_noalloc", "qmoe_noalloc_scratch_bytes",
            "qmoe_noalloc_read_device_status", "qmoe_set_score_correction_bias",
-           "qmoe_quantize_act_i8")
+           "qmoe_quantize_act_i8", "qmoe_ep_state_bytes", "qmoe_ep_dispatch",
+           "qmoe_ep_rows_workspace_size", "qmoe_ep_expert_rows", "qmoe_ep_combine")
 QMOE_OPT_PATH, QMOE_OPT_WAIT_LIMIT_NS, QMOE_OPT_TEST_WITHHOLD, QMOE_OPT_PDL, QMOE_OPT_DECODE_TILES = 1, 2, 3, 4, 5
 
 
@@ -104,6 +105,16 @@ lib.qmoe_token_tile_for.restype = ctypes.c_int32
 lib.qmoe_token_tile_for.argtypes = [_vp, _i64]
 lib.qmoe_quantize_act_i8.restype = ctypes.c_int
 lib.qmoe_quantize_act_i8.argtypes = [_vp, ctypes.c_int32, _i64, _i64, ctypes.c_int32, _vp, _vp, _vp]
+lib.qmoe_ep_state_bytes.restype = _sz
+lib.qmoe_ep_state_bytes.argtypes = [_vp, _i64]
+lib.qmoe_ep_dispatch.restype = ctypes.c_int
+lib.qmoe_ep_dispatch.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.qmoe_ep_rows_workspace_size.restype = _sz
+lib.qmoe_ep_rows_workspace_size.argtypes = [_vp, _i64]
+lib.qmoe_ep_expert_rows.restype = ctypes.c_int
+lib.qmoe_ep_expert_rows.argtypes = [_vp, _i64, _vp, _vp, ctypes.c_int32, _vp, _vp, _sz, _vp]
+lib.qmoe_ep_combine.restype = ctypes.c_int
+lib.qmoe_ep_combine.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp]
 
 
 class QMoEError(RuntimeError):
@@ -253,6 +264,35 @@ def qmoe_quantize_act_i8(x, dtype: int, rows: int, K: int, block_size: int, q, s
     [rows, K] int8 and scales [rows, K / block_size] fp32 (device buffers)."""
     _check(lib.qmoe_quantize_act_i8(_ptr(x), dtype, rows, K, block_size, _ptr(q), _ptr(scales),
                                     _stream(stream)))
+
+
+def qmoe_ep_state_bytes(h, T: int) -> int:
+    return int(lib.qmoe_ep_state_bytes(h, T))
+
+
+def qmoe_ep_dispatch(h, T, x, router_logits, rows, row_expert, offsets, state, state_bytes, stream=None):
+    """Expert parallel, token owner: route, sort the routes by expert, gather
+    x's rows in that order (see include/qmoe.h)."""
+    _check(lib.qmoe_ep_dispatch(h, T, _ptr(x), _ptr(router_logits), _ptr(rows), _ptr(row_expert),
+                                _ptr(offsets), _ptr(state), state_bytes, _stream(stream)), h)
+
+
+def qmoe_ep_rows_workspace_size(h, R: int) -> int:
+    return int(lib.qmoe_ep_rows_workspace_size(h, R))
+
+
+def qmoe_ep_expert_rows(h, R, rows, row_expert, expert_base, out, workspace, workspace_bytes, stream=None):
+    """Expert parallel, expert owner: each row's expert output (o + fc2 bias,
+    fp32) for global expert ids expert_base .. expert_base + E_h - 1."""
+    _check(lib.qmoe_ep_expert_rows(h, R, _ptr(rows), _ptr(row_expert), int(expert_base), _ptr(out),
+                                   _ptr(workspace), workspace_bytes, _stream(stream)), h)
+
+
+def qmoe_ep_combine(h, T, expert_out, state, shared_output, y, stream=None):
+    """Expert parallel, token owner: the router-weighted combine of the expert
+    outputs that came back in dispatch order."""
+    _check(lib.qmoe_ep_combine(h, T, _ptr(expert_out), _ptr(state), _ptr(shared_output), _ptr(y),
+                               _stream(stream)), h)
 
 
 # ------------------------------------------------------------- torch plumbing
