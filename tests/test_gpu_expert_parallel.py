@@ -132,3 +132,49 @@ def test_out_of_range_expert_ids_set_the_status_word(cuda_device):
     lg[np.arange(16), ok_ids.cpu().numpy()] = 0.0
     ref = oracle.forward(dataclasses.replace(inp, cfg=c1, logits=gen._store(lg, cfg.act_dtype), shared=None))["y"]
     assert max_rel(good.cpu().numpy(), ref) <= TOL_BF16
+
+
+def _nccl_rank_main(rank, port, out_path):
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+
+    from weight_only_quantized_warp_b200 import expert_parallel as ep
+    from weight_only_quantized_warp_b200 import qmoe
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=timedelta(seconds=60), device_id=dev)
+    try:
+        cfg = _cfg(T=40, E=4, k=2)
+        inp = _rank_inputs(cfg, 91, 1)[0]
+        ops = ep.LibraryOps(cfg, inp, 1, 0, dev)
+        # the collectives forced on: NCCL all-to-alls of the counts, the bf16
+        # rows, the int32 expert ids and the fp32 outputs (one rank)
+        model = ep.ExpertParallelQMoE(ops, 1, 0, exchange=ep.torch_all_to_all(),
+                                      counts=lambda c: ep.exchange_counts(c, dev))
+        y = model(qmoe.to_device(inp.x, dev), qmoe.to_device(inp.logits, dev))
+        torch.cuda.synchronize()
+        np.save(out_path, to_numpy(y))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_nccl_all_to_all_path_on_one_rank(cuda_device, tmp_path):
+    import socket
+
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    out = str(tmp_path / "y.npy")
+    mp.start_processes(_nccl_rank_main, args=(port, out), nprocs=1, join=True, start_method="spawn")
+    cfg = _cfg(T=40, E=4, k=2)
+    inp = _rank_inputs(cfg, 91, 1)[0]
+    err = max_rel(np.load(out), oracle.forward(inp)["y"])
+    assert err <= TOL_BF16, f"y max rel err {err:.3e}"
