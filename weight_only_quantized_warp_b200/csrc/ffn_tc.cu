@@ -56,7 +56,7 @@ constexpr int kWarpMma = 17;
 constexpr int kWarpEpi0 = 18;
 constexpr int kEpiWarps = 8;
 constexpr int kWarpProd2 = kWarpEpi0 + kEpiWarps;          // second producer (weights)
-constexpr int kTcThreads = (kWarpProd2 + 1) * 32;           // 608
+constexpr int kTcThreads = (kWarpProd2 + 1) * 32;           // 864
 constexpr int kBK = 64;                                    // k per stage
 constexpr int kAStageCols = kBK / 2;                       // TMEM columns of one A tile
 constexpr int kScaleBytesMax = 4 * kTilesPerBlock * 16 * 4;  // 4 blocks of fp32 pairs

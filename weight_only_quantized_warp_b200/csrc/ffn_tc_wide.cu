@@ -36,8 +36,8 @@ constexpr int kWWarpProd = 16;
 constexpr int kWWarpMma = 17;
 constexpr int kWEpi0 = 18;
 constexpr int kWEpiWarps = 8;
-constexpr int kWWarpProd2 = kWEpi0 + kWEpiWarps;  // 18
-constexpr int kWThreads = (kWWarpProd2 + 1) * 32;  // 608
+constexpr int kWWarpProd2 = kWEpi0 + kWEpiWarps;  // 26
+constexpr int kWThreads = (kWWarpProd2 + 1) * 32;  // 864
 constexpr int kWScaleMax = 4 * kTilesPerBlock * 16 * 4;  // four blocks of fp32 pairs
 
 template <int BITS>
