@@ -402,37 +402,67 @@ __device__ __forceinline__ void tc_epilogue_item(const TcArgs& a, const Item& it
         const bool gate_lane = (lane & 8) == 0;
         const int64_t I = a.N / 2;
         __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(a.out) + p0 * I + (prow >> 4) * 8 + (row & 7);
+        // decided once per item (uniform over the warp): the scale/bias pass
+        // only where a scale or a bias exists, SwiGLU inline, its clamps only
+        // for a finite limit
+        const bool affine = PERCOL || a.bias != nullptr;
+        const bool swiglu = a.act_type == QMOE_ACT_SWIGLU;
+        const bool clamp = swiglu && a.limit < INFINITY;
+        const int ncols = valid ? it.rows : 0;  // columns this lane stores
+        const int coff = gate_lane ? 0 : 8;
         for (int c0 = c_first; c0 < ncol; c0 += c_step) {
             float v[16];
             tmem_ld16(tbase + uint32_t(c0), v);
+            if (empty_k) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = empty_k ? 0.0f : fmaf(v[j], s, bias);
+                for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+            } else if (affine) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = fmaf(v[j], s, bias);
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float recv = __shfl_xor_sync(0xffffffffu, gate_lane ? v[j + 8] : v[j], 8);
-                const float g = gate_lane ? v[j] : recv;
-                const float u = gate_lane ? recv : v[j + 8];
-                const int col = c0 + j + (gate_lane ? 0 : 8);
-                if (col < it.rows && valid)
-                    hout[int64_t(col) * I] =
-                        __float2bfloat16_rn(act_gated(a.act_type, g, u, a.alpha, a.beta, a.limit));
+                float g = gate_lane ? v[j] : recv;
+                float u = gate_lane ? recv : v[j + 8];
+                const int col = c0 + j + coff;
+                float hv;
+                if (swiglu) {
+                    if (clamp) {
+                        g = fminf(g, a.limit);
+                        u = fminf(fmaxf(u, -a.limit), a.limit);
+                    }
+                    hv = (u + a.beta) * g * sigmoidf_(a.alpha * g);
+                } else {
+                    hv = act_gated(a.act_type, g, u, a.alpha, a.beta, a.limit);
+                }
+                if (col < ncols) hout[int64_t(col) * I] = __float2bfloat16_rn(hv);
             }
         }
     } else {
+        const bool affine = PERCOL || a.bias != nullptr;
+        const int ncols = valid ? it.rows : 0;  // columns this lane stores
         for (int c0 = c_first; c0 < ncol; c0 += c_step) {
             float v[16];
             tmem_ld16(tbase + uint32_t(c0), v);
+            if (empty_k) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int col = c0 + j;
-                const float val = empty_k ? 0.0f : fmaf(v[j], s, bias);
-                if (col >= it.rows || !valid) continue;
-                const int64_t p = p0 + col;  // permuted row
-                if (a.is_fc1)
-                    reinterpret_cast<__nv_bfloat16*>(a.out)[p * a.N + prow] =
-                        __float2bfloat16_rn(act_plain(a.act_type, val));
-                else
-                    reinterpret_cast<float*>(a.out)[(int64_t(it.split) * a.R + p) * a.N + prow] = val;
+                for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+            } else if (affine) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = fmaf(v[j], s, bias);
+            }
+            if (a.is_fc1) {
+                __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + (p0 + c0) * a.N + prow;
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (c0 + j < ncols) o[int64_t(j) * a.N] = __float2bfloat16_rn(act_plain(a.act_type, v[j]));
+            } else {
+                // FC2: this split's fp32 partial of permuted rows p0 + c0 + j
+                float* o = reinterpret_cast<float*>(a.out) + (int64_t(it.split) * a.R + p0 + c0) * a.N + prow;
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (c0 + j < ncols) o[int64_t(j) * a.N] = v[j];
             }
         }
     }
