@@ -178,3 +178,25 @@ def test_nccl_all_to_all_path_on_one_rank(cuda_device, tmp_path):
     inp = _rank_inputs(cfg, 91, 1)[0]
     err = max_rel(np.load(out), oracle.forward(inp)["y"])
     assert err <= TOL_BF16, f"y max rel err {err:.3e}"
+
+
+@pytest.mark.parametrize("name", ["int4_bs64", "tensor_core_rows", "weights_on_input_shared_scaled", "int8_tier",
+                                  "f32_acts"])
+def test_one_rank_split_path_equals_the_fused_forward_bitwise(cuda_device, name):
+    """With one rank nothing is exchanged: the split calls run the same plan
+    and kernels as qmoe_forward, the expert outputs cross in fp32 and the
+    combine rounds once, so y matches the fused forward bit for bit."""
+    import torch
+    from weight_only_quantized_warp_b200 import expert_parallel as ep
+    from weight_only_quantized_warp_b200 import qmoe
+    cfg = _cfg(**CASES[name])
+    inp = _rank_inputs(cfg, 700 + list(CASES).index(name), 1)[0]
+    m = qmoe.QMoE(cfg, cuda_device)
+    m.set_weights_from(inp)
+    x, lg = qmoe.to_device(inp.x, cuda_device), qmoe.to_device(inp.logits, cuda_device)
+    sh = qmoe.to_device(inp.shared, cuda_device)
+    y_fused = m.forward(x, lg, sh)
+    y_split = ep.ExpertParallelQMoE(ep.LibraryOps(cfg, inp, 1, 0, cuda_device), 1, 0)(x, lg, sh)
+    torch.cuda.synchronize()
+    assert torch.equal(y_fused.view(torch.int16) if y_fused.dtype == torch.bfloat16 else y_fused,
+                       y_split.view(torch.int16) if y_split.dtype == torch.bfloat16 else y_split)
