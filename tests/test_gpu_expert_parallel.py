@@ -39,6 +39,8 @@ CASES = {
     "grouped_topk": dict(E=8, k=2, n_group=4, topk_group=2, normalize=False),
     "int8_tier": dict(compute_mode=gen.COMPUTE_INT8_BLOCK, block_size=128, T=48),
     "f32_acts": dict(act_dtype=gen.DT_F32, scale_dtype=gen.DT_F32, block_size=32),
+    "score_bias_fc3_bias": dict(has_score_bias=True, fusion=0, has_fc3=True, has_fc1_bias=True,
+                                has_fc3_bias=True),
 }
 
 
